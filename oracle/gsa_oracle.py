@@ -1,0 +1,503 @@
+"""CPU oracle for sparse global attention over N views (GSA) and dense global attention.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the package entry's ``smoke()``
+check and the ``cpu_baseline`` / ``--impl reference`` legs of the benchmark
+may import this module.  The CUDA library never calls it and shares no code
+with it; both are fed from the seeded generators in ``synthetic``.
+
+Everything is computed in float64 from the exact values of the bf16 inputs,
+step by step in the order the Speed3R pages give the method:
+
+  "Speed3R: Sparse Feed-forward 3D Reconstruction Models" (gist.science, ja
+  and it), technical summary, section 2.1 "Dual-branch attention mechanism"
+  (ja) / section 2 "Methodology" (it):
+    1. compression branch -- spatial down-sampling of the tokens (e.g. 4x4
+       average pooling), attention in the compressed space, the result
+       up-sampled back to the original resolution;
+    2. the compressed branch's scores (S_guide, it page) pick, for every
+       query, the Top-K most relevant token regions;
+    3. selection branch -- fine-grained attention over only the selected
+       key/value regions;
+    4. gated aggregation -- a learnable sigmoid gate computed from the query
+       mixes the two branch outputs;
+  plus the Speed3R-VGGT adaptation ("the selection branch always keeps the
+  reference-frame / camera-token information", section 2.2) and the dense
+  global attention the module replaces (section 1, "Background").
+
+Where the pages are silent, the readings used here are:
+  * queries, keys and values are all pooled in the compression branch; the
+    up-sampling is nearest (each fine token takes its block's output);
+  * special tokens are singleton entries of the compressed sequence (they
+    are not pooled), take part in compressed attention as queries and keys,
+    are not top-K candidates, and are always attended to by the selection
+    branch;
+  * the score ranked by top-K is the scaled logit (q_mean . k_mean) / sqrt(D);
+    selection is per head and per query block; ties go to the lower block id;
+    K_eff = min(K, number of patch blocks);
+  * a selected partial edge block contributes only its valid tokens;
+  * one softmax scale 1/sqrt(D) for every attention;
+  * the gate is g = sigmoid(q_mean . w_h) per (query block, head); g weights
+    the compression branch and (1 - g) the selection branch.
+
+Inputs are torch tensors (bf16 or fp32, CPU) or NumPy arrays of shape
+[T, H, D]; they are read in slices and converted exactly to float64, so the
+full-size workloads never need a float64 copy of the whole tensor.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+import torch
+
+
+# ----------------------------------------------------------------------------
+# token geometry
+
+
+@dataclasses.dataclass(frozen=True)
+class Geometry:
+    """Sizes of one layer call.
+
+    Frame f holds ``S`` special tokens then ``Hp*Wp`` patch tokens (row-major).
+    Pooling with factor ``P`` cuts each frame's patch grid into
+    ``Bh x Bw`` blocks (``Bh = ceil(Hp/P)``); a block at the right or bottom
+    edge holds only the patches that exist.  The compressed sequence has, per
+    frame, the ``S`` specials followed by the ``Bh*Bw`` blocks (row-major), so
+    entry ``a`` of frame f is ``f*E + j`` with ``E = S + Bh*Bw``.  Patch block
+    ``beta`` (a top-K candidate id) of frame f, grid position (br, bc), is
+    ``f*Bh*Bw + br*Bw + bc``.
+    """
+
+    N: int
+    S: int
+    Hp: int
+    Wp: int
+    H: int
+    D: int
+    P: int
+    K: int
+    scale: float | None = None
+
+    @property
+    def L(self) -> int:
+        return self.S + self.Hp * self.Wp
+
+    @property
+    def T(self) -> int:
+        return self.N * self.L
+
+    @property
+    def Bh(self) -> int:
+        return -(-self.Hp // self.P)
+
+    @property
+    def Bw(self) -> int:
+        return -(-self.Wp // self.P)
+
+    @property
+    def Bf(self) -> int:
+        return self.Bh * self.Bw
+
+    @property
+    def E(self) -> int:
+        return self.S + self.Bf
+
+    @property
+    def Tc(self) -> int:
+        return self.N * self.E
+
+    @property
+    def NB(self) -> int:
+        return self.N * self.Bf
+
+    @property
+    def K_eff(self) -> int:
+        return min(self.K, self.NB)
+
+    @property
+    def sm_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D) if self.scale is None else float(self.scale)
+
+    @property
+    def NS(self) -> int:
+        return self.N * self.S
+
+    # --- index maps -------------------------------------------------------
+
+    def special_token(self, f: int, j: int) -> int:
+        return f * self.L + j
+
+    def patch_token(self, f: int, r: int, c: int) -> int:
+        return f * self.L + self.S + r * self.Wp + c
+
+    def block_rows_cols(self, br: int, bc: int) -> tuple[range, range]:
+        return (range(self.P * br, min(self.P * br + self.P, self.Hp)),
+                range(self.P * bc, min(self.P * bc + self.P, self.Wp)))
+
+    def block_tokens(self, beta: int) -> np.ndarray:
+        """Valid token ids of patch block ``beta``."""
+        f, j = divmod(int(beta), self.Bf)
+        br, bc = divmod(j, self.Bw)
+        rows, cols = self.block_rows_cols(br, bc)
+        return np.array([self.patch_token(f, r, c) for r in rows for c in cols], dtype=np.int64)
+
+    def entry_of_block(self, beta: int) -> int:
+        f, j = divmod(int(beta), self.Bf)
+        return f * self.E + self.S + j
+
+    def entry_of_token(self, t: int) -> int:
+        f, i = divmod(int(t), self.L)
+        if i < self.S:
+            return f * self.E + i
+        r, c = divmod(i - self.S, self.Wp)
+        return f * self.E + self.S + (r // self.P) * self.Bw + (c // self.P)
+
+    def tokens_of_entry(self, a: int) -> np.ndarray:
+        f, j = divmod(int(a), self.E)
+        if j < self.S:
+            return np.array([self.special_token(f, j)], dtype=np.int64)
+        return self.block_tokens(f * self.Bf + (j - self.S))
+
+    def special_tokens(self) -> np.ndarray:
+        return np.array([self.special_token(f, j) for f in range(self.N) for j in range(self.S)],
+                        dtype=np.int64)
+
+    def patch_block_entries(self) -> np.ndarray:
+        """Compressed-sequence index of every patch block, in block-id order."""
+        return np.array([self.entry_of_block(b) for b in range(self.NB)], dtype=np.int64)
+
+
+def geometry_of(workload, **overrides) -> Geometry:
+    """Geometry of a ``synthetic.Workload`` (fields copied by name)."""
+    g = Geometry(N=workload.n_frames, S=workload.n_special, Hp=workload.hp, Wp=workload.wp,
+                 H=workload.n_heads, D=workload.head_dim, P=workload.pool, K=workload.top_k)
+    return dataclasses.replace(g, **overrides) if overrides else g
+
+
+# ----------------------------------------------------------------------------
+# exact float64 views of the inputs
+
+
+def f64(x, rows=None) -> np.ndarray:
+    """Exact float64 copy of ``x`` or of ``x[rows]`` (bf16/fp32 -> fp64 is exact)."""
+    if isinstance(x, torch.Tensor):
+        if rows is None:
+            t = x
+        elif isinstance(rows, slice):
+            t = x[rows]
+        else:
+            t = x[torch.as_tensor(np.asarray(rows), dtype=torch.long)]
+        return t.to(torch.float64).numpy()
+    a = np.asarray(x)
+    return (a if rows is None else a[rows]).astype(np.float64)
+
+
+def f64_head(x, rows, h: int) -> np.ndarray:
+    """Exact float64 copy of ``x[rows, h]``: [len(rows), D]."""
+    if isinstance(x, torch.Tensor):
+        return x[torch.as_tensor(np.asarray(rows), dtype=torch.long), h].to(torch.float64).numpy()
+    return np.asarray(x)[np.asarray(rows), h].astype(np.float64)
+
+
+def softmax(z: np.ndarray, axis: int = -1) -> np.ndarray:
+    """Textbook softmax, shifted by the maximum for range (exact in real arithmetic)."""
+    m = np.max(z, axis=axis, keepdims=True)
+    e = np.exp(z - m)
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+# ----------------------------------------------------------------------------
+# step 1: compression by spatial average pooling
+
+
+def pool(geo: Geometry, X, frames_per_chunk: int = 32) -> np.ndarray:
+    """Compressed sequence of X: [Tc, H, D] float64.
+
+    Speed3R, technical summary 2.1, compression branch: the tokens are
+    down-sampled spatially, e.g. by 4x4 average pooling, into a coarse
+    context.  Each patch block's entry is the arithmetic mean over the
+    patches the block actually holds (fewer than P*P at the right/bottom
+    edges); each special token is copied as its own entry.
+    """
+    out = np.empty((geo.Tc, geo.H, geo.D), dtype=np.float64)
+    for f0 in range(0, geo.N, frames_per_chunk):
+        f1 = min(geo.N, f0 + frames_per_chunk)
+        x = f64(X, slice(f0 * geo.L, f1 * geo.L)).reshape(f1 - f0, geo.L, geo.H, geo.D)
+        spec = x[:, :geo.S]
+        grid = x[:, geo.S:].reshape(f1 - f0, geo.Hp, geo.Wp, geo.H, geo.D)
+        ent = out[f0 * geo.E:f1 * geo.E].reshape(f1 - f0, geo.E, geo.H, geo.D)
+        ent[:, :geo.S] = spec
+        for br in range(geo.Bh):
+            for bc in range(geo.Bw):
+                rows, cols = geo.block_rows_cols(br, bc)
+                cell = grid[:, rows.start:rows.stop, cols.start:cols.stop]
+                ent[:, geo.S + br * geo.Bw + bc] = cell.sum(axis=(1, 2)) / (len(rows) * len(cols))
+    return out
+
+
+# ----------------------------------------------------------------------------
+# step 2: attention in the compressed space; step 3: S_guide; step 4: top-K
+
+
+def heads_first(x: np.ndarray) -> np.ndarray:
+    """[n, H, D] -> contiguous [H, n, D] (so per-head products are plain matmuls)."""
+    return np.ascontiguousarray(np.asarray(x).transpose(1, 0, 2))
+
+
+def qk_logits(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
+    """(q . k) * scale for every query row and key row, per head: [rows, H, keys]."""
+    s = np.matmul(heads_first(q), heads_first(k).transpose(0, 2, 1)) * scale  # [H, rows, keys]
+    return s.transpose(1, 0, 2)
+
+
+def weighted_values(p: np.ndarray, v: np.ndarray) -> np.ndarray:
+    """sum_j p[r, h, j] v[j, h, :]: [rows, H, D]."""
+    o = np.matmul(heads_first(p), heads_first(v))  # [H, rows, D]
+    return o.transpose(1, 0, 2)
+
+
+def compressed_logits(geo: Geometry, Qc_rows: np.ndarray, Kc: np.ndarray) -> np.ndarray:
+    """Scaled logits of compressed queries against every compressed key: [rows, H, Tc]."""
+    return qk_logits(Qc_rows, Kc, geo.sm_scale)
+
+
+def compressed_attention(geo: Geometry, Qc_rows: np.ndarray, Kc: np.ndarray, Vc: np.ndarray):
+    """O_cmp for the given compressed queries, and their logits.
+
+    Speed3R, technical summary 2.1: attention computed in the compressed
+    space (every compressed entry, specials included, is a key).
+    Returns (O [rows, H, D], logits [rows, H, Tc]).
+    """
+    s = compressed_logits(geo, Qc_rows, Kc)
+    p = softmax(s, axis=-1)
+    return weighted_values(p, Vc), s
+
+
+def guide_scores(geo: Geometry, logits: np.ndarray) -> np.ndarray:
+    """S_guide: the compressed logits restricted to patch-block keys, [rows, H, NB].
+
+    Speed3R (it), technical summary 2, compression branch: the branch
+    produces a score matrix S_guide that identifies the most relevant regions.
+    Column beta is patch block beta; special entries are not candidates.
+    """
+    return logits[..., geo.patch_block_entries()]
+
+
+def top_k_blocks(geo: Geometry, guide: np.ndarray) -> np.ndarray:
+    """Top-K patch blocks per (query, head): [rows, H, K] ascending ids, -1 pad.
+
+    Speed3R, technical summary 2.1, selection branch: the K most relevant
+    token regions for each query by the compressed branch's scores.  Blocks
+    are ranked by (-score, block id), so equal scores go to the lower id; the
+    first K_eff = min(K, NB) are kept.  (The candidates are first narrowed to
+    the blocks scoring at least the K-th largest score, which cannot change
+    the ranking's first K_eff entries.)
+    """
+    rows, H, NB = guide.shape
+    k = geo.K_eff
+    sel = np.full((rows, H, geo.K), -1, dtype=np.int64)
+    kth = -np.partition(-guide, k - 1, axis=-1)[..., k - 1]
+    for a in range(rows):
+        for h in range(H):
+            g = guide[a, h]
+            cand = np.nonzero(g >= kth[a, h])[0]
+            ranked = cand[np.lexsort((cand, -g[cand]))]
+            sel[a, h, :k] = np.sort(ranked[:k])
+    return sel
+
+
+def top_k_gap(geo: Geometry, guide: np.ndarray) -> np.ndarray:
+    """s_(K) - s_(K+1) per (query, head), the K-th minus the (K+1)-th largest
+    score (inf when every block is selected)."""
+    if geo.K_eff >= guide.shape[-1]:
+        return np.full(guide.shape[:-1], np.inf)
+    k = geo.K_eff
+    part = -np.partition(-guide, (k - 1, k), axis=-1)
+    return part[..., k - 1] - part[..., k]
+
+
+# ----------------------------------------------------------------------------
+# step 5: selected (fine) attention
+
+
+def selected_keys(geo: Geometry, sel_row: np.ndarray) -> np.ndarray:
+    """Key token ids for one (query block, head): valid tokens of the selected
+    blocks, then every special token of every frame (listed once).
+
+    Speed3R, technical summary 2.1 (selection branch: fine-grained attention on
+    only the selected key/value regions) and 2.2 (Speed3R-VGGT keeps the
+    reference-frame / camera-token information in the selection branch; here
+    every special token is always attended to).
+    """
+    parts = [geo.block_tokens(b) for b in sel_row if b >= 0]
+    parts.append(geo.special_tokens())
+    return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+
+
+def selected_attention(geo: Geometry, Q, K, V, sel: np.ndarray, rows: np.ndarray,
+                       entries: np.ndarray) -> np.ndarray:
+    """O_sel for fine query tokens ``rows``: [len(rows), H, D].
+
+    ``sel`` is [len(entries), H, K] (the top-K of each compressed entry) and
+    row t uses the selection of its own entry (its query block).  One softmax
+    runs over the whole key set of selected_keys().
+    """
+    pos = {int(a): i for i, a in enumerate(entries)}
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, geo.H, geo.D), dtype=np.float64)
+    q_all = f64(Q, rows)
+    by_entry: dict[int, list[int]] = {}
+    for i, t in enumerate(rows):
+        by_entry.setdefault(geo.entry_of_token(int(t)), []).append(i)
+    for a, idx in by_entry.items():
+        for h in range(geo.H):
+            keys = selected_keys(geo, sel[pos[a], h])
+            k = f64_head(K, keys, h)
+            v = f64_head(V, keys, h)
+            s = q_all[idx, h] @ k.T * geo.sm_scale
+            out[idx, h] = softmax(s, axis=-1) @ v
+    return out
+
+
+# ----------------------------------------------------------------------------
+# step 6: gate and nearest up-sampling
+
+
+def gate(geo: Geometry, Qc_rows: np.ndarray, w) -> np.ndarray:
+    """g = sigmoid(q_mean . w_h) per (compressed entry, head): [rows, H].
+
+    Speed3R, technical summary 2.1, gated aggregation: a learnable sigmoid
+    gate computed from the query weights the two branch outputs.
+    """
+    wv = f64(w)
+    z = np.sum(Qc_rows * wv[None], axis=-1)
+    with np.errstate(over="ignore"):  # exp(-z) = inf gives g = 0 exactly
+        return 1.0 / (1.0 + np.exp(-z))
+
+
+def combine(g_rows: np.ndarray, o_cmp_up: np.ndarray, o_sel: np.ndarray) -> np.ndarray:
+    """out = g * up(O_cmp) + (1 - g) * O_sel (g broadcast over D)."""
+    return g_rows[..., None] * o_cmp_up + (1.0 - g_rows[..., None]) * o_sel
+
+
+# ----------------------------------------------------------------------------
+# the whole layer
+
+
+def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
+              chunk_elems: int = 50_000_000) -> dict:
+    """The GSA layer for fine query tokens ``rows`` (all tokens when None).
+
+    Returns a dict of float64 arrays:
+      rows, entries (compressed entries owning the rows), o_cmp [entries,H,D],
+      guide [entries,H,NB] (only when NB*len(entries) is small), gap
+      [entries,H], sel [entries,H,K] (the oracle's own top-K), o_sel
+      [rows,H,D], g [entries,H], out [rows,H,D], and the pooled tensors qc,
+      kc, vc when they are small.
+
+    ``sel_override`` ({entry: [H, K] ids}) replaces the selection used by the
+    selection branch (to evaluate fine attention on another valid top-K
+    set); the oracle's own selection is still returned in ``sel``.
+    """
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
+    Qc = pool(geo, Q)
+    Kc = pool(geo, K)
+    Vc = pool(geo, V)
+    entries = np.array(sorted({geo.entry_of_token(int(t)) for t in rows}), dtype=np.int64)
+    nE = entries.size
+    o_cmp = np.empty((nE, geo.H, geo.D))
+    sel = np.empty((nE, geo.H, geo.K), dtype=np.int64)
+    gap = np.empty((nE, geo.H))
+    keep_guide = nE * geo.NB * geo.H <= 50_000_000
+    guide_all = np.empty((nE, geo.H, geo.NB)) if keep_guide else None
+    step = max(1, chunk_elems // (geo.H * geo.Tc))
+    for e0 in range(0, nE, step):
+        e1 = min(nE, e0 + step)
+        o, logits = compressed_attention(geo, Qc[entries[e0:e1]], Kc, Vc)
+        o_cmp[e0:e1] = o
+        guide = guide_scores(geo, logits)
+        sel[e0:e1] = top_k_blocks(geo, guide)
+        gap[e0:e1] = top_k_gap(geo, guide)
+        if keep_guide:
+            guide_all[e0:e1] = guide
+    sel_used = sel.copy()
+    if sel_override is not None:
+        pos = {int(a): i for i, a in enumerate(entries)}
+        for a, s in sel_override.items():
+            sel_used[pos[int(a)]] = np.asarray(s)
+    o_sel = selected_attention(geo, Q, K, V, sel_used, rows, entries)
+    g = gate(geo, Qc[entries], w)
+    pos = {int(a): i for i, a in enumerate(entries)}
+    own = np.array([pos[geo.entry_of_token(int(t))] for t in rows], dtype=np.int64)
+    out = combine(g[own], o_cmp[own], o_sel)
+    res = dict(rows=rows, entries=entries, own=own, o_cmp=o_cmp, sel=sel, gap=gap,
+               o_sel=o_sel, g=g, out=out, o_cmp_up=o_cmp[own])
+    if keep_guide:
+        res["guide"] = guide_all
+    if geo.Tc * geo.H * geo.D <= 20_000_000:
+        res.update(qc=Qc, kc=Kc, vc=Vc)
+    return res
+
+
+# ----------------------------------------------------------------------------
+# dense global attention (the layer GSA replaces)
+
+
+def dense_attention(geo: Geometry, Q, K, V, rows=None, max_bytes: int = 1 << 30) -> np.ndarray:
+    """softmax(q K^T / sqrt(D)) V over all T tokens, for fine query ``rows``.
+
+    Speed3R, technical summary 1 (Background): the dense global attention of
+    DUSt3R / VGGT-style models, quadratic in the number of tokens.
+    """
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, geo.H, geo.D))
+    step = max(1, min(rows.size, max_bytes // max(geo.H * geo.T * 8, 1)))
+    kc = 1 << 16
+    small = geo.T <= kc
+    if small:
+        k_all, v_all = f64(K), f64(V)
+    for r0 in range(0, rows.size, step):
+        r1 = min(rows.size, r0 + step)
+        q = f64(Q, rows[r0:r1])
+        if small:
+            out[r0:r1] = weighted_values(softmax(qk_logits(q, k_all, geo.sm_scale)), v_all)
+            continue
+        # the full score row is built key slice by key slice, then one softmax
+        s = np.empty((r1 - r0, geo.H, geo.T))
+        for t0 in range(0, geo.T, kc):
+            t1 = min(geo.T, t0 + kc)
+            s[..., t0:t1] = qk_logits(q, f64(K, slice(t0, t1)), geo.sm_scale)
+        p = softmax(s)
+        acc = np.zeros((r1 - r0, geo.H, geo.D))
+        for t0 in range(0, geo.T, kc):
+            t1 = min(geo.T, t0 + kc)
+            acc += weighted_values(p[..., t0:t1], f64(V, slice(t0, t1)))
+        out[r0:r1] = acc
+    return out
+
+
+# ----------------------------------------------------------------------------
+# selection checks used by parity tests
+
+
+def selection_is_valid_top_k(geo: Geometry, guide_row: np.ndarray, chosen: np.ndarray,
+                             window: float) -> bool:
+    """True if ``chosen`` (ids, -1 pad) is a top-K of ``guide_row`` up to ``window``.
+
+    A set is accepted when it has K_eff distinct valid ids and no unchosen
+    block beats a chosen one by more than ``window``.  With window 0 and no
+    ties this is exactly the oracle's own top-K.
+    """
+    ids = np.asarray([b for b in chosen if b >= 0], dtype=np.int64)
+    if ids.size != geo.K_eff or np.unique(ids).size != ids.size:
+        return False
+    if ids.min(initial=0) < 0 or ids.max(initial=0) >= guide_row.size:
+        return False
+    if ids.size == guide_row.size:
+        return True
+    mask = np.zeros(guide_row.size, dtype=bool)
+    mask[ids] = True
+    return bool(guide_row[~mask].max() - guide_row[mask].min() < window)

@@ -1,0 +1,270 @@
+"""Checks that pin the CPU oracle to facts outside itself.
+
+Each ``pin_*`` raises AssertionError when the oracle disagrees with a closed
+form, a library routine (torch's scaled_dot_product_attention in float64), the
+independent pure-Python brute force in ``bruteforce.py``, or an invariant the
+method fixes.  The oracle is looked up through its module at call time so the
+mutation tests can plant mistakes in it and see these checks fail.
+"""
+
+import numpy as np
+import torch
+
+import bruteforce
+from oracle import gsa_oracle as O
+from synthetic import Workload, generate
+
+TOL = 1e-11
+
+
+def micro(N=2, S=1, Hp=6, Wp=7, H=2, D=8, P=4, K=2, seed=5):
+    wl = Workload("micro", N, S, Hp, Wp, H, D, P, K, seed, "gaussian")
+    x = generate(wl)
+    geo = O.Geometry(N=N, S=S, Hp=Hp, Wp=Wp, H=H, D=D, P=P, K=K)
+    return geo, x
+
+
+def sdpa_dense(q, k, v):
+    """torch's scaled_dot_product_attention in float64: [T, H, D] -> [T, H, D]."""
+    t = lambda x: x.to(torch.float64).permute(1, 0, 2).unsqueeze(0)  # noqa: E731
+    o = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v))
+    return o.squeeze(0).permute(1, 0, 2).numpy()
+
+
+def close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol, f"{what}: max abs err {err:.3e} > {tol:.1e}"
+
+
+def read_block_structure_fixture(path):
+    vals = {}
+    for line in open(path):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            k, v = line.split("=")
+            vals[k.strip()] = int(v)
+    return vals
+
+
+# ---------------------------------------------------------------------------
+
+
+def pin_block_structure(fixture_path):
+    """37x37 grid, P=4: 100 blocks per frame; 81 of 16, 18 of 4, 1 of 1 tokens."""
+    want = read_block_structure_fixture(fixture_path)
+    geo = O.Geometry(N=1, S=5, Hp=37, Wp=37, H=1, D=64, P=4, K=1)
+    sizes = [O.Geometry.block_tokens(geo, b).size for b in range(geo.NB)]
+    assert geo.Bf == want["blocks_per_frame"]
+    assert sizes.count(16) == want["full_blocks"]
+    assert sizes.count(4) == want["edge_blocks"]
+    assert sizes.count(1) == want["corner_blocks"]
+    assert sum(sizes) == want["patch_tokens"]
+
+
+def pin_pool_ramp():
+    """Pooling a ramp: the block mean has a closed form from the row/col ranges."""
+    N, S, Hp, Wp, H, D, P = 2, 2, 7, 6, 2, 3, 4
+    geo = O.Geometry(N=N, S=S, Hp=Hp, Wp=Wp, H=H, D=D, P=P, K=1)
+    L = S + Hp * Wp
+    X = np.zeros((N * L, H, D))
+    for f in range(N):
+        for j in range(S):
+            X[f * L + j] = -(100.0 + 10 * f + j)
+        for r in range(Hp):
+            for c in range(Wp):
+                for h in range(H):
+                    for d in range(D):
+                        X[f * L + S + r * Wp + c, h, d] = 1000 * f + 10 * r + c + 0.25 * h + 0.125 * d
+    got = O.pool(geo, X)
+    E = S + (-(-Hp // P)) * (-(-Wp // P))
+    assert got.shape == (N * E, H, D)
+    for f in range(N):
+        for j in range(S):
+            close(got[f * E + j], np.full((H, D), -(100.0 + 10 * f + j)), what="special entry")
+        i = S
+        for r0 in range(0, Hp, P):
+            r1 = min(r0 + P, Hp)
+            for c0 in range(0, Wp, P):
+                c1 = min(c0 + P, Wp)
+                mr, mc = (r0 + r1 - 1) / 2.0, (c0 + c1 - 1) / 2.0
+                want = np.array([[1000 * f + 10 * mr + mc + 0.25 * h + 0.125 * d for d in range(D)]
+                                 for h in range(H)])
+                close(got[f * E + i], want, what=f"block ({r0},{c0})")
+                i += 1
+
+
+def pin_dense_matches_sdpa():
+    geo, x = micro(N=3, S=2, Hp=5, Wp=4, H=3, D=16)
+    close(O.dense_attention(geo, x.q, x.k, x.v), sdpa_dense(x.q, x.k, x.v), what="dense vs sdpa")
+
+
+def pin_compressed_is_dense_at_pool_1():
+    """P=1: every block is one patch, so the compression branch is dense attention."""
+    geo, x = micro(N=2, S=2, Hp=4, Wp=5, H=2, D=16, P=1, K=3)
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    close(res["o_cmp"], sdpa_dense(x.q, x.k, x.v), what="o_cmp(P=1) vs dense")
+
+
+def pin_selected_is_dense_at_k_all():
+    """K >= number of blocks: the selection branch attends to every token once."""
+    geo, x = micro(N=2, S=2, Hp=6, Wp=7, H=2, D=16, P=4, K=99)
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    close(res["o_sel"], sdpa_dense(x.q, x.k, x.v), what="o_sel(K=all) vs dense")
+
+
+def pin_layer_is_dense_at_pool_1_k_all():
+    geo, x = micro(N=2, S=1, Hp=3, Wp=5, H=2, D=8, P=1, K=1000)
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    close(res["out"], sdpa_dense(x.q, x.k, x.v), what="out(P=1,K=all) vs dense")
+
+
+def pin_constant_values():
+    geo, x = micro(N=2, S=1, Hp=6, Wp=7, H=2, D=8)
+    c = np.linspace(-1.5, 2.0, geo.H * geo.D).reshape(geo.H, geo.D)
+    v = torch.from_numpy(np.broadcast_to(c, (geo.T, geo.H, geo.D)).copy())
+    res = O.gsa_layer(geo, x.q, x.k, v, x.w)
+    for name in ("o_cmp", "o_sel", "out"):
+        close(res[name], np.broadcast_to(c, res[name].shape), what=f"constant V: {name}")
+
+
+def pin_zero_queries():
+    """Q = 0: every score ties at 0, so blocks 0..K-1 are chosen (lower id wins)
+    and each branch returns a plain mean over its keys."""
+    N, S, Hp, Wp, H, D, P, K = 2, 1, 6, 7, 2, 8, 4, 3
+    geo, x = micro(N=N, S=S, Hp=Hp, Wp=Wp, H=H, D=D, P=P, K=K)
+    q = torch.zeros_like(x.q)
+    res = O.gsa_layer(geo, q, x.k, x.v, x.w)
+    assert (res["sel"] == np.arange(K)).all(), "ties must go to the lowest block ids"
+    frames = bruteforce.layout(N, S, Hp, Wp, P)
+    blocks = [b for _, bl in frames for b in bl]
+    specials = [t for sp, _ in frames for t in sp]
+    v = x.v.to(torch.float64).numpy()
+    keys = [t for b in blocks[:K] for t in b] + specials
+    close(res["o_sel"], np.broadcast_to(v[keys].mean(axis=0), res["o_sel"].shape), what="o_sel(Q=0)")
+    entries = []
+    for sp, bl in frames:
+        entries += [[t] for t in sp] + bl
+    vbar = np.stack([v[e].mean(axis=0) for e in entries])
+    close(res["o_cmp"], np.broadcast_to(vbar.mean(axis=0), res["o_cmp"].shape), what="o_cmp(Q=0)")
+    close(res["g"], np.full(res["g"].shape, 0.5), what="g(Q=0)")
+
+
+def pin_gate_limits():
+    geo, x = micro(N=2, S=1, Hp=6, Wp=7, H=2, D=8)
+    q = x.q.clone()
+    q[..., 0] = q[..., 0].abs() + 1.0  # every pooled query has q_mean[0] >= 1
+    zero = torch.zeros_like(x.w)
+    res = O.gsa_layer(geo, q, x.k, x.v, zero)
+    close(res["g"], np.full(res["g"].shape, 0.5), what="g(w=0)")
+    close(res["out"], 0.5 * (res["o_cmp_up"] + res["o_sel"]), what="out(w=0)")
+    big = torch.zeros_like(x.w)
+    big[:, 0] = 1000.0
+    res = O.gsa_layer(geo, q, x.k, x.v, big)
+    close(res["out"], res["o_cmp_up"], tol=1e-9, what="g->1 keeps the compression branch")
+    res = O.gsa_layer(geo, q, x.k, x.v, -big)
+    close(res["out"], res["o_sel"], tol=1e-9, what="g->0 keeps the selection branch")
+
+
+def pin_planted_top_k():
+    """Every query equals u; block beta's keys all equal c_beta * u, so its score
+    is c_beta |u|^2 / sqrt(D).  Special keys score highest of all but are not
+    candidates.  Two blocks tie at the boundary: the lower id must win."""
+    N, S, Hp, Wp, H, D, P, K = 3, 2, 6, 7, 2, 8, 4, 4
+    geo = O.Geometry(N=N, S=S, Hp=Hp, Wp=Wp, H=H, D=D, P=P, K=K)
+    rng = np.random.default_rng(11)
+    u = rng.standard_normal((H, D))
+    NB = geo.NB
+    c = rng.permutation(NB).astype(np.float64)  # distinct 0..NB-1
+    c[c == NB - K] = NB - K - 1.0  # the K-th largest now ties with the (K+1)-th
+    L = S + Hp * Wp
+    q = np.broadcast_to(u, (N * L, H, D)).copy()
+    k = np.zeros((N * L, H, D))
+    frames = bruteforce.layout(N, S, Hp, Wp, P)
+    beta = 0
+    for sp, bl in frames:
+        for t in sp:
+            k[t] = 1000.0 * u
+        for toks in bl:
+            for t in toks:
+                k[t] = c[beta] * u
+            beta += 1
+    v = rng.standard_normal((N * L, H, D))
+    res = O.gsa_layer(geo, q, k, v, np.zeros((H, D)))
+    want = sorted(sorted(range(NB), key=lambda b: (-c[b], b))[:K])
+    for a in range(res["sel"].shape[0]):
+        for h in range(H):
+            assert list(res["sel"][a, h]) == want, f"planted top-K: {list(res['sel'][a, h])} != {want}"
+
+
+def pin_bruteforce_layer():
+    geo, x = micro(N=2, S=1, Hp=6, Wp=7, H=2, D=8, P=4, K=2)
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    Q = x.q.to(torch.float64).tolist()
+    K = x.k.to(torch.float64).tolist()
+    V = x.v.to(torch.float64).tolist()
+    W = x.w.to(torch.float64).tolist()
+    bf = bruteforce.gsa_bruteforce(Q, K, V, W, geo.N, geo.S, geo.Hp, geo.Wp, geo.P, geo.K)
+    close(res["o_cmp"], bf["o_cmp"], what="brute force o_cmp")
+    assert res["sel"].tolist() == bf["sel"], "brute force selection"
+    close(res["o_sel"], bf["o_sel"], what="brute force o_sel")
+    close(res["g"], bf["g"], what="brute force gate")
+    close(res["out"], bf["out"], what="brute force out")
+
+
+def pin_bruteforce_dense():
+    geo, x = micro(N=2, S=1, Hp=3, Wp=4, H=2, D=8)
+    Q, K, V = (t.to(torch.float64).tolist() for t in (x.q, x.k, x.v))
+    close(O.dense_attention(geo, x.q, x.k, x.v), bruteforce.dense_bruteforce(Q, K, V), what="dense bf")
+
+
+def pin_frame_permutation():
+    """Reordering the frames reorders every output the same way and renames the
+    selected blocks by the same permutation (inputs without ties)."""
+    geo, x = micro(N=3, S=1, Hp=5, Wp=6, H=2, D=8, P=4, K=3)
+    perm = [2, 0, 1]
+    L = geo.L
+    idx = torch.cat([torch.arange(p * L, (p + 1) * L) for p in perm])
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    res2 = O.gsa_layer(geo, x.q[idx], x.k[idx], x.v[idx], x.w)
+    close(res2["out"], res["out"][idx.numpy()], what="permuted out")
+    Bf, E = geo.Bf, geo.E
+    new_frame = {p: f for f, p in enumerate(perm)}  # old frame -> new frame
+    for f, p in enumerate(perm):
+        for j in range(E):
+            a2, a = f * E + j, p * E + j
+            for h in range(geo.H):
+                want = sorted(new_frame[int(b) // Bf] * Bf + int(b) % Bf for b in res["sel"][a, h])
+                assert list(res2["sel"][a2, h]) == want, "permuted selection"
+
+
+def pin_row_subset():
+    """Evaluating a subset of query rows gives those rows of the full layer."""
+    geo, x = micro(N=2, S=1, Hp=6, Wp=7, H=2, D=8)
+    full = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    rows = np.array([0, 5, 17, 43, geo.T - 1])
+    sub = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows)
+    close(sub["out"], full["out"][rows], what="row subset out")
+    close(O.dense_attention(geo, x.q, x.k, x.v, rows=rows),
+          O.dense_attention(geo, x.q, x.k, x.v)[rows], what="row subset dense")
+
+
+def all_pins(fixture_path):
+    return {
+        "block_structure": lambda: pin_block_structure(fixture_path),
+        "pool_ramp": pin_pool_ramp,
+        "dense_sdpa": pin_dense_matches_sdpa,
+        "compressed_p1": pin_compressed_is_dense_at_pool_1,
+        "selected_kall": pin_selected_is_dense_at_k_all,
+        "layer_dense_limit": pin_layer_is_dense_at_pool_1_k_all,
+        "constant_v": pin_constant_values,
+        "zero_q": pin_zero_queries,
+        "gate_limits": pin_gate_limits,
+        "planted_topk": pin_planted_top_k,
+        "bruteforce_layer": pin_bruteforce_layer,
+        "bruteforce_dense": pin_bruteforce_dense,
+        "frame_permutation": pin_frame_permutation,
+        "row_subset": pin_row_subset,
+    }

@@ -1,0 +1,117 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check the pins catch each.
+
+A pin set that still passes with a dropped term, a wrong sign or index, or a
+swapped operand would not be worth much; every mutation below must make at
+least one pin in ``pins.py`` fail.
+"""
+
+import os
+import warnings
+
+import numpy as np
+import pytest
+
+import pins
+from oracle import gsa_oracle as O
+
+FIXTURE = os.path.join(os.path.dirname(__file__), "golden", "block_structure_37x37_p4.txt")
+
+
+def _pool_full_denominator(geo, X, frames_per_chunk=32):
+    out = _orig["pool"](geo, X, frames_per_chunk)
+    # re-weight every block entry as if it always held P*P patches
+    for f in range(geo.N):
+        for br in range(geo.Bh):
+            for bc in range(geo.Bw):
+                rows, cols = geo.block_rows_cols(br, bc)
+                out[f * geo.E + geo.S + br * geo.Bw + bc] *= len(rows) * len(cols) / (geo.P * geo.P)
+    return out
+
+
+def _compressed_values_are_keys(geo, Qc_rows, Kc, Vc):
+    return _orig["compressed_attention"](geo, Qc_rows, Kc, Kc)
+
+
+def _top_k_ties_high(geo, guide):
+    rows, H, NB = guide.shape
+    sel = np.full((rows, H, geo.K), -1, dtype=np.int64)
+    ids = np.arange(NB)
+    for a in range(rows):
+        for h in range(H):
+            order = np.lexsort((-ids, -guide[a, h]))
+            sel[a, h, :geo.K_eff] = np.sort(order[:geo.K_eff])
+    return sel
+
+
+def _selected_keys_without_specials(geo, sel_row):
+    parts = [geo.block_tokens(b) for b in sel_row if b >= 0]
+    return np.concatenate(parts)
+
+
+def _selected_keys_specials_twice(geo, sel_row):
+    return np.concatenate([_orig["selected_keys"](geo, sel_row), geo.special_tokens()])
+
+
+def _combine_swapped(g, o_cmp_up, o_sel):
+    return _orig["combine"](g, o_sel, o_cmp_up)
+
+
+def _combine_no_one_minus(g, o_cmp_up, o_sel):
+    return g[..., None] * o_cmp_up + o_sel
+
+
+def _guide_counts_specials(geo, logits):
+    return logits[..., :geo.NB]
+
+
+def _entry_of_token_shifted(self, t):
+    f, i = divmod(int(t), self.L)
+    if i < self.S:
+        return f * self.E + i
+    r, c = divmod(i - self.S, self.Wp)
+    return f * self.E + self.S + (r // self.P) * self.Bw + min((c + 1) // self.P, self.Bw - 1)
+
+
+def _block_rows_cols_short(self, br, bc):
+    return (range(self.P * br, min(self.P * br + self.P, self.Hp - 1)) if br == self.Bh - 1
+            else range(self.P * br, self.P * br + self.P),
+            range(self.P * bc, min(self.P * bc + self.P, self.Wp)))
+
+
+def _gate_wrong_sign(geo, Qc_rows, w):
+    return 1.0 - _orig["gate"](geo, Qc_rows, w)
+
+
+_orig = {n: getattr(O, n) for n in ("pool", "compressed_attention", "selected_keys", "combine", "gate")}
+
+MUTATIONS = {
+    "pool divides partial blocks by P*P": ("pool", _pool_full_denominator),
+    "compressed branch multiplies by K instead of V": ("compressed_attention", _compressed_values_are_keys),
+    "ties go to the higher block id": ("top_k_blocks", _top_k_ties_high),
+    "selection drops the special tokens": ("selected_keys", _selected_keys_without_specials),
+    "selection lists special tokens twice": ("selected_keys", _selected_keys_specials_twice),
+    "gate weights the selection branch": ("combine", _combine_swapped),
+    "combine drops the (1 - g) factor": ("combine", _combine_no_one_minus),
+    "special entries ranked as candidates": ("guide_scores", _guide_counts_specials),
+    "fine token up-sampled from the wrong block": ("Geometry.entry_of_token", _entry_of_token_shifted),
+    "last block row loses a patch row": ("Geometry.block_rows_cols", _block_rows_cols_short),
+    "gate sigmoid of -z": ("gate", _gate_wrong_sign),
+    "softmax scale 1/D": ("Geometry.sm_scale", property(lambda self: 1.0 / self.D)),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(name, monkeypatch):
+    target, repl = MUTATIONS[name]
+    if target.startswith("Geometry."):
+        monkeypatch.setattr(O.Geometry, target.split(".", 1)[1], repl)
+    else:
+        monkeypatch.setattr(O, target, repl)
+    failed = []
+    warnings.simplefilter("ignore")
+    for pin_name, fn in pins.all_pins(FIXTURE).items():
+        try:
+            fn()
+        except Exception:  # a failed assertion, or the mutant breaking outright
+            failed.append(pin_name)
+    assert failed, f"no pin caught the planted mistake: {name}"

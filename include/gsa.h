@@ -1,0 +1,199 @@
+/*
+ * gsa.h -- C ABI of libgsa: sparse global attention over N views (GSA) and the
+ * dense global attention it replaces, hand-written CUDA for sm_100a (B200).
+ *
+ * The operation is the global self-attention layer of VGGT-style feed-forward
+ * multi-view reconstruction in the sparse dual-branch form of
+ * "Speed3R: Sparse Feed-forward 3D Reconstruction Models" (technical summary,
+ * section 2.1 "Dual-branch attention", and section 2.2 "Speed3R-VGGT"):
+ *   - compression branch: per frame, 4x4 (generally P x P) average pooling of
+ *     Q, K and V over the patch grid, dense attention in the pooled sequence,
+ *     output up-sampled (nearest) back to the fine tokens;
+ *   - S_guide: the pooled scores of each compressed query against every patch
+ *     block; the Top-K blocks per (query block, head) are selected;
+ *   - selection branch: fine attention of each token over the tokens of its
+ *     block's selected blocks plus every special token (always kept);
+ *   - gated aggregation: g = sigmoid(q_mean . w_h) per (query block, head),
+ *     out = g * up(O_cmp) + (1 - g) * O_sel.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Tokens: frame f holds S special tokens, then Hp*Wp patch tokens (row-major);
+ * frames are concatenated: T = N * (S + Hp*Wp).  Q, K, V, out are row-major
+ * [T][H][64] bf16 (gsa_bf16 = the raw 16-bit pattern).
+ * Compressed sequence: per frame, the S specials then the Bh*Bw blocks
+ * (row-major), Bh = ceil(Hp/P), Bw = ceil(Wp/P): Tc = N * (S + Bh*Bw) entries,
+ * stored [Tc][H][64].  Patch block id beta = f*Bh*Bw + br*Bw + bc (0 <= beta <
+ * NB = N*Bh*Bw).  A block at the right/bottom edge holds only the patches that
+ * exist; its pooled value is the mean over those.
+ * Special-token copies: [H][N*S][64] bf16 (head-major, frame-major).
+ *
+ * Pointers: every buffer pointer is a device pointer (cudaMalloc'd or a slice of
+ * one) and must be 16-byte aligned; the caller owns all memory and the library
+ * never allocates, frees or keeps a pointer after a call returns.  `stream` is
+ * a cudaStream_t (NULL = the legacy default stream); all work is enqueued on it
+ * and the calls return without synchronising (except gsa_check_device_error).
+ *
+ * Workspace: every compute call takes `ws`, device memory of at least
+ * GSA_WS_HEADER_BYTES whose first word is the device error word.  Zero it once
+ * after allocation (gsa_workspace_init); kernels only set bits in it, and
+ * gsa_check_device_error reads and clears it.  gsa_forward also carves its
+ * intermediates from `ws` (size from gsa_workspace_size).
+ *
+ * Errors: arguments are validated on the host before anything is enqueued; a
+ * failed check returns GSA_ERR_INVALID_ARG / GSA_ERR_UNSUPPORTED /
+ * GSA_ERR_WORKSPACE and launches nothing.  A launch failure returns
+ * GSA_ERR_CUDA.  Nothing in the library traps the device.
+ */
+#ifndef GSA_H_
+#define GSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef uint16_t gsa_bf16; /* bfloat16 bit pattern */
+
+typedef enum {
+  GSA_OK = 0,
+  GSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or count */
+  GSA_ERR_UNSUPPORTED = 2,   /* valid but not built for (head_dim != 64, pool > 4, top_k > 128) */
+  GSA_ERR_WORKSPACE = 3,     /* workspace smaller than required */
+  GSA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
+  GSA_ERR_TIMEOUT = 5,       /* device error word: a bounded wait ran out */
+  GSA_ERR_DEVICE_CHECK = 6   /* device error word: an in-kernel bounds check failed */
+} gsa_status;
+
+/* One layer call's sizes.  All fields are read by every entry point. */
+typedef struct {
+  int32_t n_frames;  /* N >= 1 */
+  int32_t n_special; /* S >= 0 special tokens per frame (camera/register) */
+  int32_t hp;        /* patch grid height >= 1 */
+  int32_t wp;        /* patch grid width >= 1 */
+  int32_t n_heads;   /* H in [1, 128] */
+  int32_t head_dim;  /* D; only 64 is built */
+  int32_t pool;      /* P in [1, 4]: P x P average pooling of the patch grid */
+  int32_t top_k;     /* K in [1, 128]: selected blocks per (query block, head) */
+  float scale;       /* softmax scale; 0 means 1/sqrt(D) */
+} gsa_shape;
+
+/* Derived sizes (see the conventions above). */
+typedef struct {
+  int64_t T;     /* fine tokens N*(S+Hp*Wp) */
+  int64_t Tc;    /* compressed entries N*(S+Bh*Bw) */
+  int64_t NB;    /* patch blocks N*Bh*Bw (top-K candidates) */
+  int64_t NS;    /* special tokens N*S */
+  int32_t L;     /* tokens per frame S+Hp*Wp */
+  int32_t E;     /* compressed entries per frame S+Bh*Bw */
+  int32_t Bh, Bw, Bf;
+  int32_t K_eff; /* min(K, NB) */
+} gsa_sizes;
+
+#define GSA_WS_HEADER_BYTES 256
+
+/* Validate `shape` and fill `out`.  Pure host code (needs no GPU). */
+gsa_status gsa_derive(const gsa_shape* shape, gsa_sizes* out);
+
+/* Bytes of workspace gsa_forward needs for `shape` (header included).  Host only. */
+gsa_status gsa_workspace_size(const gsa_shape* shape, size_t* bytes);
+
+/* Zero the workspace header (the device error word) on `stream`. */
+gsa_status gsa_workspace_init(void* ws, void* stream);
+
+/*
+ * Step 1, compression by pooling (Speed3R technical summary 2.1, compression
+ * branch: spatial down-sampling, e.g. 4x4 average pooling, to a coarse context).
+ * Reads q, k, v [T][H][64] bf16.  Writes, per compressed entry a and head h:
+ *   qc32, kc32   [Tc][H][64] fp32  mean of Q / K (scores and the gate use these)
+ *   vc           [Tc][H][64] bf16  mean of V (round-to-nearest-even)
+ *   qc, kc       [Tc][H][64] bf16  mean of Q / K (may be NULL: not written)
+ *   ks, vs       [H][N*S][64] bf16 copies of the special tokens' K / V
+ *                (ignored when S == 0; may be NULL: not written)
+ * A special token's entry is the token itself.
+ */
+gsa_status gsa_pool_kv(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                       const gsa_bf16* v, float* qc32, float* kc32, gsa_bf16* vc, gsa_bf16* qc,
+                       gsa_bf16* kc, gsa_bf16* ks, gsa_bf16* vs, void* ws, void* stream);
+
+/*
+ * Steps 2-3, attention in the compressed space and its block scores
+ * (technical summary 2.1; S_guide on the it page, section 2).
+ *   oc [Tc][H][64] fp32: softmax(scale * qc kc^T) vc over all Tc entries.
+ *   cand_score / cand_idx [H][Tc][n_split][K]: for every (head, entry) and each
+ *   of `n_split` equal slices of the patch-block range, the K largest
+ *   S_guide[h][a][beta] = scale * (qc32[a,h] . kc32[entry(beta),h]) of that
+ *   slice with their block ids, unordered, padded with (-inf, -1).
+ * qc / kc are the bf16 pooled tensors of gsa_pool_kv, qc32 / kc32 the fp32 ones.
+ * n_split in [1, 64].
+ */
+gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const gsa_bf16* kc,
+                               const gsa_bf16* vc, const float* qc32, const float* kc32,
+                               float* oc, float* cand_score, int32_t* cand_idx, int32_t n_split,
+                               void* ws, void* stream);
+
+/*
+ * Step 4, Top-K block selection (technical summary 2.1, selection branch:
+ * the K most relevant token regions per query by the compressed scores).
+ * Merges the n_split candidate lists of gsa_compressed_attn into
+ *   sel [H][Tc][K] int32: the K_eff blocks with the largest score (ties go to
+ *   the lower block id), in ascending id order, padded with -1.
+ */
+gsa_status gsa_topk_blocks(const gsa_shape* shape, const float* cand_score,
+                           const int32_t* cand_idx, int32_t n_split, int32_t* sel, void* ws,
+                           void* stream);
+
+/*
+ * Step 5, selected attention (technical summary 2.1, selection branch;
+ * 2.2, Speed3R-VGGT keeps the special/camera tokens).  For token t in
+ * compressed entry a and head h: one softmax over the valid tokens of the
+ * blocks sel[h][a][:] plus all N*S special tokens (ks/vs, NULL when S == 0):
+ *   o_sel [T][H][64] bf16, and lse [T][H] fp32 = log sum exp of the scaled
+ *   logits (may be NULL).
+ */
+gsa_status gsa_selected_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                             const gsa_bf16* v, const gsa_bf16* ks, const gsa_bf16* vs,
+                             const int32_t* sel, gsa_bf16* o_sel, float* lse, void* ws,
+                             void* stream);
+
+/*
+ * Step 6, gated aggregation and nearest up-sampling (technical summary 2.1:
+ * a learnable sigmoid gate computed from the query mixes the two branches).
+ *   g[a,h] = sigmoid(qc32[a,h] . w[h]),  w [H][64] fp32
+ *   out[t,h] = g * oc[a(t),h] + (1 - g) * o_sel[t,h]   -> out [T][H][64] bf16
+ */
+gsa_status gsa_gate_combine(const gsa_shape* shape, const float* qc32, const float* w,
+                            const float* oc, const gsa_bf16* o_sel, gsa_bf16* out, void* ws,
+                            void* stream);
+
+/*
+ * Dense global attention (technical summary 1: the quadratic all-to-all
+ * attention GSA replaces): out = softmax(scale * q k^T) v over all T tokens,
+ * per head.  Uses n_frames, n_special, hp, wp, n_heads, head_dim, scale.
+ */
+gsa_status dense_global_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                             const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream);
+
+/*
+ * The whole GSA layer: steps 1-6 enqueued on `stream`, intermediates in `ws`
+ * (ws_bytes >= gsa_workspace_size).  w [H][64] fp32 gate vectors; out
+ * [T][H][64] bf16.  Steps 5 and 6 run fused in one kernel.
+ */
+gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                       const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
+                       size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read the device error word in `ws`, clear it, and
+ * return GSA_OK, GSA_ERR_TIMEOUT or GSA_ERR_DEVICE_CHECK. */
+gsa_status gsa_check_device_error(void* ws, void* stream);
+
+/* Static text for a status code. */
+const char* gsa_status_string(gsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSA_H_ */

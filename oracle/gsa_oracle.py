@@ -388,19 +388,21 @@ def combine(g_rows: np.ndarray, o_cmp_up: np.ndarray, o_sel: np.ndarray) -> np.n
 
 
 def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
-              chunk_elems: int = 50_000_000) -> dict:
+              tie_window: float = 1e-3, chunk_elems: int = 50_000_000) -> dict:
     """The GSA layer for fine query tokens ``rows`` (all tokens when None).
 
     Returns a dict of float64 arrays:
-      rows, entries (compressed entries owning the rows), o_cmp [entries,H,D],
-      guide [entries,H,NB] (only when NB*len(entries) is small), gap
-      [entries,H], sel [entries,H,K] (the oracle's own top-K), o_sel
-      [rows,H,D], g [entries,H], out [rows,H,D], and the pooled tensors qc,
-      kc, vc when they are small.
+      rows, entries (compressed entries owning the rows), own (entry position of
+      each row), o_cmp [entries,H,D], sel [entries,H,K] (the oracle's own
+      top-K), gap [entries,H] (K-th minus (K+1)-th score), o_sel [rows,H,D],
+      g [entries,H], out [rows,H,D], o_cmp_up [rows,H,D]; guide
+      [entries,H,NB] and the pooled tensors qc, kc, vc when they are small.
 
-    ``sel_override`` ({entry: [H, K] ids}) replaces the selection used by the
-    selection branch (to evaluate fine attention on another valid top-K
-    set); the oracle's own selection is still returned in ``sel``.
+    ``sel_override`` ([Tc, H, K] block ids, -1 pad) is another selection to
+    evaluate the selection branch with.  It is checked against this oracle's
+    S_guide scores: ``sel_exact`` [entries,H] says it equals the oracle's own
+    top-K, ``sel_valid`` [entries,H] that it is a top-K up to ``tie_window``
+    (no unchosen block beats a chosen one by ``tie_window`` or more).
     """
     rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
     Qc = pool(geo, Q)
@@ -413,6 +415,11 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     gap = np.empty((nE, geo.H))
     keep_guide = nE * geo.NB * geo.H <= 50_000_000
     guide_all = np.empty((nE, geo.H, geo.NB)) if keep_guide else None
+    other = None
+    if sel_override is not None:
+        other = np.asarray(sel_override)[entries].astype(np.int64)
+        sel_exact = np.zeros((nE, geo.H), dtype=bool)
+        sel_valid = np.zeros((nE, geo.H), dtype=bool)
     step = max(1, chunk_elems // (geo.H * geo.Tc))
     for e0 in range(0, nE, step):
         e1 = min(nE, e0 + step)
@@ -423,11 +430,13 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
         gap[e0:e1] = top_k_gap(geo, guide)
         if keep_guide:
             guide_all[e0:e1] = guide
-    sel_used = sel.copy()
-    if sel_override is not None:
-        pos = {int(a): i for i, a in enumerate(entries)}
-        for a, s in sel_override.items():
-            sel_used[pos[int(a)]] = np.asarray(s)
+        if other is not None:
+            for i in range(e0, e1):
+                for h in range(geo.H):
+                    sel_exact[i, h] = np.array_equal(other[i, h], sel[i, h])
+                    sel_valid[i, h] = selection_is_valid_top_k(geo, guide[i - e0, h], other[i, h],
+                                                               tie_window)
+    sel_used = sel if other is None else other
     o_sel = selected_attention(geo, Q, K, V, sel_used, rows, entries)
     g = gate(geo, Qc[entries], w)
     pos = {int(a): i for i, a in enumerate(entries)}
@@ -435,6 +444,8 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     out = combine(g[own], o_cmp[own], o_sel)
     res = dict(rows=rows, entries=entries, own=own, o_cmp=o_cmp, sel=sel, gap=gap,
                o_sel=o_sel, g=g, out=out, o_cmp_up=o_cmp[own])
+    if other is not None:
+        res.update(sel_exact=sel_exact, sel_valid=sel_valid)
     if keep_guide:
         res["guide"] = guide_all
     if geo.Tc * geo.H * geo.D <= 20_000_000:

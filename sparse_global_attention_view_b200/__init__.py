@@ -1,0 +1,22 @@
+"""Sparse global attention over N views (GSA) and dense global attention on B200.
+
+The compute lives in ``lib/libgsa.so`` (CUDA for sm_100a, C ABI in
+``include/gsa.h``); this package is its Python binding.
+"""
+
+from ._lib import GsaError, GsaShape, GsaSizes, LIB_PATH, load  # noqa: F401
+from .api import (  # noqa: F401
+    GsaLayer,
+    Shape,
+    check_device_error,
+    compressed_attn,
+    dense_global_attn,
+    derive,
+    forward,
+    gate_combine,
+    new_workspace,
+    pool_kv,
+    selected_attn,
+    topk_blocks,
+    workspace_size,
+)

@@ -1,0 +1,191 @@
+"""Thin Python binding of libgsa: torch tensors in, C-ABI calls out.
+
+Every function here only checks tensor placement, dtype, contiguity and size,
+turns tensors into device pointers and calls the entry point of the same name
+in ``include/gsa.h``; all arithmetic runs in the library's CUDA kernels.  There
+is no CPU fallback: a missing library or a CPU tensor raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import torch
+
+from ._lib import GsaShape, GsaSizes, WS_HEADER_BYTES, check, load
+
+BF16 = torch.bfloat16
+F32 = torch.float32
+I32 = torch.int32
+
+
+@dataclass(frozen=True)
+class Shape:
+    """One layer call's sizes (``gsa_shape``)."""
+
+    n_frames: int
+    n_special: int
+    hp: int
+    wp: int
+    n_heads: int
+    head_dim: int = 64
+    pool: int = 4
+    top_k: int = 16
+    scale: float = 0.0
+
+    def c(self) -> GsaShape:
+        return GsaShape(self.n_frames, self.n_special, self.hp, self.wp, self.n_heads,
+                        self.head_dim, self.pool, self.top_k, float(self.scale))
+
+    @staticmethod
+    def of(workload) -> "Shape":
+        return Shape(workload.n_frames, workload.n_special, workload.hp, workload.wp,
+                     workload.n_heads, workload.head_dim, workload.pool, workload.top_k)
+
+
+def derive(shape: Shape) -> GsaSizes:
+    z = GsaSizes()
+    check(load().gsa_derive(ctypes.byref(shape.c()), ctypes.byref(z)), "gsa_derive")
+    return z
+
+
+def workspace_size(shape: Shape) -> int:
+    n = ctypes.c_size_t()
+    check(load().gsa_workspace_size(ctypes.byref(shape.c()), ctypes.byref(n)), "gsa_workspace_size")
+    return n.value
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t, dtype, numel, name, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} has {t.numel()} elements, expected {numel}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ws(ws, min_bytes=WS_HEADER_BYTES):
+    if not isinstance(ws, torch.Tensor) or not ws.is_cuda or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    if ws.numel() * ws.element_size() < min_bytes:
+        raise ValueError(f"workspace holds {ws.numel() * ws.element_size()} bytes, needs {min_bytes}")
+    return ctypes.c_void_p(ws.data_ptr())
+
+
+def new_workspace(shape: Shape | None = None, device="cuda", stream=None) -> torch.Tensor:
+    """A zeroed workspace: the forward's size for ``shape``, else just the header."""
+    n = workspace_size(shape) if shape is not None else WS_HEADER_BYTES
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    check(load().gsa_workspace_init(ctypes.c_void_p(ws.data_ptr()), _stream(stream)),
+          "gsa_workspace_init")
+    return ws
+
+
+def pool_kv(shape, q, k, v, qc32, kc32, vc, qc=None, kc=None, ks=None, vs=None, ws=None, stream=None):
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    ent = z.Tc * shape.n_heads * shape.head_dim
+    spc = z.NS * shape.n_heads * shape.head_dim
+    check(load().gsa_pool_kv(
+        ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(qc32, F32, ent, "qc32"), _ptr(kc32, F32, ent, "kc32"), _ptr(vc, BF16, ent, "vc"),
+        _ptr(qc, BF16, ent, "qc", True), _ptr(kc, BF16, ent, "kc", True),
+        _ptr(ks, BF16, spc, "ks", True), _ptr(vs, BF16, spc, "vs", True), _ws(ws), _stream(stream)),
+        "gsa_pool_kv")
+
+
+def compressed_attn(shape, qc, kc, vc, qc32, kc32, oc, cand_score, cand_idx, n_split, ws, stream=None):
+    z = derive(shape)
+    ent = z.Tc * shape.n_heads * shape.head_dim
+    cand = shape.n_heads * z.Tc * n_split * shape.top_k
+    check(load().gsa_compressed_attn(
+        ctypes.byref(shape.c()), _ptr(qc, BF16, ent, "qc"), _ptr(kc, BF16, ent, "kc"),
+        _ptr(vc, BF16, ent, "vc"), _ptr(qc32, F32, ent, "qc32"), _ptr(kc32, F32, ent, "kc32"),
+        _ptr(oc, F32, ent, "oc"), _ptr(cand_score, F32, cand, "cand_score"),
+        _ptr(cand_idx, I32, cand, "cand_idx"), ctypes.c_int32(n_split), _ws(ws), _stream(stream)),
+        "gsa_compressed_attn")
+
+
+def topk_blocks(shape, cand_score, cand_idx, n_split, sel, ws, stream=None):
+    z = derive(shape)
+    cand = shape.n_heads * z.Tc * n_split * shape.top_k
+    check(load().gsa_topk_blocks(
+        ctypes.byref(shape.c()), _ptr(cand_score, F32, cand, "cand_score"),
+        _ptr(cand_idx, I32, cand, "cand_idx"), ctypes.c_int32(n_split),
+        _ptr(sel, I32, shape.n_heads * z.Tc * shape.top_k, "sel"), _ws(ws), _stream(stream)),
+        "gsa_topk_blocks")
+
+
+def selected_attn(shape, q, k, v, ks, vs, sel, o_sel, lse=None, ws=None, stream=None):
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    spc = z.NS * shape.n_heads * shape.head_dim
+    need_sp = z.NS > 0
+    check(load().gsa_selected_attn(
+        ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(ks, BF16, spc, "ks", not need_sp), _ptr(vs, BF16, spc, "vs", not need_sp),
+        _ptr(sel, I32, shape.n_heads * z.Tc * shape.top_k, "sel"), _ptr(o_sel, BF16, tok, "o_sel"),
+        _ptr(lse, F32, z.T * shape.n_heads, "lse", True), _ws(ws), _stream(stream)),
+        "gsa_selected_attn")
+
+
+def gate_combine(shape, qc32, w, oc, o_sel, out, ws, stream=None):
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    ent = z.Tc * shape.n_heads * shape.head_dim
+    check(load().gsa_gate_combine(
+        ctypes.byref(shape.c()), _ptr(qc32, F32, ent, "qc32"),
+        _ptr(w, F32, shape.n_heads * shape.head_dim, "w"), _ptr(oc, F32, ent, "oc"),
+        _ptr(o_sel, BF16, tok, "o_sel"), _ptr(out, BF16, tok, "out"), _ws(ws), _stream(stream)),
+        "gsa_gate_combine")
+
+
+def dense_global_attn(shape, q, k, v, out, ws, stream=None):
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    check(load().dense_global_attn(
+        ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(out, BF16, tok, "out"), _ws(ws), _stream(stream)), "dense_global_attn")
+
+
+def forward(shape, q, k, v, w, out, ws, stream=None):
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    need = workspace_size(shape)
+    check(load().gsa_forward(
+        ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(w, F32, shape.n_heads * shape.head_dim, "w"), _ptr(out, BF16, tok, "out"), _ws(ws, need),
+        ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)), "gsa_forward")
+
+
+def check_device_error(ws, stream=None) -> None:
+    check(load().gsa_check_device_error(_ws(ws), _stream(stream)), "gsa_check_device_error")
+
+
+class GsaLayer:
+    """Convenience owner of a workspace for repeated ``forward`` calls of one shape."""
+
+    def __init__(self, shape: Shape, device="cuda"):
+        self.shape = shape
+        self.sizes = derive(shape)
+        self.ws = new_workspace(shape, device)
+
+    def __call__(self, q, k, v, w, out=None, stream=None):
+        if out is None:
+            out = torch.empty_like(q)
+        forward(self.shape, q, k, v, w, out, self.ws, stream)
+        return out

@@ -1,0 +1,317 @@
+// The C ABI of libgsa (include/gsa.h): argument validation, size derivation,
+// workspace layout, and the enqueueing of each step on the caller's stream.
+// Nothing here allocates device memory or keeps state between calls.
+#include <math.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+using gsa::bf16;
+using gsa::Dims;
+
+namespace {
+
+inline bool al16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+inline bool dev_ptr(const void* p) { return p != nullptr && al16(p); }
+inline bool opt_ptr(const void* p) { return p == nullptr || al16(p); }
+inline size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline gsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GSA_OK : GSA_ERR_CUDA; }
+
+gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
+  if (s == nullptr) return GSA_ERR_INVALID_ARG;
+  if (s->n_frames < 1 || s->n_special < 0 || s->hp < 1 || s->wp < 1 || s->n_heads < 1 ||
+      s->head_dim < 1 || s->pool < 1 || s->top_k < 1)
+    return GSA_ERR_INVALID_ARG;
+  if (!(s->scale >= 0.f) || isinf(s->scale)) return GSA_ERR_INVALID_ARG;
+  if (s->head_dim != gsa::kHeadDim || s->pool > gsa::kMaxPool || s->top_k > gsa::kMaxTopK ||
+      s->n_heads > 128)
+    return GSA_ERR_UNSUPPORTED;
+  const long long L = (long long)s->n_special + (long long)s->hp * s->wp;
+  const long long Bh = (s->hp + s->pool - 1) / s->pool, Bw = (s->wp + s->pool - 1) / s->pool;
+  const long long Bf = Bh * Bw, E = s->n_special + Bf;
+  const long long N = s->n_frames;
+  const long long T = N * L, Tc = N * E, NB = N * Bf, NS = N * s->n_special;
+  // token / block ids are int32 on the device, grids are at most 2^31-1 wide
+  if (L > INT32_MAX || T > INT32_MAX || NB + NS > INT32_MAX) return GSA_ERR_INVALID_ARG;
+  Dims t;
+  t.N = s->n_frames;
+  t.S = s->n_special;
+  t.Hp = s->hp;
+  t.Wp = s->wp;
+  t.H = s->n_heads;
+  t.P = s->pool;
+  t.K = s->top_k;
+  t.Keff = (int)(NB < s->top_k ? NB : s->top_k);
+  t.L = (int)L;
+  t.E = (int)E;
+  t.Bh = (int)Bh;
+  t.Bw = (int)Bw;
+  t.Bf = (int)Bf;
+  t.T = T;
+  t.Tc = Tc;
+  t.NB = NB;
+  t.NS = NS;
+  t.scale = s->scale > 0.f ? s->scale : 1.f / sqrtf((float)s->head_dim);
+  t.scale_log2 = t.scale * 1.4426950408889634f;
+  if (d) *d = t;
+  if (z) {
+    z->T = T;
+    z->Tc = Tc;
+    z->NB = NB;
+    z->NS = NS;
+    z->L = t.L;
+    z->E = t.E;
+    z->Bh = t.Bh;
+    z->Bw = t.Bw;
+    z->Bf = t.Bf;
+    z->K_eff = t.Keff;
+  }
+  return GSA_OK;
+}
+
+constexpr int kMaxCandidates = 2048;  // n_split * K per row in the merge
+
+int forward_splits(const Dims& d) {
+  const long long row_ctas = ((d.Tc + 127) / 128) * d.H;
+  long long ns = (2 * 148 + row_ctas - 1) / row_ctas;
+  if (ns < 1) ns = 1;
+  if (ns > 16) ns = 16;
+  if (ns > d.NB) ns = d.NB;
+  while (ns > 1 && ns * d.K > kMaxCandidates) --ns;
+  return (int)ns;
+}
+
+struct Layout {
+  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cs, ci, sel, total;
+  int n_split;
+};
+
+Layout forward_layout(const Dims& d) {
+  Layout l;
+  l.n_split = forward_splits(d);
+  const size_t ent = (size_t)d.Tc * d.H * gsa::kHeadDim;
+  const size_t spc = (size_t)d.NS * d.H * gsa::kHeadDim;
+  const size_t cand = (size_t)d.H * d.Tc * l.n_split * d.K;
+  size_t o = GSA_WS_HEADER_BYTES;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += up256(bytes);
+    return at;
+  };
+  l.qc32 = take(ent * 4);
+  l.kc32 = take(ent * 4);
+  l.vc = take(ent * 2);
+  l.qc = take(ent * 2);
+  l.kc = take(ent * 2);
+  l.ks = take(spc * 2);
+  l.vs = take(spc * 2);
+  l.oc = take(ent * 4);
+  l.cs = take(cand * 4);
+  l.ci = take(cand * 4);
+  l.sel = take((size_t)d.H * d.Tc * d.K * 4);
+  l.total = o;
+  return l;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gsa_status_string(gsa_status s) {
+  switch (s) {
+    case GSA_OK: return "ok";
+    case GSA_ERR_INVALID_ARG: return "invalid argument";
+    case GSA_ERR_UNSUPPORTED: return "unsupported shape (head_dim must be 64, pool <= 4, top_k <= 128, n_heads <= 128)";
+    case GSA_ERR_WORKSPACE: return "workspace too small";
+    case GSA_ERR_CUDA: return "CUDA error";
+    case GSA_ERR_TIMEOUT: return "device wait timed out";
+    case GSA_ERR_DEVICE_CHECK: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+gsa_status gsa_derive(const gsa_shape* shape, gsa_sizes* out) {
+  if (out == nullptr) return GSA_ERR_INVALID_ARG;
+  return make_dims(shape, nullptr, out);
+}
+
+gsa_status gsa_workspace_size(const gsa_shape* shape, size_t* bytes) {
+  Dims d;
+  if (bytes == nullptr) return GSA_ERR_INVALID_ARG;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  *bytes = forward_layout(d).total;
+  return GSA_OK;
+}
+
+gsa_status gsa_workspace_init(void* ws, void* stream) {
+  if (!dev_ptr(ws)) return GSA_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, GSA_WS_HEADER_BYTES, as_stream(stream)));
+}
+
+gsa_status gsa_pool_kv(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                       const gsa_bf16* v, float* qc32, float* kc32, gsa_bf16* vc, gsa_bf16* qc,
+                       gsa_bf16* kc, gsa_bf16* ks, gsa_bf16* vs, void* ws, void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(qc32) || !dev_ptr(kc32) ||
+      !dev_ptr(vc) || !opt_ptr(qc) || !opt_ptr(kc) || !opt_ptr(ks) || !opt_ptr(vs) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  if ((ks == nullptr) != (vs == nullptr)) return GSA_ERR_INVALID_ARG;
+  if (d.NS == 0) ks = vs = nullptr;
+  return cuda_status(gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32,
+                                      (bf16*)vc, (bf16*)qc, (bf16*)kc, (bf16*)ks, (bf16*)vs,
+                                      as_stream(stream)));
+}
+
+gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const gsa_bf16* kc,
+                               const gsa_bf16* vc, const float* qc32, const float* kc32,
+                               float* oc, float* cand_score, int32_t* cand_idx, int32_t n_split,
+                               void* ws, void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(qc) || !dev_ptr(kc) || !dev_ptr(vc) || !dev_ptr(qc32) || !dev_ptr(kc32) ||
+      !dev_ptr(oc) || !dev_ptr(cand_score) || !dev_ptr(cand_idx) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  if (n_split < 1 || n_split > 64 || (long long)n_split * d.K > kMaxCandidates)
+    return GSA_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  gsa::AttnArgs a;
+  a.q = (const bf16*)qc;
+  a.k = (const bf16*)kc;
+  a.v = (const bf16*)vc;
+  a.q_row = a.kv_row = a.o_row = (long long)d.H * gsa::kHeadDim;
+  a.q_head = a.kv_head = a.o_head = gsa::kHeadDim;
+  a.n_q = a.n_k = d.Tc;
+  a.o = oc;
+  a.o_f32 = true;
+  a.lse = nullptr;
+  a.lse_row = a.lse_head = 0;
+  a.H = d.H;
+  a.scale = d.scale;
+  a.scale_log2 = d.scale_log2;
+  cudaError_t e = gsa::launch_attn_mma(a, s);
+  if (e != cudaSuccess) return GSA_ERR_CUDA;
+  return cuda_status(gsa::launch_block_scores_topk(d, qc32, kc32, cand_score, cand_idx, n_split, s));
+}
+
+gsa_status gsa_topk_blocks(const gsa_shape* shape, const float* cand_score,
+                           const int32_t* cand_idx, int32_t n_split, int32_t* sel, void* ws,
+                           void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(cand_score) || !dev_ptr(cand_idx) || !dev_ptr(sel) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  if (n_split < 1 || n_split > 64 || (long long)n_split * d.K > kMaxCandidates)
+    return GSA_ERR_INVALID_ARG;
+  return cuda_status(gsa::launch_topk_merge(d, cand_score, cand_idx, n_split, sel, as_stream(stream)));
+}
+
+gsa_status gsa_selected_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                             const gsa_bf16* v, const gsa_bf16* ks, const gsa_bf16* vs,
+                             const int32_t* sel, gsa_bf16* o_sel, float* lse, void* ws,
+                             void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(sel) || !dev_ptr(o_sel) ||
+      !opt_ptr(lse) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  if (d.NS > 0 && (!dev_ptr(ks) || !dev_ptr(vs))) return GSA_ERR_INVALID_ARG;
+  return cuda_status(gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v,
+                                          (const bf16*)ks, (const bf16*)vs, sel, nullptr, nullptr,
+                                          nullptr, (bf16*)o_sel, lse, (unsigned*)ws,
+                                          as_stream(stream)));
+}
+
+gsa_status gsa_gate_combine(const gsa_shape* shape, const float* qc32, const float* w,
+                            const float* oc, const gsa_bf16* o_sel, gsa_bf16* out, void* ws,
+                            void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(qc32) || !dev_ptr(w) || !dev_ptr(oc) || !dev_ptr(o_sel) || !dev_ptr(out) ||
+      !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  return cuda_status(
+      gsa::launch_gate_combine(d, qc32, w, oc, (const bf16*)o_sel, (bf16*)out, as_stream(stream)));
+}
+
+gsa_status dense_global_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                             const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(out) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  gsa::AttnArgs a;
+  a.q = (const bf16*)q;
+  a.k = (const bf16*)k;
+  a.v = (const bf16*)v;
+  a.q_row = a.kv_row = a.o_row = (long long)d.H * gsa::kHeadDim;
+  a.q_head = a.kv_head = a.o_head = gsa::kHeadDim;
+  a.n_q = a.n_k = d.T;
+  a.o = out;
+  a.o_f32 = false;
+  a.lse = nullptr;
+  a.lse_row = a.lse_head = 0;
+  a.H = d.H;
+  a.scale = d.scale;
+  a.scale_log2 = d.scale_log2;
+  return cuda_status(gsa::launch_attn_mma(a, as_stream(stream)));
+}
+
+gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                       const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
+                       size_t ws_bytes, void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(w) || !dev_ptr(out) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  const Layout l = forward_layout(d);
+  if (ws_bytes < l.total) return GSA_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  float* qc32 = (float*)(base + l.qc32);
+  float* kc32 = (float*)(base + l.kc32);
+  bf16* vc = (bf16*)(base + l.vc);
+  bf16* qc = (bf16*)(base + l.qc);
+  bf16* kc = (bf16*)(base + l.kc);
+  bf16* ks = d.NS > 0 ? (bf16*)(base + l.ks) : nullptr;
+  bf16* vs = d.NS > 0 ? (bf16*)(base + l.vs) : nullptr;
+  float* oc = (float*)(base + l.oc);
+  float* cs = (float*)(base + l.cs);
+  int* ci = (int*)(base + l.ci);
+  int* sel = (int*)(base + l.sel);
+  cudaStream_t s = as_stream(stream);
+  cudaError_t e = gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32,
+                                   vc, qc, kc, ks, vs, s);
+  if (e != cudaSuccess) return GSA_ERR_CUDA;
+  st = gsa_compressed_attn(shape, (const gsa_bf16*)qc, (const gsa_bf16*)kc, (const gsa_bf16*)vc,
+                           qc32, kc32, oc, cs, ci, l.n_split, ws, stream);
+  if (st != GSA_OK) return st;
+  e = gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s);
+  if (e != cudaSuccess) return GSA_ERR_CUDA;
+  e = gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, ks, vs, sel, qc32, w,
+                           oc, (bf16*)out, nullptr, (unsigned*)ws, s);
+  return cuda_status(e);
+}
+
+gsa_status gsa_check_device_error(void* ws, void* stream) {
+  if (!dev_ptr(ws)) return GSA_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GSA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GSA_ERR_CUDA;
+  if (word != 0 && cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return GSA_ERR_CUDA;
+  if (word & gsa::kErrTimeout) return GSA_ERR_TIMEOUT;
+  if (word & gsa::kErrDeviceCheck) return GSA_ERR_DEVICE_CHECK;
+  return GSA_OK;
+}
+
+}  // extern "C"

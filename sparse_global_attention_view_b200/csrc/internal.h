@@ -1,0 +1,51 @@
+// Launchers shared between the C-ABI layer (host.cu) and the kernel files.
+// Each returns cudaGetLastError() after enqueueing on `st`; arguments are
+// validated by the caller.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace gsa {
+
+cudaError_t launch_pool(const Dims& d, const bf16* q, const bf16* k, const bf16* v, float* qc32,
+                        float* kc32, bf16* vc, bf16* qc, bf16* kc, bf16* ks, bf16* vs,
+                        cudaStream_t st);
+
+// Flash-style attention over rows of a strided [rows][H][64] layout, per head.
+struct AttnArgs {
+  const bf16* q;
+  long long q_row, q_head;  // element strides
+  long long n_q;
+  const bf16* k;
+  const bf16* v;
+  long long kv_row, kv_head;
+  long long n_k;
+  void* o;  // bf16 or fp32
+  long long o_row, o_head;
+  bool o_f32;
+  float* lse;  // nullable, [n_q][H] with strides lse_row, lse_head
+  long long lse_row, lse_head;
+  int H;
+  float scale, scale_log2;
+};
+cudaError_t launch_attn_mma(const AttnArgs& a, cudaStream_t st);
+
+cudaError_t launch_block_scores_topk(const Dims& d, const float* qc32, const float* kc32,
+                                     float* cand_score, int* cand_idx, int n_split,
+                                     cudaStream_t st);
+cudaError_t launch_topk_merge(const Dims& d, const float* cand_score, const int* cand_idx,
+                              int n_split, int* sel, cudaStream_t st);
+
+// Selection branch; when `w` is non-null the gate is fused and `out` receives
+// g*oc + (1-g)*o_sel, otherwise `out` receives o_sel (and lse if non-null).
+cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const bf16* v,
+                            const bf16* ks, const bf16* vs, const int* sel, const float* qc32,
+                            const float* w, const float* oc, bf16* out, float* lse,
+                            unsigned* err, cudaStream_t st);
+
+cudaError_t launch_gate_combine(const Dims& d, const float* qc32, const float* w, const float* oc,
+                                const bf16* o_sel, bf16* out, cudaStream_t st);
+
+}  // namespace gsa

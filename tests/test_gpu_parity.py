@@ -1,0 +1,196 @@
+"""CUDA path vs the float64 CPU oracle, through the C ABI (needs a B200).
+
+Every step of the path is checked element by element on workloads the oracle
+finishes in seconds (several tiles, ragged tails, partial edge blocks, K >= the
+number of blocks, pool factors 1-4, no special tokens), and the whole layer on
+sampled query rows of the 100-, 300- and 1000-frame workloads.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import parity as PT
+from oracle import gsa_oracle as O
+from synthetic import WORKLOADS, Workload, generate
+from synthetic.workloads import sample_rows
+
+pytestmark = pytest.mark.gpu
+
+CASES = {
+    "tiny": WORKLOADS["tiny"],
+    "small": WORKLOADS["small"],
+    # pool 3 with ragged blocks in both directions, 2 specials per frame
+    "p3_ragged": Workload("p3_ragged", 3, 2, 10, 11, 2, 64, 3, 5, 7, "gaussian"),
+    # pool 1 (every block one patch), no specials, T not a multiple of 64
+    "p1_nospecial": Workload("p1_nospecial", 2, 0, 5, 7, 2, 64, 1, 6, 8, "gaussian"),
+    # K larger than the number of blocks: every block kept, -1 padding
+    "k_all": Workload("k_all", 2, 3, 6, 7, 3, 64, 4, 128, 9, "gaussian"),
+    # pool 2, one head, single special
+    "p2_onehead": Workload("p2_onehead", 4, 1, 9, 9, 1, 64, 2, 7, 10, "gaussian"),
+    # one VGGT-shaped frame
+    "one_frame": Workload("one_frame", 1, 5, 37, 37, 4, 64, 4, 16, 11, "gaussian"),
+}
+
+_cache = {}
+
+
+def _dev(x):
+    return (x.q.cuda(), x.k.cuda(), x.v.cuda(), x.w.cuda())
+
+
+def case(name, n_split=1):
+    key = (name, n_split)
+    if key not in _cache:
+        import sparse_global_attention_view_b200 as G
+        wl = CASES[name]
+        x = generate(wl)
+        geo = O.geometry_of(wl)
+        shape = G.Shape.of(wl)
+        q, k, v, w = _dev(x)
+        st = PT.Stages(shape, q, k, v, w, n_split).run()
+        res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, sel_override=st.sel_by_entry())
+        _cache[key] = (x, geo, shape, st, res)
+    return _cache[key]
+
+
+NAMES = list(CASES)
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_pool(name):
+    x, geo, shape, st, res = case(name)
+    np.testing.assert_allclose(st.qc32.cpu().double().numpy(), res["qc"], rtol=1e-6, atol=1e-7)
+    np.testing.assert_allclose(st.kc32.cpu().double().numpy(), res["kc"], rtol=1e-6, atol=1e-7)
+    # bf16 round-to-nearest of the mean: within half an ulp (2^-8 relative bounds it)
+    np.testing.assert_allclose(st.vc.cpu().double().numpy(), res["vc"], rtol=2.0 ** -8, atol=1e-30)
+    np.testing.assert_allclose(st.qc.cpu().double().numpy(), res["qc"], rtol=2.0 ** -8, atol=1e-30)
+    if geo.NS:
+        spec = torch.as_tensor(geo.special_tokens())
+        assert torch.equal(st.ks.cpu(), x.k[spec].permute(1, 0, 2))
+        assert torch.equal(st.vs.cpu(), x.v[spec].permute(1, 0, 2))
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_compressed_attention(name):
+    x, geo, shape, st, res = case(name)
+    assert PT.zeros_fail(res["o_cmp"])
+    PT.assert_close(st.oc, res["o_cmp"], f"{name} o_cmp")
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_top_k_selection(name):
+    x, geo, shape, st, res = case(name)
+    PT.assert_selection(res, name)
+    sel = st.sel_by_entry()
+    assert (sel[:, :, geo.K_eff:] == -1).all()
+    chosen = sel[:, :, :geo.K_eff]
+    assert (chosen >= 0).all() and (chosen < geo.NB).all()
+    assert (np.diff(chosen, axis=-1) > 0).all(), "ids must be strictly ascending"
+
+
+@pytest.mark.parametrize("name", ["small", "p3_ragged"])
+def test_split_candidates_merge_to_same_selection(name):
+    a = case(name, 1)[3].sel.cpu()
+    b = case(name, 3)[3].sel.cpu()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_selected_attention(name):
+    x, geo, shape, st, res = case(name)
+    assert PT.zeros_fail(res["o_sel"])
+    PT.assert_close(st.o_sel, res["o_sel"], f"{name} o_sel")
+    assert torch.isfinite(st.lse).all()
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_gate_combine(name):
+    x, geo, shape, st, res = case(name)
+    assert PT.zeros_fail(res["out"])
+    PT.assert_close(st.out, res["out"], f"{name} out (stages)")
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_forward(name):
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    layer = G.GsaLayer(shape)
+    out1 = torch.full_like(st.q, float("nan"))
+    layer(st.q, st.k, st.v, st.w, out1)
+    out2 = layer(st.q, st.k, st.v, st.w)
+    torch.cuda.synchronize()
+    G.check_device_error(layer.ws)
+    PT.assert_close(out1, res["out"], f"{name} out (forward)")
+    assert torch.equal(out1, out2), "forward must be deterministic"
+
+
+@pytest.mark.parametrize("name", ["tiny", "p3_ragged", "p1_nospecial", "k_all", "p2_onehead"])
+def test_dense_full(name):
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    out = torch.full_like(st.q, float("nan"))
+    G.dense_global_attn(shape, st.q, st.k, st.v, out, st.ws)
+    ref = O.dense_attention(geo, x.q, x.k, x.v)
+    assert PT.zeros_fail(ref)
+    PT.assert_close(out, ref, f"{name} dense")
+
+
+@pytest.mark.parametrize("name", ["small", "one_frame"])
+def test_dense_sampled(name):
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    out = torch.full_like(st.q, float("nan"))
+    G.dense_global_attn(shape, st.q, st.k, st.v, out, st.ws)
+    rows = sample_rows(geo.T, 384, seed=1, forced=PT.forced_rows(geo))
+    ref = O.dense_attention(geo, x.q, x.k, x.v, rows=rows)
+    PT.assert_close(out[torch.as_tensor(rows).cuda()], ref, f"{name} dense sampled")
+    assert not torch.isnan(out).any()
+
+
+# ---- the 100, 300 and 1000-frame workloads on sampled rows -----------------
+
+BIG = {"medium": 384, "large": 256, "pages": 128}
+
+
+@pytest.mark.parametrize("name", list(BIG))
+def test_big_workload_sampled(name):
+    import sparse_global_attention_view_b200 as G
+    wl = WORKLOADS[name]
+    x = generate(wl)
+    geo = O.geometry_of(wl)
+    shape = G.Shape.of(wl)
+    q, k, v, w = _dev(x)
+    st = PT.Stages(shape, q, k, v, w).run()
+    layer = G.GsaLayer(shape)
+    out = torch.full_like(q, float("nan"))
+    layer(q, k, v, w, out)
+    torch.cuda.synchronize()
+    G.check_device_error(layer.ws)
+    assert not torch.isnan(out).any()
+    rows = sample_rows(geo.T, BIG[name], seed=2, forced=PT.forced_rows(geo))
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows, sel_override=st.sel_by_entry())
+    PT.assert_selection(res, name)
+    idx = torch.as_tensor(rows).cuda()
+    ent = torch.as_tensor(res["entries"]).cuda()
+    PT.assert_close(st.oc[ent], res["o_cmp"], f"{name} o_cmp")
+    PT.assert_close(st.o_sel[idx], res["o_sel"], f"{name} o_sel")
+    PT.assert_close(out[idx], res["out"], f"{name} out")
+    del st, layer
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["medium"])
+def test_big_dense_sampled(name):
+    import sparse_global_attention_view_b200 as G
+    wl = WORKLOADS[name]
+    x = generate(wl)
+    geo = O.geometry_of(wl)
+    shape = G.Shape.of(wl)
+    q, k, v, w = _dev(x)
+    ws = G.new_workspace(None)
+    out = torch.full_like(q, float("nan"))
+    G.dense_global_attn(shape, q, k, v, out, ws)
+    rows = sample_rows(geo.T, 64, seed=3, forced=PT.forced_rows(geo))
+    ref = O.dense_attention(geo, x.q, x.k, x.v, rows=rows)
+    PT.assert_close(out[torch.as_tensor(rows).cuda()], ref, f"{name} dense sampled")

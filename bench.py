@@ -1,0 +1,462 @@
+"""Benchmark of the GSA layer (sparse global attention over N views) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload pages]
+    python bench.py --impl reference ...      # the float64 CPU oracle, timed
+
+A step is one whole GSA layer (pooling, compressed attention, S_guide top-K,
+top-K merge, selected attention with the gate) over the workload's tokens, with
+Q/K/V resident in HBM.  The metric is tokens per second of the layer (and ms
+per layer); the dense global attention it replaces is timed in the same run.
+Multi-GPU runs (torchrun, one rank per GPU) give every rank its own scene of the
+same size: there is no exchange inside the layer, so the scaling is weak and
+the value is all ranks' tokens over the slowest rank's time.
+
+Prints one JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synthetic import WORKLOADS, generate  # noqa: E402
+
+METRIC = "global-attn layer ms & tokens/s at N views; % of bf16 tensor peak / HBM BW"
+UNIT = "tokens/s"
+SM_COUNT = 148
+FFMA_PER_SM_PER_CLK = 128
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return dict(hbm_gbs=p["hbm_gbs"], bf16_tflops=p["bf16_tflops"],
+                    bf16_tflops_sustained=p.get("bf16_tflops_sustained", p["bf16_tflops"]),
+                    sm_max_mhz=p.get("sm_max_mhz", 1965.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, sm_max_mhz=1965.0,
+                source="fallback")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per step (counts only what the method computes)
+
+
+def stage_work(z, H, D, K_eff) -> dict:
+    """Per-stage algorithmic work of one layer: (bound, amount, unit)."""
+    T, Tc, NB, NS = z.T, z.Tc, z.NB, z.NS
+    return {
+        # read Q, K, V once; write qc32, kc32 (fp32), vc, qc, kc (bf16) and the special copies
+        "pool": ("hbm", 3 * T * H * D * 2 + Tc * H * D * (4 + 4 + 2 + 2 + 2) + 2 * NS * H * D * 2, "bytes"),
+        # QK^T and PV over the Tc x Tc pooled sequence
+        "compressed_attn": ("tensor", 4 * Tc * Tc * H * D, "flop"),
+        # one fp32 dot product of length D per (entry, patch block, head)
+        "block_scores": ("alu", 2 * Tc * NB * H * D, "flop"),
+        # candidates read once, selection written once
+        "topk_merge": ("hbm", H * Tc * K_eff * 8 + H * Tc * K_eff * 4, "bytes"),
+        # QK^T and PV of every token over the specials plus K_eff blocks of (at most) 16 tokens
+        "selected_gate": ("tensor", 4 * T * H * D * (NS + 16 * K_eff), "flop"),
+    }
+
+
+def dense_flops(z, H, D) -> int:
+    return 4 * z.T * z.T * H * D
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        try:
+            p = torch.cuda.get_device_properties(device)
+            self.bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            self.bus = None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+        if self.bus:
+            cmd += ["-i", self.bus]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (cpu_baseline and --impl reference)
+
+
+def sample_entries(geo, n_entries: int, seed: int) -> np.ndarray:
+    """All fine tokens of ``n_entries`` seeded compressed entries (query blocks)."""
+    rng = np.random.default_rng([seed, 5])
+    ents = np.sort(rng.choice(geo.Tc, size=min(n_entries, geo.Tc), replace=False))
+    return np.concatenate([geo.tokens_of_entry(int(a)) for a in ents])
+
+
+def oracle_sample(x, n_entries: int, seed: int, pooled=None):
+    """Time the oracle: one pooling pass (unless given), then the rest of the
+    layer for every token of ``n_entries`` sampled query blocks.  Returns
+    (pool_s, rest_s, res, rows, pooled); the full layer takes about
+    pool_s + rest_s * Tc / n_entries."""
+    from oracle import gsa_oracle as O
+    geo = O.geometry_of(x.workload)
+    t0 = time.perf_counter()
+    if pooled is None:
+        pooled = (O.pool(geo, x.q), O.pool(geo, x.k), O.pool(geo, x.v))
+    t1 = time.perf_counter()
+    rows = sample_entries(geo, n_entries, seed)
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows, pooled=pooled)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1, res, rows, pooled
+
+
+def cpu_threads() -> int:
+    return torch.get_num_threads()
+
+
+def run_reference(args) -> None:
+    """The float64 CPU oracle as the reference arm (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    torch.set_num_threads(os.cpu_count() or 1)
+    wl = WORKLOADS[args.workload]
+    x = generate(wl)
+    from oracle import gsa_oracle as O
+    geo = O.geometry_of(wl)
+    t0 = time.perf_counter()
+    pooled = (O.pool(geo, x.q), O.pool(geo, x.k), O.pool(geo, x.v))
+    t_pool = time.perf_counter() - t0
+    n_ent = args.ref_entries
+    times = []
+    for i in range(args.warmup + args.steps):
+        _, t_rest, _, _, _ = oracle_sample(x, n_ent, seed=100 + i, pooled=pooled)
+        if i >= args.warmup:
+            times.append(t_rest)
+    t_rest = statistics.mean(times)
+    layer_s = t_pool + t_rest * geo.Tc / n_ent
+    value = geo.T / layer_s
+    sample = (f"float64 oracle: one pooling pass over all {geo.T} tokens ({t_pool:.1f} s) plus, per step, "
+              f"all tokens of {n_ent} seeded query blocks through compressed attention, top-K, selected "
+              f"attention and the gate ({t_rest:.2f} s mean); full-layer time extrapolated as "
+              f"pool + sample * Tc / {n_ent} = {layer_s:.0f} s")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(wl, l2_note=None) -> dict:
+    c = {"workload": f"{wl.name}: N={wl.n_frames} frames x ({wl.n_special} special + {wl.hp}x{wl.wp} patches) "
+                     f"= {wl.n_tokens} tokens, {wl.n_heads} heads x {wl.head_dim}, pool {wl.pool}x{wl.pool}, "
+                     f"top-K {wl.top_k}, {wl.kind} generator seed {wl.seed}",
+         "n_frames": wl.n_frames, "tokens": wl.n_tokens, "heads": wl.n_heads, "head_dim": wl.head_dim,
+         "pool": wl.pool, "top_k": wl.top_k, "parallelism": "replicas (independent scene per rank)"}
+    if l2_note:
+        c["l2"] = l2_note
+    return c
+
+
+# ---------------------------------------------------------------------------
+
+
+def source_hash(path: str) -> str:
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel's
+    source is unchanged since it was captured."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    try:
+        rec = json.load(open(path)).get(f"{kernel_file}@{workload}")
+        src = os.path.join(ROOT, "sparse_global_attention_view_b200", "csrc", kernel_file)
+        if rec and rec.get("source_sha") == source_hash(src):
+            return rec["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+STAGE_SOURCE = {"pool": "pool.cu", "compressed_attn": "attn_mma.cu", "block_scores": "topk.cu",
+                "topk_merge": "topk.cu", "selected_gate": "selected.cu"}
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["gsa", "reference"], default="gsa")
+    ap.add_argument("--workload", choices=list(WORKLOADS), default="pages")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense global attention baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
+    ap.add_argument("--dense-steps", type=int, default=1)
+    ap.add_argument("--cpu-entries", type=int, default=48, help="query blocks in the cpu_baseline sample")
+    ap.add_argument("--ref-entries", type=int, default=16, help="query blocks per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "gsa":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import sparse_global_attention_view_b200 as G
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = WORKLOADS[args.workload]
+    if rank:
+        wl = wl.with_(seed=wl.seed + 1000 * rank)  # an independent scene per rank
+    x = generate(wl)
+    shape = G.Shape.of(wl)
+    z = G.derive(shape)
+    H, D = shape.n_heads, shape.head_dim
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    q, k, v, w = (t.to(dev) for t in (x.q, x.k, x.v, x.w))
+    out = torch.empty_like(q)
+    layer = G.GsaLayer(shape, dev)
+    in_bytes = 3 * q.numel() * 2
+    big = in_bytes > 4 * 126 * 2**20
+    flush = None if big else torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
+    n_ev = len(G.FORWARD_STEPS) + 1
+
+    def new_events(n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(n)]
+        for row in evs:
+            for e in row:
+                e.record(stream)  # create the handles
+        return evs
+
+    warm = new_events(1)[0]
+    for _ in range(args.warmup):
+        G.forward_timed(shape, q, k, v, w, out, layer.ws, warm, stream)
+        if flush is not None:
+            flush.fill_(1)
+    torch.cuda.synchronize()
+    G.check_device_error(layer.ws)
+
+    evs = new_events(args.steps)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    launches = 0
+    start.record(stream)
+    for i in range(args.steps):
+        launches += G.forward_timed(shape, q, k, v, w, out, layer.ws, evs[i], stream)
+        if flush is not None:
+            flush.fill_(1)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    G.check_device_error(layer.ws)
+
+    per_step = [[evs[i][s].elapsed_time(evs[i][s + 1]) for s in range(n_ev - 1)] for i in range(args.steps)]
+    stage_ms = {name: statistics.mean(r[s] for r in per_step) for s, name in enumerate(G.FORWARD_STEPS)}
+    step_ms_local = (start.elapsed_time(stop) / args.steps) if flush is None else \
+        statistics.mean(sum(r) for r in per_step)
+    step_ms = max_over_ranks(step_ms_local)
+    value = world * z.T / (step_ms / 1e3)
+
+    # ---- per-stage roofline from the same timed steps ----
+    P = peaks()
+    work = stage_work(z, H, D, min(shape.top_k, z.NB))
+    alu_peak = SM_COUNT * FFMA_PER_SM_PER_CLK * 2 * P["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s fp32 FMA
+    stages = {}
+    for name in G.FORWARD_STEPS:
+        bound, amount, unit = work[name]
+        ms = stage_ms[name]
+        if ms <= 0:
+            continue
+        if bound == "hbm":
+            ach, peak, u = amount / (ms / 1e3) / 1e9, P["hbm_gbs"], "GB/s"
+        elif bound == "tensor":
+            ach, peak, u = amount / (ms / 1e3) / 1e12, P["bf16_tflops"], "TFLOP/s"
+        else:
+            ach, peak, u = amount / (ms / 1e3) / 1e12, alu_peak, "TFLOP/s"
+        stages[name] = {"ms": round(ms, 4), "share": round(ms / sum(stage_ms.values()), 4), "bound": bound,
+                        "achieved": round(ach, 2), "peak": round(peak, 1), "unit": u,
+                        "frac": round(ach / peak, 4)}
+    dom = max(stages, key=lambda n: stages[n]["ms"])
+    ds = stages[dom]
+    traffic = recorded_traffic(STAGE_SOURCE[dom], wl.name)
+    roofline = {"kernel": dom, "bound": ds["bound"], "achieved": ds["achieved"], "peak": ds["peak"],
+                "unit": ds["unit"], "frac": ds["frac"], "traffic": traffic,
+                "peak_source": (f"{P['source']} (MEASURED_PEAKS.json)" if ds["bound"] != "alu" else
+                                f"fp32 FFMA: {SM_COUNT} SMs x {FFMA_PER_SM_PER_CLK} FMA/clk x 2 x "
+                                f"{P['sm_max_mhz']:.0f} MHz")}
+
+    # ---- end to end: pinned host buffers, copies inside the timed region ----
+    hq, hk, hv, hw = (t.pin_memory() for t in (x.q, x.k, x.v, x.w))
+    hout = torch.empty_like(x.q).pin_memory()
+    e_steps = max(1, min(args.steps, 5))
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        w.copy_(hw, non_blocking=True)
+        G.forward(shape, q, k, v, w, out, layer.ws, stream)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hw))
+    d2h = hout.numel() * hout.element_size()
+    e2e = {"value": world * z.T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+           "path": "pinned host Q/K/V/w -> device, gsa_forward, device -> pinned host out"}
+
+    # ---- the dense global attention baseline on the same inputs ----
+    dense = None
+    if not args.no_dense:
+        dout = torch.empty_like(q)
+        G.dense_global_attn(shape, q, k, v, dout, layer.ws, stream)
+        torch.cuda.synchronize()
+        barrier()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(args.dense_steps):
+            G.dense_global_attn(shape, q, k, v, dout, layer.ws, stream)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        dms = max_over_ranks(d0.elapsed_time(d1) / args.dense_steps)
+        tf = dense_flops(z, H, D) / (dms / 1e3) / 1e12
+        dense = {"ms_per_layer": round(dms, 3), "tokens_per_s": world * z.T / (dms / 1e3),
+                 "tflops": round(tf, 1), "frac_bf16_peak": round(tf / P["bf16_tflops"], 4),
+                 "gsa_speedup": round(dms / step_ms, 2), "kernel": "mma.sync m16n8k16 flash attention",
+                 "steps": args.dense_steps}
+        del dout
+
+    # ---- the CPU oracle on a bounded sample, and parity of the sampled rows ----
+    cpu = None
+    parity = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        torch.set_num_threads(os.cpu_count() or 1)
+        sel_gpu = G.workspace_view(layer.ws, shape, "sel").permute(1, 0, 2).contiguous().cpu().numpy()
+        out_host = out.cpu()
+        t_pool, t_rest, res0, rows, pooled = oracle_sample(x, args.cpu_entries, seed=7)
+        layer_s = t_pool + t_rest * z.Tc / args.cpu_entries
+        cpu = {"value": z.T / layer_s, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+               "sample": (f"one float64 pooling pass over all {z.T} tokens ({t_pool:.1f} s) + all tokens of "
+                          f"{args.cpu_entries} seeded query blocks through the rest of the layer "
+                          f"({t_rest:.1f} s); full-layer time extrapolated as pool + sample * Tc / "
+                          f"{args.cpu_entries} = {layer_s:.0f} s")}
+        from oracle import gsa_oracle as O
+        geo = O.geometry_of(wl)
+        res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows, sel_override=sel_gpu, pooled=pooled)
+        a = out_host[torch.as_tensor(rows)].double().numpy()
+        b = res["out"]
+        d = np.abs(a - b)
+        wide = res["gap"] >= 1e-3
+        parity = {"rows": int(len(rows)), "max_abs": float(d.max()), "mean_abs": float(d.mean()),
+                  "rel_l2": float(np.linalg.norm(a - b) / np.linalg.norm(b)),
+                  "sel_valid_frac": float(res["sel_valid"].mean()),
+                  "sel_exact_where_gap_ge_1e-3": float(res["sel_exact"][wide].mean()) if wide.any() else None,
+                  "sel_exact_frac": float(res["sel_exact"].mean())}
+
+    l2 = (f"inputs larger than L2 ({in_bytes / 1e9:.1f} GB of Q/K/V)" if big else
+          "L2 flushed between steps (256 MB write, outside the per-kernel events)")
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded scene model, random projections)",
+        "config": workload_config(wl, l2), "roofline": roofline, "stages": stages, "cpu_baseline": cpu,
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk, "dense_baseline": dense, "parity": parity,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del layer
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

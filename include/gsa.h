@@ -185,6 +185,30 @@ gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
                        const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
                        size_t ws_bytes, void* stream);
 
+/*
+ * gsa_forward with per-kernel timing: `events` is NULL or GSA_FORWARD_STEPS + 1
+ * cudaEvent_t handles created by the caller; events[0] is recorded on `stream`
+ * before the first kernel and events[i+1] after step i, the steps being
+ *   0 pooling, 1 compressed attention, 2 S_guide block scores with the
+ *   streaming top-K, 3 top-K merge, 4 selected attention with the gate.
+ * A step fused into the previous one records an empty interval.  If
+ * `n_launched` is not NULL it receives the number of kernels enqueued.
+ */
+#define GSA_FORWARD_STEPS 5
+gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                             const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
+                             size_t ws_bytes, void* const* events, int32_t* n_launched,
+                             void* stream);
+
+/* Byte offsets of gsa_forward's intermediates inside its workspace (host only),
+ * for inspecting them after a call: the buffers of gsa_pool_kv (qc32, kc32, vc,
+ * qc, kc, ks, vs), oc, the candidates (n_split lists per row) and sel. */
+typedef struct {
+  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cand_score, cand_idx, sel, total;
+  int32_t n_split;
+} gsa_ws_offsets;
+gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out);
+
 /* Synchronise `stream`, read the device error word in `ws`, clear it, and
  * return GSA_OK, GSA_ERR_TIMEOUT or GSA_ERR_DEVICE_CHECK. */
 gsa_status gsa_check_device_error(void* ws, void* stream);

@@ -388,7 +388,7 @@ def combine(g_rows: np.ndarray, o_cmp_up: np.ndarray, o_sel: np.ndarray) -> np.n
 
 
 def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
-              tie_window: float = 1e-3, chunk_elems: int = 50_000_000) -> dict:
+              tie_window: float = 1e-3, chunk_elems: int = 50_000_000, pooled=None) -> dict:
     """The GSA layer for fine query tokens ``rows`` (all tokens when None).
 
     Returns a dict of float64 arrays:
@@ -403,11 +403,15 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     S_guide scores: ``sel_exact`` [entries,H] says it equals the oracle's own
     top-K, ``sel_valid`` [entries,H] that it is a top-K up to ``tie_window``
     (no unchosen block beats a chosen one by ``tie_window`` or more).
+
+    ``pooled`` = (pool(Q), pool(K), pool(V)) from an earlier call on the same
+    inputs skips recomputing step 1.
     """
     rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
-    Qc = pool(geo, Q)
-    Kc = pool(geo, K)
-    Vc = pool(geo, V)
+    if pooled is None:
+        Qc, Kc, Vc = pool(geo, Q), pool(geo, K), pool(geo, V)
+    else:
+        Qc, Kc, Vc = pooled
     entries = np.array(sorted({geo.entry_of_token(int(t)) for t in rows}), dtype=np.int64)
     nE = entries.size
     o_cmp = np.empty((nE, geo.H, geo.D))

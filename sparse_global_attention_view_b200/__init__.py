@@ -4,7 +4,7 @@ The compute lives in ``lib/libgsa.so`` (CUDA for sm_100a, C ABI in
 ``include/gsa.h``); this package is its Python binding.
 """
 
-from ._lib import GsaError, GsaShape, GsaSizes, LIB_PATH, load  # noqa: F401
+from ._lib import FORWARD_STEPS, GsaError, GsaShape, GsaSizes, LIB_PATH, load  # noqa: F401
 from .api import (  # noqa: F401
     GsaLayer,
     Shape,
@@ -13,10 +13,13 @@ from .api import (  # noqa: F401
     dense_global_attn,
     derive,
     forward,
+    forward_timed,
     gate_combine,
     new_workspace,
     pool_kv,
     selected_attn,
     topk_blocks,
+    workspace_offsets,
     workspace_size,
+    workspace_view,
 )

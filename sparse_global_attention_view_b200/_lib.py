@@ -54,6 +54,13 @@ class GsaSizes(ctypes.Structure):
     ]
 
 
+class GsaWsOffsets(ctypes.Structure):
+    _fields_ = [(n, c_size) for n in ("qc32", "kc32", "vc", "qc", "kc", "ks", "vs", "oc",
+                                      "cand_score", "cand_idx", "sel", "total")] + [("n_split", c_i32)]
+
+
+FORWARD_STEPS = ("pool", "compressed_attn", "block_scores", "topk_merge", "selected_gate")
+
 P_SHAPE = ctypes.POINTER(GsaShape)
 
 # name -> argument types (all return gsa_status, an int, except gsa_status_string)
@@ -68,6 +75,8 @@ SIGNATURES = {
     "gsa_gate_combine": [P_SHAPE] + [c_vp] * 7,
     "dense_global_attn": [P_SHAPE] + [c_vp] * 6,
     "gsa_forward": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp],
+    "gsa_forward_timed": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp, ctypes.POINTER(c_i32), c_vp],
+    "gsa_workspace_offsets": [P_SHAPE, ctypes.POINTER(GsaWsOffsets)],
     "gsa_check_device_error": [c_vp, c_vp],
     "gsa_status_string": [c_i32],
 }

@@ -13,7 +13,7 @@ from dataclasses import dataclass
 
 import torch
 
-from ._lib import GsaShape, GsaSizes, WS_HEADER_BYTES, check, load
+from ._lib import FORWARD_STEPS, GsaShape, GsaSizes, GsaWsOffsets, WS_HEADER_BYTES, check, load
 
 BF16 = torch.bfloat16
 F32 = torch.float32
@@ -170,6 +170,52 @@ def forward(shape, q, k, v, w, out, ws, stream=None):
         ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
         _ptr(w, F32, shape.n_heads * shape.head_dim, "w"), _ptr(out, BF16, tok, "out"), _ws(ws, need),
         ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)), "gsa_forward")
+
+
+def forward_timed(shape, q, k, v, w, out, ws, events, stream=None) -> int:
+    """``forward`` recording ``events`` (len(FORWARD_STEPS) + 1 torch.cuda.Event
+    with timing, already recorded once so their handles exist) between its
+    kernels; returns the number of kernels enqueued."""
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    need = workspace_size(shape)
+    if len(events) != len(FORWARD_STEPS) + 1:
+        raise ValueError(f"need {len(FORWARD_STEPS) + 1} events")
+    handles = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    n = ctypes.c_int32()
+    check(load().gsa_forward_timed(
+        ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(w, F32, shape.n_heads * shape.head_dim, "w"), _ptr(out, BF16, tok, "out"), _ws(ws, need),
+        ctypes.c_size_t(ws.numel() * ws.element_size()), handles, ctypes.byref(n), _stream(stream)),
+        "gsa_forward_timed")
+    return n.value
+
+
+def workspace_offsets(shape) -> GsaWsOffsets:
+    o = GsaWsOffsets()
+    check(load().gsa_workspace_offsets(ctypes.byref(shape.c()), ctypes.byref(o)), "gsa_workspace_offsets")
+    return o
+
+
+def workspace_view(ws, shape, name: str) -> torch.Tensor:
+    """A typed view of one of gsa_forward's intermediates inside ``ws``."""
+    z = derive(shape)
+    o = workspace_offsets(shape)
+    H, D, K = shape.n_heads, shape.head_dim, shape.top_k
+    spec = {
+        "qc32": (F32, (z.Tc, H, D)), "kc32": (F32, (z.Tc, H, D)), "vc": (BF16, (z.Tc, H, D)),
+        "qc": (BF16, (z.Tc, H, D)), "kc": (BF16, (z.Tc, H, D)), "ks": (BF16, (H, z.NS, D)),
+        "vs": (BF16, (H, z.NS, D)), "oc": (F32, (z.Tc, H, D)),
+        "cand_score": (F32, (H, z.Tc, o.n_split, K)), "cand_idx": (I32, (H, z.Tc, o.n_split, K)),
+        "sel": (I32, (H, z.Tc, K)),
+    }[name]
+    dtype, shp = spec
+    n = 1
+    for s in shp:
+        n *= s
+    off = getattr(o, name)
+    nbytes = n * torch.tensor([], dtype=dtype).element_size()
+    return ws[off:off + nbytes].view(dtype).view(shp)
 
 
 def check_device_error(ws, stream=None) -> None:

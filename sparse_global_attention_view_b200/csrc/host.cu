@@ -265,14 +265,18 @@ gsa_status dense_global_attn(const gsa_shape* shape, const gsa_bf16* q, const gs
   return cuda_status(gsa::launch_attn_mma(a, as_stream(stream)));
 }
 
-gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
-                       const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
-                       size_t ws_bytes, void* stream) {
+gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                             const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
+                             size_t ws_bytes, void* const* events, int32_t* n_launched,
+                             void* stream) {
   Dims d;
   gsa_status st = make_dims(shape, &d, nullptr);
   if (st != GSA_OK) return st;
   if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(w) || !dev_ptr(out) || !dev_ptr(ws))
     return GSA_ERR_INVALID_ARG;
+  if (events != nullptr)
+    for (int i = 0; i <= GSA_FORWARD_STEPS; ++i)
+      if (events[i] == nullptr) return GSA_ERR_INVALID_ARG;
   const Layout l = forward_layout(d);
   if (ws_bytes < l.total) return GSA_ERR_WORKSPACE;
   char* base = static_cast<char*>(ws);
@@ -288,17 +292,69 @@ gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
   int* ci = (int*)(base + l.ci);
   int* sel = (int*)(base + l.sel);
   cudaStream_t s = as_stream(stream);
-  cudaError_t e = gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32,
-                                   vc, qc, kc, ks, vs, s);
-  if (e != cudaSuccess) return GSA_ERR_CUDA;
-  st = gsa_compressed_attn(shape, (const gsa_bf16*)qc, (const gsa_bf16*)kc, (const gsa_bf16*)vc,
-                           qc32, kc32, oc, cs, ci, l.n_split, ws, stream);
+  int launched = 0;
+  auto mark = [&](int i) -> bool {
+    return events == nullptr || cudaEventRecord((cudaEvent_t)events[i], s) == cudaSuccess;
+  };
+  auto step = [&](cudaError_t e, int i) -> bool {
+    ++launched;
+    return e == cudaSuccess && mark(i);
+  };
+  if (!mark(0)) return GSA_ERR_CUDA;
+  if (!step(gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32, vc, qc,
+                             kc, ks, vs, s), 1))
+    return GSA_ERR_CUDA;
+  gsa::AttnArgs a;
+  a.q = qc;
+  a.k = kc;
+  a.v = vc;
+  a.q_row = a.kv_row = a.o_row = (long long)d.H * gsa::kHeadDim;
+  a.q_head = a.kv_head = a.o_head = gsa::kHeadDim;
+  a.n_q = a.n_k = d.Tc;
+  a.o = oc;
+  a.o_f32 = true;
+  a.lse = nullptr;
+  a.lse_row = a.lse_head = 0;
+  a.H = d.H;
+  a.scale = d.scale;
+  a.scale_log2 = d.scale_log2;
+  if (!step(gsa::launch_attn_mma(a, s), 2)) return GSA_ERR_CUDA;
+  if (!step(gsa::launch_block_scores_topk(d, qc32, kc32, cs, ci, l.n_split, s), 3)) return GSA_ERR_CUDA;
+  if (!step(gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s), 4)) return GSA_ERR_CUDA;
+  if (!step(gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, ks, vs, sel, qc32,
+                                 w, oc, (bf16*)out, nullptr, (unsigned*)ws, s),
+            5))
+    return GSA_ERR_CUDA;
+  if (n_launched) *n_launched = launched;
+  return GSA_OK;
+}
+
+gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                       const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
+                       size_t ws_bytes, void* stream) {
+  return gsa_forward_timed(shape, q, k, v, w, out, ws, ws_bytes, nullptr, nullptr, stream);
+}
+
+gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out) {
+  Dims d;
+  if (out == nullptr) return GSA_ERR_INVALID_ARG;
+  gsa_status st = make_dims(shape, &d, nullptr);
   if (st != GSA_OK) return st;
-  e = gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s);
-  if (e != cudaSuccess) return GSA_ERR_CUDA;
-  e = gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, ks, vs, sel, qc32, w,
-                           oc, (bf16*)out, nullptr, (unsigned*)ws, s);
-  return cuda_status(e);
+  const Layout l = forward_layout(d);
+  out->qc32 = l.qc32;
+  out->kc32 = l.kc32;
+  out->vc = l.vc;
+  out->qc = l.qc;
+  out->kc = l.kc;
+  out->ks = l.ks;
+  out->vs = l.vs;
+  out->oc = l.oc;
+  out->cand_score = l.cs;
+  out->cand_idx = l.ci;
+  out->sel = l.sel;
+  out->total = l.total;
+  out->n_split = l.n_split;
+  return GSA_OK;
 }
 
 gsa_status gsa_check_device_error(void* ws, void* stream) {

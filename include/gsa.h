@@ -64,7 +64,8 @@ typedef enum {
   GSA_ERR_WORKSPACE = 3,     /* workspace smaller than required */
   GSA_ERR_CUDA = 4,          /* a CUDA launch or runtime call failed */
   GSA_ERR_TIMEOUT = 5,       /* device error word: a bounded wait ran out */
-  GSA_ERR_DEVICE_CHECK = 6   /* device error word: an in-kernel bounds check failed */
+  GSA_ERR_DEVICE_CHECK = 6,  /* device error word: an in-kernel bounds check failed */
+  GSA_ERR_SCRATCH_LIMIT = 7  /* gsa_forward_noalloc: the shape needs more than its fixed scratch */
 } gsa_status;
 
 /* One layer call's sizes.  All fields are read by every entry point. */
@@ -208,6 +209,35 @@ typedef struct {
   int32_t n_split;
 } gsa_ws_offsets;
 gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out);
+
+/*
+ * gsa_forward without a workspace argument, for callers that cannot allocate
+ * device memory.  (The Speed3R pages have no counterpart: this is a deployment
+ * variant of gsa_forward.)  Some host programs may not call cudaMalloc at all:
+ * applications whose own memory manager owns every byte of device memory and
+ * forbids allocations it does not make, or latency-critical loops where a
+ * cudaMalloc/cudaFree would synchronise the device.  Such callers still pass
+ * q, k, v, w and out, which they own; the layer's intermediates go to one
+ * fixed array of GSA_NOALLOC_SCRATCH_BYTES in the library's device memory,
+ * which every GPU that loads the library holds until the process exits.
+ *
+ * - Shapes whose gsa_workspace_size exceeds GSA_NOALLOC_SCRATCH_BYTES are
+ *   rejected with GSA_ERR_SCRATCH_LIMIT before any work is enqueued (the
+ *   32 MiB array fits up to about the 8-frame VGGT layout: 8 x (5 + 37x37)
+ *   tokens, 16 heads, K = 16).
+ * - The first call on each device looks up the array's device address (with
+ *   that device current) and caches it; make that first call before any
+ *   stream capture.
+ * - Every call on a device shares the one array and leaves its intermediates
+ *   in it.  Each call zeroes the array's error-word header first.  Calls that
+ *   overlap on the GPU (on different streams, or from several host threads
+ *   without ordering) race on the array and corrupt each other's results:
+ *   order them.
+ * - Allocates nothing: no cudaMalloc / cudaFree and no allocating library call.
+ */
+#define GSA_NOALLOC_SCRATCH_BYTES (32u << 20)
+gsa_status gsa_forward_noalloc(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                               const gsa_bf16* v, const float* w, gsa_bf16* out, void* stream);
 
 /* Synchronise `stream`, read the device error word in `ws`, clear it, and
  * return GSA_OK, GSA_ERR_TIMEOUT or GSA_ERR_DEVICE_CHECK. */

@@ -13,6 +13,7 @@ from .api import (  # noqa: F401
     dense_global_attn,
     derive,
     forward,
+    forward_noalloc,
     forward_timed,
     gate_combine,
     new_workspace,

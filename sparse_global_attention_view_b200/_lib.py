@@ -21,7 +21,9 @@ STATUS_NAMES = {
     4: "GSA_ERR_CUDA",
     5: "GSA_ERR_TIMEOUT",
     6: "GSA_ERR_DEVICE_CHECK",
+    7: "GSA_ERR_SCRATCH_LIMIT",
 }
+NOALLOC_SCRATCH_BYTES = 32 << 20
 WS_HEADER_BYTES = 256
 
 
@@ -77,6 +79,7 @@ SIGNATURES = {
     "gsa_forward": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp],
     "gsa_forward_timed": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp, ctypes.POINTER(c_i32), c_vp],
     "gsa_workspace_offsets": [P_SHAPE, ctypes.POINTER(GsaWsOffsets)],
+    "gsa_forward_noalloc": [P_SHAPE] + [c_vp] * 6,
     "gsa_check_device_error": [c_vp, c_vp],
     "gsa_status_string": [c_i32],
 }

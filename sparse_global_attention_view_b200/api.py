@@ -172,6 +172,18 @@ def forward(shape, q, k, v, w, out, ws, stream=None):
         ctypes.c_size_t(ws.numel() * ws.element_size()), _stream(stream)), "gsa_forward")
 
 
+def forward_noalloc(shape, q, k, v, w, out, stream=None) -> None:
+    """``forward`` without a workspace: the intermediates use the library's
+    fixed device array (for callers that cannot allocate; see gsa.h).  Calls
+    on one device share that array, so they must not overlap on the GPU."""
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    check(load().gsa_forward_noalloc(
+        ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(w, F32, shape.n_heads * shape.head_dim, "w"), _ptr(out, BF16, tok, "out"), _stream(stream)),
+        "gsa_forward_noalloc")
+
+
 def forward_timed(shape, q, k, v, w, out, ws, events, stream=None) -> int:
     """``forward`` recording ``events`` (len(FORWARD_STEPS) + 1 torch.cuda.Event
     with timing, already recorded once so their handles exist) between its

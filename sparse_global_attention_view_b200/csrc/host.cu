@@ -127,6 +127,9 @@ const char* gsa_status_string(gsa_status s) {
     case GSA_ERR_CUDA: return "CUDA error";
     case GSA_ERR_TIMEOUT: return "device wait timed out";
     case GSA_ERR_DEVICE_CHECK: return "device-side check failed";
+    case GSA_ERR_SCRATCH_LIMIT:
+      return "shape needs more scratch than gsa_forward_noalloc's fixed device array "
+             "(GSA_NOALLOC_SCRATCH_BYTES); use gsa_forward with a workspace";
   }
   return "unknown status";
 }

@@ -33,6 +33,7 @@ def declared_functions():
 
 def declared_arity():
     text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"^\s*#.*$", "", text, flags=re.M)  # preprocessor lines
     out = {}
     for m in re.finditer(r"([A-Za-z_]\w*)\s*\(([^;{]*?)\)\s*;", text):
         args = m.group(2).strip()
@@ -139,8 +140,19 @@ def test_small_workspace_is_rejected(lib):
                            ctypes.c_void_p(0)) == 3
 
 
+def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
+    from sparse_global_attention_view_b200 import workspace_size
+    from sparse_global_attention_view_b200._lib import NOALLOC_SCRATCH_BYTES
+    big = shape(n_frames=100, top_k=32)
+    assert workspace_size(big) > NOALLOC_SCRATCH_BYTES
+    p = ctypes.c_void_p(FAKE)
+    # rejected on the host before any CUDA call
+    assert lib.gsa_forward_noalloc(ctypes.byref(big.c()), p, p, p, p, p, ctypes.c_void_p(0)) == 7
+    assert b"noalloc" in lib.gsa_status_string(7)
+
+
 def test_status_strings(lib):
-    for code in range(7):
+    for code in range(8):
         assert lib.gsa_status_string(code)
     assert b"unknown" in lib.gsa_status_string(99)
 

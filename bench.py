@@ -230,6 +230,25 @@ def recorded_traffic(kernel_file: str, workload: str):
     return None
 
 
+def rank_workload(wl, rank: int):
+    """Rank r > 0 runs an independent scene of the same size (seed + 1000 r)."""
+    return wl if rank == 0 else wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def reduce_max(value: float, dist, device) -> float:
+    """Max of ``value`` over all ranks (identity without a process group)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world: int, tokens_per_rank: int, step_ms_max: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
+    return world * tokens_per_rank / (step_ms_max / 1e3)
+
+
 STAGE_SOURCE = {"pool": "pool.cu", "compressed_attn": "attn_mma.cu", "block_scores": "topk.cu",
                 "topk_merge": "topk.cu", "selected_gate": "selected.cu"}
 
@@ -270,15 +289,9 @@ def main() -> None:
             dist.barrier()
 
     def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(v, dist, torch.device("cuda", local))
 
-    wl = WORKLOADS[args.workload]
-    if rank:
-        wl = wl.with_(seed=wl.seed + 1000 * rank)  # an independent scene per rank
+    wl = rank_workload(WORKLOADS[args.workload], rank)
     x = generate(wl)
     shape = G.Shape.of(wl)
     z = G.derive(shape)
@@ -333,7 +346,7 @@ def main() -> None:
     step_ms_local = (start.elapsed_time(stop) / args.steps) if flush is None else \
         statistics.mean(sum(r) for r in per_step)
     step_ms = max_over_ranks(step_ms_local)
-    value = world * z.T / (step_ms / 1e3)
+    value = job_value(world, z.T, step_ms)
 
     # ---- per-stage roofline from the same timed steps ----
     P = peaks()
@@ -389,7 +402,7 @@ def main() -> None:
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hw))
     d2h = hout.numel() * hout.element_size()
-    e2e = {"value": world * z.T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    e2e = {"value": job_value(world, z.T, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
            "path": "pinned host Q/K/V/w -> device, gsa_forward, device -> pinned host out"}
 
@@ -409,7 +422,7 @@ def main() -> None:
         barrier()
         dms = max_over_ranks(d0.elapsed_time(d1) / args.dense_steps)
         tf = dense_flops(z, H, D) / (dms / 1e3) / 1e12
-        dense = {"ms_per_layer": round(dms, 3), "tokens_per_s": world * z.T / (dms / 1e3),
+        dense = {"ms_per_layer": round(dms, 3), "tokens_per_s": job_value(world, z.T, dms),
                  "tflops": round(tf, 1), "frac_bf16_peak": round(tf / P["bf16_tflops"], 4),
                  "gsa_speedup": round(dms / step_ms, 2), "kernel": "mma.sync m16n8k16 flash attention",
                  "steps": args.dense_steps}

@@ -172,10 +172,20 @@ gsa_status gsa_gate_combine(const gsa_shape* shape, const float* qc32, const flo
 /*
  * Dense global attention (technical summary 1: the quadratic all-to-all
  * attention GSA replaces): out = softmax(scale * q k^T) v over all T tokens,
- * per head.  Uses n_frames, n_special, hp, wp, n_heads, head_dim, scale.
+ * per head, on tcgen05/TMEM fed by TMA.  Uses n_frames, n_special, hp, wp,
+ * n_heads, head_dim, scale.  A wait that runs out of time sets GSA_ERR_TIMEOUT
+ * in the workspace's error word (see gsa_check_device_error).
  */
 gsa_status dense_global_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
                              const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream);
+
+/*
+ * dense_global_attn on the warp-level tensor-core instruction (mma.sync
+ * m16n8k16), the pre-tcgen05 path; kept as a measured baseline for the
+ * tcgen05 kernel.  Same arguments and result.
+ */
+gsa_status dense_global_attn_mma(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                                 const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream);
 
 /*
  * The whole GSA layer: steps 1-6 enqueued on `stream`, intermediates in `ws`

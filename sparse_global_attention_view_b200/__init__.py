@@ -11,6 +11,7 @@ from .api import (  # noqa: F401
     check_device_error,
     compressed_attn,
     dense_global_attn,
+    dense_global_attn_mma,
     derive,
     forward,
     forward_noalloc,

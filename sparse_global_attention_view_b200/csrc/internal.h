@@ -32,6 +32,23 @@ struct AttnArgs {
 };
 cudaError_t launch_attn_mma(const AttnArgs& a, cudaStream_t st);
 
+// Attention on tcgen05/TMEM fed by TMA.  Q is token-major [n_q][H][64]; K/V are
+// token-major [kv_rows][H][64] or, with kv_head_major, [H][kv_rows][64].
+struct AttnTcArgs {
+  long long n_q, n_k;
+  int H;
+  float c2;  // softmax scale * log2(e)
+  void* out;
+  int out_f32;
+  long long o_row, o_head;
+  float* lse;  // nullable: natural-log sum of exp of the scaled logits
+  long long lse_row, lse_head;
+  unsigned* err;  // device error word
+  int kv_head_major;
+};
+cudaError_t launch_attn_tc(const AttnTcArgs& a, const bf16* q, const bf16* k, const bf16* v,
+                           long long kv_rows, cudaStream_t st);
+
 cudaError_t launch_block_scores_topk(const Dims& d, const float* qc32, const float* kc32,
                                      float* cand_score, int* cand_idx, int n_split,
                                      cudaStream_t st);

@@ -30,6 +30,8 @@ CASES = {
     "p2_onehead": Workload("p2_onehead", 4, 1, 9, 9, 1, 64, 2, 7, 10, "gaussian"),
     # one VGGT-shaped frame
     "one_frame": Workload("one_frame", 1, 5, 37, 37, 4, 64, 4, 16, 11, "gaussian"),
+    # nine tokens: a single, mostly empty 128-row query tile and key tile
+    "nine_tokens": Workload("nine_tokens", 1, 3, 2, 3, 2, 64, 2, 2, 12, "gaussian"),
 }
 
 _cache = {}
@@ -125,7 +127,7 @@ def test_forward(name):
     assert torch.equal(out1, out2), "forward must be deterministic"
 
 
-@pytest.mark.parametrize("name", ["tiny", "p3_ragged", "p1_nospecial", "k_all", "p2_onehead"])
+@pytest.mark.parametrize("name", ["tiny", "p3_ragged", "p1_nospecial", "k_all", "p2_onehead", "nine_tokens"])
 def test_dense_full(name):
     import sparse_global_attention_view_b200 as G
     x, geo, shape, st, res = case(name)
@@ -134,6 +136,15 @@ def test_dense_full(name):
     ref = O.dense_attention(geo, x.q, x.k, x.v)
     assert PT.zeros_fail(ref)
     PT.assert_close(out, ref, f"{name} dense")
+
+
+@pytest.mark.parametrize("name", ["tiny", "p3_ragged", "nine_tokens"])
+def test_dense_warp_mma_baseline(name):
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    out = torch.full_like(st.q, float("nan"))
+    G.dense_global_attn_mma(shape, st.q, st.k, st.v, out, st.ws)
+    PT.assert_close(out, O.dense_attention(geo, x.q, x.k, x.v), f"{name} dense (mma.sync)")
 
 
 @pytest.mark.parametrize("name", ["small", "one_frame"])

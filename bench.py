@@ -67,8 +67,11 @@ def stage_work(z, H, D, K_eff) -> dict:
         "block_scores": ("alu", 2 * Tc * NB * H * D, "flop"),
         # candidates read once, selection written once
         "topk_merge": ("hbm", H * Tc * K_eff * 8 + H * Tc * K_eff * 4, "bytes"),
-        # QK^T and PV of every token over the specials plus K_eff blocks of (at most) 16 tokens
-        "selected_gate": ("tensor", 4 * T * H * D * (NS + 16 * K_eff), "flop"),
+        # QK^T and PV of every token over all N*S special tokens
+        "specials_attn": ("tensor", 4 * T * NS * H * D, "flop"),
+        # the selected blocks' K and V gathered per (entry, head): K_eff blocks of
+        # (at most) 16 tokens x 128 bytes, K and V
+        "selected_gate": ("hbm", H * Tc * K_eff * 16 * D * 2 * 2, "bytes"),
     }
 
 
@@ -249,8 +252,8 @@ def job_value(world: int, tokens_per_rank: int, step_ms_max: float) -> float:
     return world * tokens_per_rank / (step_ms_max / 1e3)
 
 
-STAGE_SOURCE = {"pool": "pool.cu", "compressed_attn": "attn_mma.cu", "block_scores": "topk.cu",
-                "topk_merge": "topk.cu", "selected_gate": "selected.cu"}
+STAGE_SOURCE = {"pool": "pool.cu", "compressed_attn": "attn_cmp_tc.cu", "block_scores": "topk.cu",
+                "topk_merge": "topk.cu", "specials_attn": "attn_tc.cu", "selected_gate": "selected.cu"}
 
 
 def main() -> None:
@@ -352,6 +355,9 @@ def main() -> None:
     P = peaks()
     work = stage_work(z, H, D, min(shape.top_k, z.NB))
     alu_peak = SM_COUNT * FFMA_PER_SM_PER_CLK * 2 * P["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s fp32 FMA
+    # the fused compressed stage does QK^T in tf32 (half the bf16 rate) and PV in
+    # bf16, equal flops each: its tensor peak is 2/3 of the bf16 peak
+    fused_cmp = stage_ms["block_scores"] < 0.01 * stage_ms["compressed_attn"]
     stages = {}
     for name in G.FORWARD_STEPS:
         bound, amount, unit = work[name]
@@ -362,8 +368,12 @@ def main() -> None:
             ach, peak, u = amount / (ms / 1e3) / 1e9, P["hbm_gbs"], "GB/s"
         elif bound == "tensor":
             ach, peak, u = amount / (ms / 1e3) / 1e12, P["bf16_tflops"], "TFLOP/s"
+            if name == "compressed_attn" and fused_cmp:
+                peak = P["bf16_tflops"] * 2.0 / 3.0
         else:
             ach, peak, u = amount / (ms / 1e3) / 1e12, alu_peak, "TFLOP/s"
+        if ms < 0.005:
+            continue  # fused into the previous step
         stages[name] = {"ms": round(ms, 4), "share": round(ms / sum(stage_ms.values()), 4), "bound": bound,
                         "achieved": round(ach, 2), "peak": round(peak, 1), "unit": u,
                         "frac": round(ach / peak, 4)}
@@ -424,7 +434,7 @@ def main() -> None:
         tf = dense_flops(z, H, D) / (dms / 1e3) / 1e12
         dense = {"ms_per_layer": round(dms, 3), "tokens_per_s": job_value(world, z.T, dms),
                  "tflops": round(tf, 1), "frac_bf16_peak": round(tf / P["bf16_tflops"], 4),
-                 "gsa_speedup": round(dms / step_ms, 2), "kernel": "mma.sync m16n8k16 flash attention",
+                 "gsa_speedup": round(dms / step_ms, 2), "kernel": "tcgen05/TMEM + TMA flash attention",
                  "steps": args.dense_steps}
         del dout
 

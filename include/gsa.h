@@ -190,7 +190,9 @@ gsa_status dense_global_attn_mma(const gsa_shape* shape, const gsa_bf16* q, cons
 /*
  * The whole GSA layer: steps 1-6 enqueued on `stream`, intermediates in `ws`
  * (ws_bytes >= gsa_workspace_size).  w [H][64] fp32 gate vectors; out
- * [T][H][64] bf16.  Steps 5 and 6 run fused in one kernel.
+ * [T][H][64] bf16.  The attention over the always-kept special tokens runs on
+ * the tensor-core attention kernel into the workspace; the selected blocks
+ * continue that softmax in the step-5 kernel, which also applies the gate.
  */
 gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
                        const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
@@ -201,11 +203,14 @@ gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
  * cudaEvent_t handles created by the caller; events[0] is recorded on `stream`
  * before the first kernel and events[i+1] after step i, the steps being
  *   0 pooling, 1 compressed attention, 2 S_guide block scores with the
- *   streaming top-K, 3 top-K merge, 4 selected attention with the gate.
- * A step fused into the previous one records an empty interval.  If
- * `n_launched` is not NULL it receives the number of kernels enqueued.
+ *   streaming top-K, 3 top-K merge, 4 attention of every token over the
+ *   special tokens, 5 attention over the selected blocks, merged with step
+ *   4, with the gate.
+ * A step fused into another one (or absent, such as step 4 without special
+ * tokens) records an empty interval.  If `n_launched` is not NULL it receives
+ * the number of kernels enqueued.
  */
-#define GSA_FORWARD_STEPS 5
+#define GSA_FORWARD_STEPS 6
 gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
                              const gsa_bf16* v, const float* w, gsa_bf16* out, void* ws,
                              size_t ws_bytes, void* const* events, int32_t* n_launched,
@@ -213,9 +218,11 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
 
 /* Byte offsets of gsa_forward's intermediates inside its workspace (host only),
  * for inspecting them after a call: the buffers of gsa_pool_kv (qc32, kc32, vc,
- * qc, kc, ks, vs), oc, the candidates (n_split lists per row) and sel. */
+ * qc, kc, ks, vs), oc, the candidates (n_split lists per row), sel, and the
+ * special-token segment's fp32 output [T][H][64] and lse [T][H] (empty when
+ * S == 0). */
 typedef struct {
-  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cand_score, cand_idx, sel, total;
+  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cand_score, cand_idx, sel, o_spec, lse_spec, total;
   int32_t n_split;
 } gsa_ws_offsets;
 gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out);
@@ -233,7 +240,7 @@ gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out);
  *
  * - Shapes whose gsa_workspace_size exceeds GSA_NOALLOC_SCRATCH_BYTES are
  *   rejected with GSA_ERR_SCRATCH_LIMIT before any work is enqueued (the
- *   32 MiB array fits up to about the 8-frame VGGT layout: 8 x (5 + 37x37)
+ *   32 MiB array fits the VGGT token layout up to 4 frames: 4 x (5 + 37x37)
  *   tokens, 16 heads, K = 16).
  * - The first call on each device looks up the array's device address (with
  *   that device current) and caches it; make that first call before any

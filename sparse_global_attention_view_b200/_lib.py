@@ -58,10 +58,11 @@ class GsaSizes(ctypes.Structure):
 
 class GsaWsOffsets(ctypes.Structure):
     _fields_ = [(n, c_size) for n in ("qc32", "kc32", "vc", "qc", "kc", "ks", "vs", "oc",
-                                      "cand_score", "cand_idx", "sel", "total")] + [("n_split", c_i32)]
+                                      "cand_score", "cand_idx", "sel", "o_spec", "lse_spec",
+                                      "total")] + [("n_split", c_i32)]
 
 
-FORWARD_STEPS = ("pool", "compressed_attn", "block_scores", "topk_merge", "selected_gate")
+FORWARD_STEPS = ("pool", "compressed_attn", "block_scores", "topk_merge", "specials_attn", "selected_gate")
 
 P_SHAPE = ctypes.POINTER(GsaShape)
 

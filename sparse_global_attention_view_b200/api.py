@@ -229,6 +229,7 @@ def workspace_view(ws, shape, name: str) -> torch.Tensor:
         "vs": (BF16, (H, z.NS, D)), "oc": (F32, (z.Tc, H, D)),
         "cand_score": (F32, (H, z.Tc, o.n_split, K)), "cand_idx": (I32, (H, z.Tc, o.n_split, K)),
         "sel": (I32, (H, z.Tc, K)),
+        "o_spec": (F32, (z.T if z.NS else 0, H, D)), "lse_spec": (F32, (z.T if z.NS else 0, H)),
     }[name]
     dtype, shp = spec
     n = 1

@@ -1,0 +1,423 @@
+// Attention in the pooled sequence fused with the S_guide streaming top-K
+// (Speed3R technical summary 2.1: compression branch and selection branch;
+// 2.2: a streaming top-K inside the attention loop, no score matrix in memory).
+//
+// One CTA = one 128-row tile of compressed queries of one head, 12 warps:
+//   warp 0      TMA producer: the fp32 pooled query tile once, then a 2-stage
+//               ring of 128-entry key tiles (fp32 pooled K, bf16 pooled V);
+//   warp 1      MMA issuer: S = Qc Kc^T with kind::tf32 from the fp32 means
+//               (the top-K ranking needs better than bf16 scores), into one of
+//               two TMEM score buffers, then O += P Vc (bf16, P from TMEM);
+//   warp 2      TMEM allocation (S at columns 0/128, O at 256, P at 320/384);
+//   warps 4-7   softmax, one thread per query row;
+//   warps 8-11  streaming top-K, one thread per query row.
+// S(j+1) is computed while both warpgroups work on S(j): the softmax writes
+// P(j) to its own TMEM columns, so the raw scores stay readable until the
+// top-K warpgroup has loaded them.  Each top-K thread scans its row's raw
+// scores in registers: 16-column chunks whose maximum beats the row's current
+// K-th best score are
+// appended to a per-thread candidate buffer in shared memory; candidates that
+// are patch blocks (special entries are never ranked) enter a per-row min-heap
+// of (score, block id) ordered worst-first by (score ascending, id
+// descending).  Columns arrive in ascending block order and only a strictly
+// larger score displaces the root, so equal scores keep the lower block id.
+#include <math_constants.h>
+
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace gsa {
+namespace {
+
+using namespace tc;
+
+constexpr int TQ = 128;
+constexpr int TK = 128;
+constexpr int ST = 2;
+constexpr int kThreads = 384;
+constexpr int kMaxK = 64;        // heap capacity per row
+constexpr int kChunk = 16;       // columns per candidate scan chunk
+constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16) tile: 16 KB
+
+constexpr uint32_t OFF_Q = 0;                        // 2 sub-tiles (d 0-31, 32-63)
+constexpr uint32_t OFF_K = OFF_Q + 2 * kSub;         // ST x 2 sub-tiles
+constexpr uint32_t OFF_V = OFF_K + ST * 2 * kSub;    // ST x bf16 tile
+constexpr uint32_t OFF_HS = OFF_V + ST * kSub;       // heap scores [kMaxK][128]
+constexpr uint32_t OFF_HI = OFF_HS + kMaxK * TQ * 4; // heap ids
+constexpr uint32_t OFF_CS = OFF_HI + kMaxK * TQ * 4; // candidate scores [kChunk][128]
+constexpr uint32_t OFF_CC = OFF_CS + kChunk * TQ * 4;// candidate columns
+constexpr uint32_t OFF_BAR = OFF_CC + kChunk * TQ * 4;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;
+constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
+
+constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + ST, B_KVE = B_VF + ST, B_SF = B_KVE + ST,
+              B_PF = B_SF + 2, B_SR = B_PF + 2, B_OD = B_SR + 2, B_OF = B_OD + 1, B_DRAIN = B_OF + 1,
+              B_COUNT = B_DRAIN + 1;
+static_assert(B_COUNT * 8 <= 256, "barrier area");
+constexpr uint32_t kCols = 512;
+
+struct Heap {
+  float* hs;
+  int* hi;
+  int r, K, cnt;
+  float tau;  // raw score a candidate must beat (-inf until the heap is full)
+
+  __device__ __forceinline__ bool worse(float s1, int i1, float s2, int i2) const {
+    return s1 < s2 || (s1 == s2 && i1 > i2);
+  }
+  __device__ __forceinline__ void sift(int p, float s, int id) {
+    while (true) {
+      int c = 2 * p + 1;
+      if (c >= K) break;
+      float cs = hs[c * TQ + r];
+      int ci = hi[c * TQ + r];
+      if (c + 1 < K) {
+        const float s2 = hs[(c + 1) * TQ + r];
+        const int i2 = hi[(c + 1) * TQ + r];
+        if (worse(s2, i2, cs, ci)) cs = s2, ci = i2, c = c + 1;
+      }
+      if (!worse(cs, ci, s, id)) break;
+      hs[p * TQ + r] = cs;
+      hi[p * TQ + r] = ci;
+      p = c;
+    }
+    hs[p * TQ + r] = s;
+    hi[p * TQ + r] = id;
+  }
+  __device__ __forceinline__ void push(float s, int id) {
+    if (cnt < K) {
+      hs[cnt * TQ + r] = s;
+      hi[cnt * TQ + r] = id;
+      if (++cnt == K) {
+        for (int p = K / 2 - 1; p >= 0; --p) sift(p, hs[p * TQ + r], hi[p * TQ + r]);
+        tau = hs[r];
+      }
+    } else {
+      sift(0, s, id);
+      tau = hs[r];
+    }
+  }
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_cmp_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const Dims d, float* __restrict__ oc,
+                       float* __restrict__ cand_s, int* __restrict__ cand_i, unsigned* err) {
+  extern __shared__ __align__(1024) uint8_t cmp_smem_raw[];
+  const uint32_t raw = smem_u32(cmp_smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sp = cmp_smem_raw + (sb - raw);
+  const uint32_t sQ = sb + OFF_Q, sK = sb + OFF_K, sV = sb + OFF_V;
+  auto bar = [&](int i) -> uint32_t { return sb + OFF_BAR + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + OFF_MISC + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y;
+  const long long m0 = (long long)blockIdx.x * TQ;
+  const long long n_k = d.Tc;
+  const int nt = (int)((n_k + TK - 1) / TK);
+
+  if (tid == 0) {
+    mbar_init(bar(B_Q), 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(bar(B_KF + s), 1);
+      mbar_init(bar(B_VF + s), 1);
+      mbar_init(bar(B_KVE + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_SF + b), 1);
+      mbar_init(bar(B_PF + b), TQ);
+      mbar_init(bar(B_SR + b), TQ);  // top-K warpgroup has read S buffer b
+    }
+    mbar_init(bar(B_OD), 1);
+    mbar_init(bar(B_OF), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), kCols);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tmap(&tq);
+      prefetch_tmap(&tk);
+      prefetch_tmap(&tv);
+      mbar_expect_tx(bar(B_Q), 2 * kSub);
+      for (int half = 0; half < 2; ++half)
+        tma_load_3d(sQ + half * kSub, &tq, bar(B_Q), 32 * half, h, (int)m0);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % ST;
+        if (j >= ST && !mbar_wait(bar(B_KVE + s), ((j / ST) - 1) & 1, abort_flag, err)) break;
+        mbar_expect_tx(bar(B_KF + s), 2 * kSub);
+        for (int half = 0; half < 2; ++half)
+          tma_load_3d(sK + (2 * s + half) * kSub, &tk, bar(B_KF + s), 32 * half, h, j * TK);
+        mbar_expect_tx(bar(B_VF + s), kSub);
+        tma_load_3d(sV + s * kSub, &tv, bar(B_VF + s), 0, h, j * TK);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        mbar_wait(bar(B_Q), 0, &never, err);
+        for (int j = issued - 1; j >= 0 && j >= issued - ST; --j) {
+          mbar_wait(bar(B_KF + j % ST), (j / ST) & 1, &never, err);
+          mbar_wait(bar(B_VF + j % ST), (j / ST) & 1, &never, err);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id_qk = idesc(128, 128, kFmtTF32, 0, 0);
+      const uint32_t id_pv = idesc(128, 64, kFmtBF16, 0, 1);
+      auto issue_s = [&](int s, int b) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+          mma_tf32_ss(tbase + b * 128, sdesc_k(sQ + off), sdesc_k(sK + 2 * s * kSub + off), id_qk, kk > 0);
+        }
+        mma_commit(bar(B_SF + b));
+      };
+      bool ok = mbar_wait(bar(B_Q), 0, abort_flag, err) && mbar_wait(bar(B_KF), 0, abort_flag, err);
+      if (ok) {
+        fence_after_sync();
+        issue_s(0, 0);
+      }
+      for (int j = 0; ok && j < nt; ++j) {
+        const int s = j % ST, b = j & 1;
+        if (j + 1 < nt) {
+          const int s1 = (j + 1) % ST;
+          ok = mbar_wait(bar(B_KF + s1), ((j + 1) / ST) & 1, abort_flag, err);
+          // S(j+1) reuses the buffer of S(j-1): the top-K warpgroup must have read it
+          if (ok && j >= 1) ok = mbar_wait(bar(B_SR + (b ^ 1)), (((j + 1) >> 1) - 1) & 1, abort_flag, err);
+          if (!ok) break;
+          fence_after_sync();
+          issue_s(s1, b ^ 1);
+        }
+        ok = mbar_wait(bar(B_VF + s), (j / ST) & 1, abort_flag, err) &&
+             mbar_wait(bar(B_PF + b), (j >> 1) & 1, abort_flag, err);
+        if (!ok) break;
+        fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tbase + 256, tbase + 320 + b * 64 + kk * 8, sdesc_mn(sV + s * kSub + kk * 2048), id_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar(B_OD));
+        mma_commit(bar(B_KVE + s));
+      }
+      if (ok) {
+        mma_commit(bar(B_OF));
+      } else {
+        volatile int never = 0;
+        mma_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, &never, err);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------- softmax ----------------
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t o_addr = tbase + lane_off + 256;
+    const float c2 = d.scale_log2;
+    float m_used = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int b = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + b), (j >> 1) & 1, abort_flag, err))) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      const uint32_t s_addr = tbase + lane_off + b * 128;
+      const uint32_t p_addr = tbase + lane_off + 320 + b * 64;
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
+      tmem_wait_ld();
+      const long long rem = n_k - (long long)j * TK;
+      if (rem < TK) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
+      }
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
+      const float mxs = mx * c2;
+      const bool need = mxs > m_used + 8.f;
+      if (__any_sync(0xffffffffu, need)) {
+        const float corr = need ? exp2f(m_used - mxs) : 1.f;
+        if (j > 0) {
+          // the previous P V product must be complete before O is rescaled
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OD), (j - 1) & 1, abort_flag, err))) {
+            ok = false;
+            break;
+          }
+          fence_after_sync();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t ov[16];
+            tmem_ld16(o_addr + 16 * c, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
+            tmem_st16(o_addr + 16 * c, ov);
+          }
+          tmem_wait_st();
+        }
+        if (need) {
+          l *= corr;
+          m_used = mxs;
+        }
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = exp2f(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
+          const float p1 = exp2f(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used));
+          sum += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(p_addr + 16 * c, pk);
+      }
+      tmem_wait_st();
+      l += sum;
+      fence_before_sync();
+      mbar_arrive(bar(B_PF + b));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF), 0, abort_flag, err));
+    if (ok) {
+      fence_after_sync();
+      const long long row = m0 + r;
+      const bool store = row < d.Tc;
+      const float inv = 1.f / l;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t ov[16];
+        tmem_ld16(o_addr + 16 * c, ov);
+        tmem_wait_ld();
+        if (!store) continue;
+        float4* dst = reinterpret_cast<float4*>(oc + (row * d.H + h) * kHeadDim + 16 * c);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          dst[i] = make_float4(__uint_as_float(ov[4 * i]) * inv, __uint_as_float(ov[4 * i + 1]) * inv,
+                               __uint_as_float(ov[4 * i + 2]) * inv, __uint_as_float(ov[4 * i + 3]) * inv);
+      }
+    }
+  } else if (warp >= 8) {
+    // ---------------- streaming top-K over S_guide ----------------
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float* cb_s = reinterpret_cast<float*>(sp + OFF_CS);
+    int* cb_c = reinterpret_cast<int*>(sp + OFF_CC);
+    Heap heap{reinterpret_cast<float*>(sp + OFF_HS), reinterpret_cast<int*>(sp + OFF_HI), r, d.K, 0,
+              -CUDART_INF_F};
+    bool ok = true;
+    for (int j = 0; j < nt; ++j) {
+      const int b = j & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + b), (j >> 1) & 1, abort_flag, err))) {
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + lane_off + b * 128 + 32 * c, sv[c]);
+      tmem_wait_ld();
+      fence_before_sync();
+      mbar_arrive(bar(B_SR + b));  // the tensor core may overwrite this buffer now
+      const int e0 = j * TK;
+      const int rem = (int)(n_k - e0);
+      if (rem < TK) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
+      }
+      // first entry of the tile: frame f0, position r0 inside the frame
+      const int f0 = e0 / d.E;
+      const int r0 = e0 - f0 * d.E;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        float cmax = -CUDART_INF_F;
+#pragma unroll
+        for (int i = 0; i < kChunk; ++i) cmax = fmaxf(cmax, __uint_as_float(sv[q >> 1][(q & 1) * 16 + i]));
+        if (!(cmax > heap.tau)) continue;
+        int nc = 0;
+#pragma unroll
+        for (int i = 0; i < kChunk; ++i) {
+          const float v = __uint_as_float(sv[q >> 1][(q & 1) * 16 + i]);
+          if (v > heap.tau) {
+            cb_s[nc * TQ + r] = v;
+            cb_c[nc * TQ + r] = q * kChunk + i;
+            ++nc;
+          }
+        }
+        for (int n = 0; n < nc; ++n) {
+          const float v = cb_s[n * TQ + r];
+          if (!(v > heap.tau)) continue;
+          int i = r0 + cb_c[n * TQ + r], f = f0;
+          while (i >= d.E) i -= d.E, ++f;
+          if (i < d.S) continue;  // special entries are always kept, never ranked
+          heap.push(v, f * d.Bf + (i - d.S));
+        }
+      }
+    }
+    const long long row = m0 + r;
+    if (ok && row < d.Tc) {
+      const long long cb = ((long long)h * d.Tc + row) * d.K;
+      for (int k = 0; k < d.K; ++k) {
+        const bool have = k < heap.cnt;
+        cand_s[cb + k] = have ? heap.hs[k * TQ + r] * d.scale : -CUDART_INF_F;
+        cand_i[cb + k] = have ? heap.hi[k * TQ + r] : -1;
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 2) {
+    fence_after_sync();
+    tmem_dealloc(tbase, kCols);
+  }
+}
+
+}  // namespace
+
+bool compressed_tc_supported(const Dims& d) { return d.K <= kMaxK; }
+
+cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* kc32, const bf16* vc,
+                                 float* oc, float* cand_score, int* cand_idx, unsigned* err,
+                                 cudaStream_t st) {
+  if (!compressed_tc_supported(d)) return cudaErrorInvalidValue;
+  const unsigned long long H = (unsigned long long)d.H, Tc = (unsigned long long)d.Tc;
+  CUtensorMap mq, mk, mv;
+  bool ok = make_tmap_3d(&mq, true, qc32, 64, H, Tc, 256, H * 256, 32, 1, 128) &&
+            make_tmap_3d(&mk, true, kc32, 64, H, Tc, 256, H * 256, 32, 1, 128) &&
+            make_tmap_3d(&mv, false, vc, 64, H, Tc, 128, H * 128, 64, 1, 128);
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_cmp_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)((d.Tc + TQ - 1) / TQ), (unsigned)d.H);
+  attn_cmp_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, d, oc, cand_score, cand_idx, err);
+  return cudaGetLastError();
+}
+
+}  // namespace gsa

@@ -73,6 +73,7 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
 constexpr int kMaxCandidates = 2048;  // n_split * K per row in the merge
 
 int forward_splits(const Dims& d) {
+  if (gsa::compressed_tc_supported(d)) return 1;
   const long long row_ctas = ((d.Tc + 127) / 128) * d.H;
   long long ns = (2 * 148 + row_ctas - 1) / row_ctas;
   if (ns < 1) ns = 1;
@@ -83,7 +84,7 @@ int forward_splits(const Dims& d) {
 }
 
 struct Layout {
-  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cs, ci, sel, total;
+  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cs, ci, sel, ospec, lspec, total;
   int n_split;
 };
 
@@ -110,6 +111,10 @@ Layout forward_layout(const Dims& d) {
   l.cs = take(cand * 4);
   l.ci = take(cand * 4);
   l.sel = take((size_t)d.H * d.Tc * d.K * 4);
+  // the special-token segment of the selection branch: normalised output and lse
+  const size_t tok_heads = d.NS > 0 ? (size_t)d.T * d.H : 0;
+  l.ospec = take(tok_heads * gsa::kHeadDim * 4);
+  l.lspec = take(tok_heads * 4);
   l.total = o;
   return l;
 }
@@ -182,6 +187,9 @@ gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const
   if (n_split < 1 || n_split > 64 || (long long)n_split * d.K > kMaxCandidates)
     return GSA_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
+  if (n_split == 1 && gsa::compressed_tc_supported(d))
+    return cuda_status(gsa::launch_compressed_tc(d, qc32, kc32, (const bf16*)vc, oc, cand_score,
+                                                 cand_idx, (unsigned*)ws, s));
   gsa::AttnArgs a;
   a.q = (const bf16*)qc;
   a.k = (const bf16*)kc;
@@ -227,8 +235,8 @@ gsa_status gsa_selected_attn(const gsa_shape* shape, const gsa_bf16* q, const gs
   if (d.NS > 0 && (!dev_ptr(ks) || !dev_ptr(vs))) return GSA_ERR_INVALID_ARG;
   return cuda_status(gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v,
                                           (const bf16*)ks, (const bf16*)vs, sel, nullptr, nullptr,
-                                          nullptr, (bf16*)o_sel, lse, (unsigned*)ws,
-                                          as_stream(stream)));
+                                          nullptr, (bf16*)o_sel, lse, nullptr, nullptr,
+                                          (unsigned*)ws, as_stream(stream)));
 }
 
 gsa_status gsa_gate_combine(const gsa_shape* shape, const float* qc32, const float* w,
@@ -327,29 +335,60 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
     return e == cudaSuccess && mark(i);
   };
   if (!mark(0)) return GSA_ERR_CUDA;
-  if (!step(gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32, vc, qc,
-                             kc, ks, vs, s), 1))
+  const bool fused = gsa::compressed_tc_supported(d);
+  if (!step(gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32, vc,
+                             fused ? nullptr : qc, fused ? nullptr : kc, ks, vs, s), 1))
     return GSA_ERR_CUDA;
-  gsa::AttnArgs a;
-  a.q = qc;
-  a.k = kc;
-  a.v = vc;
-  a.q_row = a.kv_row = a.o_row = (long long)d.H * gsa::kHeadDim;
-  a.q_head = a.kv_head = a.o_head = gsa::kHeadDim;
-  a.n_q = a.n_k = d.Tc;
-  a.o = oc;
-  a.o_f32 = true;
-  a.lse = nullptr;
-  a.lse_row = a.lse_head = 0;
-  a.H = d.H;
-  a.scale = d.scale;
-  a.scale_log2 = d.scale_log2;
-  if (!step(gsa::launch_attn_mma(a, s), 2)) return GSA_ERR_CUDA;
-  if (!step(gsa::launch_block_scores_topk(d, qc32, kc32, cs, ci, l.n_split, s), 3)) return GSA_ERR_CUDA;
+  if (fused) {
+    // steps 1 and 2 in one kernel; step 2's interval stays empty
+    if (!step(gsa::launch_compressed_tc(d, qc32, kc32, vc, oc, cs, ci, (unsigned*)ws, s), 2) || !mark(3))
+      return GSA_ERR_CUDA;
+  } else {
+    gsa::AttnArgs a;
+    a.q = qc;
+    a.k = kc;
+    a.v = vc;
+    a.q_row = a.kv_row = a.o_row = (long long)d.H * gsa::kHeadDim;
+    a.q_head = a.kv_head = a.o_head = gsa::kHeadDim;
+    a.n_q = a.n_k = d.Tc;
+    a.o = oc;
+    a.o_f32 = true;
+    a.lse = nullptr;
+    a.lse_row = a.lse_head = 0;
+    a.H = d.H;
+    a.scale = d.scale;
+    a.scale_log2 = d.scale_log2;
+    if (!step(gsa::launch_attn_mma(a, s), 2)) return GSA_ERR_CUDA;
+    if (!step(gsa::launch_block_scores_topk(d, qc32, kc32, cs, ci, l.n_split, s), 3)) return GSA_ERR_CUDA;
+  }
   if (!step(gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s), 4)) return GSA_ERR_CUDA;
+  float* ospec = nullptr;
+  float* lspec = nullptr;
+  if (d.NS > 0) {
+    // the always-kept special tokens: every token attends to all N*S of them
+    ospec = (float*)(base + l.ospec);
+    lspec = (float*)(base + l.lspec);
+    gsa::AttnTcArgs a;
+    a.n_q = d.T;
+    a.n_k = d.NS;
+    a.H = d.H;
+    a.c2 = d.scale_log2;
+    a.out = ospec;
+    a.out_f32 = 1;
+    a.o_row = (long long)d.H * gsa::kHeadDim;
+    a.o_head = gsa::kHeadDim;
+    a.lse = lspec;
+    a.lse_row = d.H;
+    a.lse_head = 1;
+    a.err = (unsigned*)ws;
+    a.kv_head_major = 1;
+    if (!step(gsa::launch_attn_tc(a, (const bf16*)q, ks, vs, d.NS, s), 5)) return GSA_ERR_CUDA;
+  } else if (!mark(5)) {
+    return GSA_ERR_CUDA;
+  }
   if (!step(gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, ks, vs, sel, qc32,
-                                 w, oc, (bf16*)out, nullptr, (unsigned*)ws, s),
-            5))
+                                 w, oc, (bf16*)out, nullptr, ospec, lspec, (unsigned*)ws, s),
+            6))
     return GSA_ERR_CUDA;
   if (n_launched) *n_launched = launched;
   return GSA_OK;
@@ -378,6 +417,8 @@ gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out) {
   out->cand_score = l.cs;
   out->cand_idx = l.ci;
   out->sel = l.sel;
+  out->o_spec = l.ospec;
+  out->lse_spec = l.lspec;
   out->total = l.total;
   out->n_split = l.n_split;
   return GSA_OK;

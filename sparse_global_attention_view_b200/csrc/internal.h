@@ -3,6 +3,7 @@
 // validated by the caller.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -49,6 +50,19 @@ struct AttnTcArgs {
 cudaError_t launch_attn_tc(const AttnTcArgs& a, const bf16* q, const bf16* k, const bf16* v,
                            long long kv_rows, cudaStream_t st);
 
+// 3-D tiled TMA map (128-byte swizzle) over bf16 or fp32 data; dims and
+// strides innermost first, strides in bytes.  False if the driver refuses it.
+bool make_tmap_3d(CUtensorMap* m, bool fp32, const void* base, unsigned long long d0,
+                  unsigned long long d1, unsigned long long d2, unsigned long long s1,
+                  unsigned long long s2, unsigned b0, unsigned b1, unsigned b2);
+
+// Compressed attention on tcgen05 fused with the S_guide streaming top-K
+// (one candidate list per row, i.e. n_split = 1); needs K <= 64.
+bool compressed_tc_supported(const Dims& d);
+cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* kc32, const bf16* vc,
+                                 float* oc, float* cand_score, int* cand_idx, unsigned* err,
+                                 cudaStream_t st);
+
 cudaError_t launch_block_scores_topk(const Dims& d, const float* qc32, const float* kc32,
                                      float* cand_score, int* cand_idx, int n_split,
                                      cudaStream_t st);
@@ -57,10 +71,13 @@ cudaError_t launch_topk_merge(const Dims& d, const float* cand_score, const int*
 
 // Selection branch; when `w` is non-null the gate is fused and `out` receives
 // g*oc + (1-g)*o_sel, otherwise `out` receives o_sel (and lse if non-null).
+// With o_spec/lse_spec non-null the special-token segment is taken from them
+// (normalised fp32 [T][H][64] and natural-log lse [T][H]) instead of ks/vs.
 cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const bf16* v,
                             const bf16* ks, const bf16* vs, const int* sel, const float* qc32,
                             const float* w, const float* oc, bf16* out, float* lse,
-                            unsigned* err, cudaStream_t st);
+                            const float* o_spec, const float* lse_spec, unsigned* err,
+                            cudaStream_t st);
 
 cudaError_t launch_gate_combine(const Dims& d, const float* qc32, const float* w, const float* oc,
                                 const bf16* o_sel, bf16* out, cudaStream_t st);

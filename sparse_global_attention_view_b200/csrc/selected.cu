@@ -10,6 +10,10 @@
 //      the warp itself (16 token rows of 128 bytes straight from K/V, a
 //      3-stage cp.async pipeline per warp; patches outside the grid are
 //      zero-filled and masked to -inf).
+// When the specials segment was already computed elsewhere (o_spec, lse_spec:
+// its normalised output and log-sum-exp per token and head), the warp starts
+// its online softmax from that state instead of running segment 1: running
+// maximum lse/scale, row sum 1, output o_spec.
 // The epilogue normalises and either writes o_sel (+lse) or applies the gate
 // g = sigmoid(qc32[a,h] . w[h]) and writes g*oc + (1-g)*o_sel.
 #include <math_constants.h>
@@ -104,6 +108,7 @@ __global__ void __launch_bounds__(SW * 32)
                     const bf16* __restrict__ vs, const int* __restrict__ sel,
                     const float* __restrict__ qc32, const float* __restrict__ w,
                     const float* __restrict__ oc, bf16* __restrict__ out, float* __restrict__ lse,
+                    const float* __restrict__ o_spec, const float* __restrict__ lse_spec,
                     unsigned* __restrict__ err) {
   extern __shared__ __align__(128) unsigned char sel_smem_raw[];
   SelSmem& sm = *reinterpret_cast<SelSmem*>(sel_smem_raw);
@@ -137,36 +142,58 @@ __global__ void __launch_bounds__(SW * 32)
               qf[kq][2], qf[kq][3]);
   };
 
-  // ---- segment 1: the special tokens (shared tiles) ----
+  // ---- segment 1: the special tokens ----
   const long long NS = d.NS;
-  auto load_sp = [&](int buf, long long n0) {
-    for (int i = tid; i < SBN * 8; i += SW * 32) {
-      const int r = i >> 3, c = i & 7;
-      const long long idx = n0 + r;
-      const bool ok = idx < NS;
-      const long long off = ((long long)h * NS + (ok ? idx : 0)) * kHeadDim + c * 8;
-      cp_async16(smem_u32(sm.ks[buf]) + swz(r, c), ks + off, ok);
-      cp_async16(smem_u32(sm.vs[buf]) + swz(r, c), vs + off, ok);
+  if (o_spec != nullptr) {
+    // state of a softmax over the specials alone, computed by another kernel
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      const long long t = live ? entry_slot_token(d, a, (lane >> 2) + 8 * hf) : -1;
+      if (t < 0) continue;
+      const long long th = t * d.H + h;
+      m_r[hf] = lse_spec[th] / d.scale;
+      l_r[hf] = (lane & 3) == 0 ? 1.f : 0.f;
+      const float* os = o_spec + th * kHeadDim + 2 * (lane & 3);
+#pragma unroll
+      for (int dt = 0; dt < 8; ++dt) {
+        const float2 x = *reinterpret_cast<const float2*>(os + dt * 8);
+        o[dt][2 * hf] = x.x;
+        o[dt][2 * hf + 1] = x.y;
+      }
     }
-  };
-  const long long n_sp = (NS + SBN - 1) / SBN;
-  if (n_sp > 0) load_sp(0, 0);
-  cp_async_commit();
-  for (long long j = 0; j < n_sp; ++j) {
-    if (j + 1 < n_sp) load_sp((int)((j + 1) & 1), (j + 1) * SBN);
-    cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
-    if (j == 0) load_qf();
-    const long long base = j * SBN;
-    tile_step<8>(smem_u32(sm.ks[j & 1]), smem_u32(sm.vs[j & 1]), qf, o, m_r, l_r, c2, lane,
-                 [&](int key) { return base + key >= NS; });
-    __syncthreads();
-  }
-  if (n_sp == 0) {
     cp_async_wait<0>();
     __syncthreads();
     load_qf();
+  } else {
+    auto load_sp = [&](int buf, long long n0) {
+      for (int i = tid; i < SBN * 8; i += SW * 32) {
+        const int r = i >> 3, c = i & 7;
+        const long long idx = n0 + r;
+        const bool ok = idx < NS;
+        const long long off = ((long long)h * NS + (ok ? idx : 0)) * kHeadDim + c * 8;
+        cp_async16(smem_u32(sm.ks[buf]) + swz(r, c), ks + off, ok);
+        cp_async16(smem_u32(sm.vs[buf]) + swz(r, c), vs + off, ok);
+      }
+    };
+    const long long n_sp = (NS + SBN - 1) / SBN;
+    if (n_sp > 0) load_sp(0, 0);
+    cp_async_commit();
+    for (long long j = 0; j < n_sp; ++j) {
+      if (j + 1 < n_sp) load_sp((int)((j + 1) & 1), (j + 1) * SBN);
+      cp_async_commit();
+      cp_async_wait<1>();
+      __syncthreads();
+      if (j == 0) load_qf();
+      const long long base = j * SBN;
+      tile_step<8>(smem_u32(sm.ks[j & 1]), smem_u32(sm.vs[j & 1]), qf, o, m_r, l_r, c2, lane,
+                   [&](int key) { return base + key >= NS; });
+      __syncthreads();
+    }
+    if (n_sp == 0) {
+      cp_async_wait<0>();
+      __syncthreads();
+      load_qf();
+    }
   }
 
   // ---- segment 2: the selected blocks (per warp) ----
@@ -251,13 +278,15 @@ __global__ void __launch_bounds__(SW * 32)
 cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const bf16* v,
                             const bf16* ks, const bf16* vs, const int* sel, const float* qc32,
                             const float* w, const float* oc, bf16* out, float* lse,
-                            unsigned* err, cudaStream_t st) {
+                            const float* o_spec, const float* lse_spec, unsigned* err,
+                            cudaStream_t st) {
   const size_t smem = sizeof(SelSmem);
   cudaError_t e =
       cudaFuncSetAttribute(selected_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((d.Tc + SW - 1) / SW), (unsigned)d.H);
-  selected_kernel<<<grid, SW * 32, smem, st>>>(d, q, k, v, ks, vs, sel, qc32, w, oc, out, lse, err);
+  selected_kernel<<<grid, SW * 32, smem, st>>>(d, q, k, v, ks, vs, sel, qc32, w, oc, out, lse, o_spec,
+                                                lse_spec, err);
   return cudaGetLastError();
 }
 

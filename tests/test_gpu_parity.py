@@ -93,9 +93,18 @@ def test_top_k_selection(name):
 
 @pytest.mark.parametrize("name", ["small", "p3_ragged"])
 def test_split_candidates_merge_to_same_selection(name):
-    a = case(name, 1)[3].sel.cpu()
+    # n_split > 1 runs the fp32 block scorer over slices of the block range;
+    # merging 2 or 3 slice lists must give the same selection
+    a = case(name, 2)[3].sel.cpu()
     b = case(name, 3)[3].sel.cpu()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", ["small", "p3_ragged", "tiny"])
+def test_sliced_block_scorer_is_valid(name):
+    x, geo, shape, st, res = case(name, 3)
+    PT.assert_selection(res, f"{name} (3 slices)")
+    PT.assert_close(st.oc, res["o_cmp"], f"{name} o_cmp (warp-MMA path)")
 
 
 @pytest.mark.parametrize("name", NAMES)

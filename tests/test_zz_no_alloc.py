@@ -26,12 +26,18 @@ def _device_inputs(wl):
     return [t.cuda() for t in (x.q, x.k, x.v, x.w)]
 
 
-@pytest.mark.parametrize("name", ["tiny", "small"])
+# Tiny, and the VGGT token layout (37x37 patches + 5 special tokens, 16
+# heads) at 4 frames, the largest frame count whose workspace fits the array.
+CASES = {"tiny": WORKLOADS["tiny"],
+         "vggt_4_frames": WORKLOADS["small"].with_(name="vggt_4_frames", n_frames=4)}
+
+
+@pytest.mark.parametrize("name", list(CASES))
 def test_noalloc_matches_workspace_forward_on_two_calls(name):
     import sparse_global_attention_view_b200 as G
     from sparse_global_attention_view_b200._lib import NOALLOC_SCRATCH_BYTES
 
-    wl = WORKLOADS[name]
+    wl = CASES[name]
     shape = G.Shape.of(wl)
     assert G.workspace_size(shape) <= NOALLOC_SCRATCH_BYTES
     layer = G.GsaLayer(shape)

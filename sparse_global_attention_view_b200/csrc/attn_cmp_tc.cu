@@ -13,14 +13,15 @@
 //   warps 8-11  streaming top-K, one thread per query row.
 // S(j+1) is computed while both warpgroups work on S(j): the softmax writes
 // P(j) to its own TMEM columns, so the raw scores stay readable until the
-// top-K warpgroup has loaded them.  Each top-K thread scans its row's raw
-// scores in registers: 16-column chunks whose maximum beats the row's current
-// K-th best score are
-// appended to a per-thread candidate buffer in shared memory; candidates that
-// are patch blocks (special entries are never ranked) enter a per-row min-heap
-// of (score, block id) ordered worst-first by (score ascending, id
-// descending).  Columns arrive in ascending block order and only a strictly
-// larger score displaces the root, so equal scores keep the lower block id.
+// top-K warpgroup has loaded them.  Each top-K thread compares its row's raw
+// scores (in registers) with the row's current K-th best: 16-column and then
+// 4-column maxima are tested with warp votes, so the warp only touches the
+// columns where some of its 32 rows have a candidate.  Candidates go to a
+// per-row buffer in shared memory; when any row's buffer is half full the warp
+// inserts all buffered candidates in lockstep (one round of insertions serves
+// every row) into the rows' heaps of K best (score, block id) pairs; special
+// entries are never ranked.  Columns arrive in ascending block order and only a
+// strictly larger score displaces the root, so equal scores keep the lower id.
 #include <math_constants.h>
 
 #include "internal.h"
@@ -36,7 +37,7 @@ constexpr int TK = 128;
 constexpr int ST = 2;
 constexpr int kThreads = 384;
 constexpr int kMaxK = 64;        // heap capacity per row
-constexpr int kChunk = 16;       // columns per candidate scan chunk
+constexpr int kBuf = 32;         // candidate buffer entries per row
 constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16) tile: 16 KB
 
 constexpr uint32_t OFF_Q = 0;                        // 2 sub-tiles (d 0-31, 32-63)
@@ -44,9 +45,9 @@ constexpr uint32_t OFF_K = OFF_Q + 2 * kSub;         // ST x 2 sub-tiles
 constexpr uint32_t OFF_V = OFF_K + ST * 2 * kSub;    // ST x bf16 tile
 constexpr uint32_t OFF_HS = OFF_V + ST * kSub;       // heap scores [kMaxK][128]
 constexpr uint32_t OFF_HI = OFF_HS + kMaxK * TQ * 4; // heap ids
-constexpr uint32_t OFF_CS = OFF_HI + kMaxK * TQ * 4; // candidate scores [kChunk][128]
-constexpr uint32_t OFF_CC = OFF_CS + kChunk * TQ * 4;// candidate columns
-constexpr uint32_t OFF_BAR = OFF_CC + kChunk * TQ * 4;
+constexpr uint32_t OFF_CS = OFF_HI + kMaxK * TQ * 4; // candidate scores [kBuf][128]
+constexpr uint32_t OFF_CC = OFF_CS + kBuf * TQ * 4;  // candidate entry indices
+constexpr uint32_t OFF_BAR = OFF_CC + kBuf * TQ * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 
@@ -55,7 +56,17 @@ constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + ST, B_KVE = B_VF + ST, B_SF = B_K
               B_COUNT = B_DRAIN + 1;
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 constexpr uint32_t kCols = 512;
+// Register split: the block is launched with kLaunchRegs per thread; the
+// producer/MMA warpgroup gives registers to the softmax and top-K warpgroups.
+// 128 * kRegsLow + 256 * kRegsHigh must not exceed 384 * kLaunchRegs, or the
+// increase would wait forever, so the host refuses to launch unless the
+// compiled kernel uses exactly kLaunchRegs registers per thread.
+constexpr int kLaunchRegs = 168, kRegsLow = 56, kRegsHigh = 224;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 
+// The K best (score, block id) pairs of one row: a binary min-heap in shared
+// memory ([slot][row] layout, so the 128 rows hit distinct banks), worst pair
+// at the root.  Worst = smallest score, and among equal scores the largest id.
 struct Heap {
   float* hs;
   int* hi;
@@ -102,7 +113,8 @@ struct Heap {
 __global__ void __launch_bounds__(kThreads, 1)
     attn_cmp_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const Dims d, float* __restrict__ oc,
-                       float* __restrict__ cand_s, int* __restrict__ cand_i, unsigned* err) {
+                       float* __restrict__ cand_s, int* __restrict__ cand_i, int* __restrict__ sel,
+                       unsigned* err) {
   extern __shared__ __align__(1024) uint8_t cmp_smem_raw[];
   const uint32_t raw = smem_u32(cmp_smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -145,6 +157,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after_sync();
   const uint32_t tbase = *tmem_slot;
 
+  if (warp < 4) {
+    regs_dec<kRegsLow>();
+  }
   if (warp == 0) {
     if (lane == 0) {
       prefetch_tmap(&tq);
@@ -221,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 4 && warp < 8) {
+    regs_inc<kRegsHigh>();
     // ---------------- softmax ----------------
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
@@ -238,11 +254,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after_sync();
       const uint32_t s_addr = tbase + lane_off + b * 128;
       const uint32_t p_addr = tbase + lane_off + 320 + b * 64;
+      const long long rem = n_k - (long long)j * TK;
+      // all 128 scores in one round of TMEM loads: the softmax is bound by
+      // TMEM load latency, so a second round would cost as much as the first
       uint32_t sv[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
       tmem_wait_ld();
-      const long long rem = n_k - (long long)j * TK;
       if (rem < TK) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -320,14 +338,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 8) {
+    regs_inc<kRegsHigh>();
     // ---------------- streaming top-K over S_guide ----------------
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     float* cb_s = reinterpret_cast<float*>(sp + OFF_CS);
-    int* cb_c = reinterpret_cast<int*>(sp + OFF_CC);
-    Heap heap{reinterpret_cast<float*>(sp + OFF_HS), reinterpret_cast<int*>(sp + OFF_HI), r, d.K, 0,
-              -CUDART_INF_F};
+    int* cb_e = reinterpret_cast<int*>(sp + OFF_CC);
+    Heap top{reinterpret_cast<float*>(sp + OFF_HS), reinterpret_cast<int*>(sp + OFF_HI), r, d.K, 0, -CUDART_INF_F};
+    const int E = d.E, S = d.S, Bf = d.Bf;
+    const int ntok = (int)n_k;
+    int nb = 0;  // candidates waiting in this row's buffer
+    // Insert the buffered candidates.  All lanes run this together, so one
+    // round of insertions serves every row of the warp at once.
+    auto flush = [&]() {
+      for (int n = 0; n < nb; ++n) {
+        const float v = cb_s[n * TQ + r];
+        if (!(v > top.tau)) continue;
+        const int e = cb_e[n * TQ + r];
+        const int f = e / E, i = e - f * E;
+        if (i >= S) top.push(v, f * Bf + (i - S));  // special entries are never ranked
+      }
+      nb = 0;
+    };
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
@@ -343,50 +376,67 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_before_sync();
       mbar_arrive(bar(B_SR + b));  // the tensor core may overwrite this buffer now
       const int e0 = j * TK;
-      const int rem = (int)(n_k - e0);
-      if (rem < TK) {
+      if (ntok - e0 < TK) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
+            if (32 * c + i >= ntok - e0) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      // first entry of the tile: frame f0, position r0 inside the frame
-      const int f0 = e0 / d.E;
-      const int r0 = e0 - f0 * d.E;
+      // A column is a candidate for a row if it beats that row's K-th best.
+      // The vote keeps control flow uniform: only columns where some row of
+      // the warp has a candidate cost more than the compare and the vote.
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        float cmax = -CUDART_INF_F;
+        float m4[4];
 #pragma unroll
-        for (int i = 0; i < kChunk; ++i) cmax = fmaxf(cmax, __uint_as_float(sv[q >> 1][(q & 1) * 16 + i]));
-        if (!(cmax > heap.tau)) continue;
-        int nc = 0;
+        for (int u = 0; u < 4; ++u) {
+          float x = -CUDART_INF_F;
 #pragma unroll
-        for (int i = 0; i < kChunk; ++i) {
-          const float v = __uint_as_float(sv[q >> 1][(q & 1) * 16 + i]);
-          if (v > heap.tau) {
-            cb_s[nc * TQ + r] = v;
-            cb_c[nc * TQ + r] = q * kChunk + i;
-            ++nc;
-          }
+          for (int i = 0; i < 4; ++i) x = fmaxf(x, __uint_as_float(sv[q >> 1][(q & 1) * 16 + 4 * u + i]));
+          m4[u] = x;
         }
-        for (int n = 0; n < nc; ++n) {
-          const float v = cb_s[n * TQ + r];
-          if (!(v > heap.tau)) continue;
-          int i = r0 + cb_c[n * TQ + r], f = f0;
-          while (i >= d.E) i -= d.E, ++f;
-          if (i < d.S) continue;  // special entries are always kept, never ranked
-          heap.push(v, f * d.Bf + (i - d.S));
+        const float m16 = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        if (__any_sync(0xffffffffu, m16 > top.tau)) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (__any_sync(0xffffffffu, m4[u] > top.tau)) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float v = __uint_as_float(sv[q >> 1][(q & 1) * 16 + 4 * u + i]);
+                if (v > top.tau) {
+                  cb_s[nb * TQ + r] = v;
+                  cb_e[nb * TQ + r] = e0 + 16 * q + 4 * u + i;
+                  ++nb;
+                }
+              }
+            }
+          }
+          if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush();
         }
       }
     }
+    if (__all_sync(0xffffffffu, ok)) flush();
     const long long row = m0 + r;
     if (ok && row < d.Tc) {
       const long long cb = ((long long)h * d.Tc + row) * d.K;
-      for (int k = 0; k < d.K; ++k) {
-        const bool have = k < heap.cnt;
-        cand_s[cb + k] = have ? heap.hs[k * TQ + r] * d.scale : -CUDART_INF_F;
-        cand_i[cb + k] = have ? heap.hi[k * TQ + r] : -1;
+      if (cand_s != nullptr) {
+        for (int k = 0; k < d.K; ++k) {
+          const bool have = k < top.cnt;
+          cand_s[cb + k] = have ? top.hs[k * TQ + r] * d.scale : -CUDART_INF_F;
+          cand_i[cb + k] = have ? top.hi[k * TQ + r] : -1;
+        }
+      }
+      if (sel != nullptr) {
+        // the heap holds exactly this row's top-K: write its ids in ascending
+        // order (rank of each id among the row's distinct ids), then -1 padding
+        for (int k = 0; k < top.cnt; ++k) {
+          const int me = top.hi[k * TQ + r];
+          int rank = 0;
+          for (int k2 = 0; k2 < top.cnt; ++k2) rank += top.hi[k2 * TQ + r] < me;
+          sel[cb + rank] = me;
+        }
+        for (int k = top.cnt; k < d.K; ++k) sel[cb + k] = -1;
       }
     }
   }
@@ -403,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 bool compressed_tc_supported(const Dims& d) { return d.K <= kMaxK; }
 
 cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* kc32, const bf16* vc,
-                                 float* oc, float* cand_score, int* cand_idx, unsigned* err,
+                                 float* oc, float* cand_score, int* cand_idx, int* sel, unsigned* err,
                                  cudaStream_t st) {
   if (!compressed_tc_supported(d)) return cudaErrorInvalidValue;
   const unsigned long long H = (unsigned long long)d.H, Tc = (unsigned long long)d.Tc;
@@ -415,8 +465,13 @@ cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* 
   cudaError_t e = cudaFuncSetAttribute(attn_cmp_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_cmp_tc_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   dim3 grid((unsigned)((d.Tc + TQ - 1) / TQ), (unsigned)d.H);
-  attn_cmp_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, d, oc, cand_score, cand_idx, err);
+  attn_cmp_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, d, oc, cand_score, cand_idx, sel,
+                                                         err);
   return cudaGetLastError();
 }
 

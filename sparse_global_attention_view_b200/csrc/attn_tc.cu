@@ -48,6 +48,11 @@ constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + ST, B_KVE = B_VF + ST, B_SF = B_K
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 
 constexpr uint32_t kCols = 512;  // TMEM columns: S_t at 128 t, O_t at 256 + 64 t
+// Register split between the producer/MMA warpgroup and the two softmax
+// warpgroups; it must not exceed the launch allocation, or the increase would
+// wait forever (the host checks the compiled register count before launching).
+constexpr int kLaunchRegs = 168, kRegsLow = 72, kRegsHigh = 216;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -91,6 +96,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after_sync();
   const uint32_t tbase = *tmem_slot;
 
+  if (warp < 4) regs_dec<kRegsLow>();
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -173,6 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 4) {
+    regs_inc<kRegsHigh>();
     // ---------------- softmax, one thread per row ----------------
     const int t = (warp - 4) >> 2;
     const int q4 = warp & 3;
@@ -356,6 +363,10 @@ cudaError_t launch_attn_tc(const AttnTcArgs& a, const bf16* q, const bf16* k, co
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   dim3 grid((unsigned)((a.n_q + NQT * TQ - 1) / (NQT * TQ)), (unsigned)a.H);
   attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
   return cudaGetLastError();

@@ -93,7 +93,8 @@ Layout forward_layout(const Dims& d) {
   l.n_split = forward_splits(d);
   const size_t ent = (size_t)d.Tc * d.H * gsa::kHeadDim;
   const size_t spc = (size_t)d.NS * d.H * gsa::kHeadDim;
-  const size_t cand = (size_t)d.H * d.Tc * l.n_split * d.K;
+  // the fused compressed kernel writes the selection directly: no candidate lists
+  const size_t cand = gsa::compressed_tc_supported(d) ? 0 : (size_t)d.H * d.Tc * l.n_split * d.K;
   size_t o = GSA_WS_HEADER_BYTES;
   auto take = [&](size_t bytes) {
     size_t at = o;
@@ -189,7 +190,7 @@ gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const
   cudaStream_t s = as_stream(stream);
   if (n_split == 1 && gsa::compressed_tc_supported(d))
     return cuda_status(gsa::launch_compressed_tc(d, qc32, kc32, (const bf16*)vc, oc, cand_score,
-                                                 cand_idx, (unsigned*)ws, s));
+                                                 cand_idx, nullptr, (unsigned*)ws, s));
   gsa::AttnArgs a;
   a.q = (const bf16*)qc;
   a.k = (const bf16*)kc;
@@ -340,8 +341,11 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
                              fused ? nullptr : qc, fused ? nullptr : kc, ks, vs, s), 1))
     return GSA_ERR_CUDA;
   if (fused) {
-    // steps 1 and 2 in one kernel; step 2's interval stays empty
-    if (!step(gsa::launch_compressed_tc(d, qc32, kc32, vc, oc, cs, ci, (unsigned*)ws, s), 2) || !mark(3))
+    // steps 1-3 in one kernel (its heaps hold each row's final top-K, written
+    // to sel in ascending order); the intervals of steps 2 and 3 stay empty
+    if (!step(gsa::launch_compressed_tc(d, qc32, kc32, vc, oc, nullptr, nullptr, sel, (unsigned*)ws, s),
+              2) ||
+        !mark(3) || !mark(4))
       return GSA_ERR_CUDA;
   } else {
     gsa::AttnArgs a;
@@ -361,7 +365,7 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
     if (!step(gsa::launch_attn_mma(a, s), 2)) return GSA_ERR_CUDA;
     if (!step(gsa::launch_block_scores_topk(d, qc32, kc32, cs, ci, l.n_split, s), 3)) return GSA_ERR_CUDA;
   }
-  if (!step(gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s), 4)) return GSA_ERR_CUDA;
+  if (!fused && !step(gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s), 4)) return GSA_ERR_CUDA;
   float* ospec = nullptr;
   float* lspec = nullptr;
   if (d.NS > 0) {

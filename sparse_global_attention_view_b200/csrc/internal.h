@@ -57,10 +57,12 @@ bool make_tmap_3d(CUtensorMap* m, bool fp32, const void* base, unsigned long lon
                   unsigned long long s2, unsigned b0, unsigned b1, unsigned b2);
 
 // Compressed attention on tcgen05 fused with the S_guide streaming top-K
-// (one candidate list per row, i.e. n_split = 1); needs K <= 64.
+// (one candidate list per row, i.e. n_split = 1); needs K <= 64.  Writes the
+// candidate lists when cand_score/cand_idx are non-null and the final
+// selection (ascending ids, -1 padding) when sel is non-null.
 bool compressed_tc_supported(const Dims& d);
 cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* kc32, const bf16* vc,
-                                 float* oc, float* cand_score, int* cand_idx, unsigned* err,
+                                 float* oc, float* cand_score, int* cand_idx, int* sel, unsigned* err,
                                  cudaStream_t st);
 
 cudaError_t launch_block_scores_topk(const Dims& d, const float* qc32, const float* kc32,

@@ -17,6 +17,7 @@
 // The epilogue normalises and either writes o_sel (+lse) or applies the gate
 // g = sigmoid(qc32[a,h] . w[h]) and writes g*oc + (1-g)*o_sel.
 #include <math_constants.h>
+#include <stddef.h>
 
 #include "internal.h"
 
@@ -27,14 +28,34 @@ constexpr int SW = 4;       // warps (entries) per CTA
 constexpr int SBN = 64;     // special keys per shared tile
 constexpr int SSTAGE = 3;   // per-warp block pipeline depth
 
+// Shared memory of one CTA.  The special-token tiles are only used when the
+// kernel runs that segment itself; without them three CTAs fit on an SM.
 struct SelSmem {
   uint8_t q[SW][16 * 128];
-  uint8_t ks[2][SBN * 128];
-  uint8_t vs[2][SBN * 128];
   uint8_t kb[SW][SSTAGE][16 * 128];
   uint8_t vb[SW][SSTAGE][16 * 128];
   int sel[SW][kMaxTopK];
+  uint8_t ks[2][SBN * 128];
+  uint8_t vs[2][SBN * 128];
 };
+constexpr size_t kSmemNoSpecials = offsetof(SelSmem, ks);
+
+// A patch block's first token (top-left patch) and how many of its P rows and
+// P columns lie inside the grid.
+struct BlockGeo {
+  long long base;
+  int nr, nc;
+};
+__device__ __forceinline__ BlockGeo block_geo(const Dims& d, long long beta) {
+  const long long f = beta / d.Bf;
+  const int j = (int)(beta - f * d.Bf);
+  const int br = j / d.Bw, bc = j - br * d.Bw;
+  BlockGeo g;
+  g.base = f * d.L + d.S + (long long)(br * d.P) * d.Wp + bc * d.P;
+  g.nr = min(d.P, d.Hp - br * d.P);
+  g.nc = min(d.P, d.Wp - bc * d.P);
+  return g;
+}
 
 // One key tile of NT*8 keys: S = Q K^T, mask, online softmax, O += P V.
 template <int NT, typename Masked>
@@ -59,7 +80,7 @@ __device__ __forceinline__ void tile_step(uint32_t kb, uint32_t vb, const uint32
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e)
-      if (masked(nt * 8 + 2 * (lane & 3) + (e & 1))) s[nt][e] = -CUDART_INF_F;
+      if (masked(nt * 2 + (e & 1), nt * 8 + 2 * (lane & 3) + (e & 1))) s[nt][e] = -CUDART_INF_F;
 #pragma unroll
   for (int hf = 0; hf < 2; ++hf) {
     float mx = m_r[hf];
@@ -186,7 +207,7 @@ __global__ void __launch_bounds__(SW * 32)
       if (j == 0) load_qf();
       const long long base = j * SBN;
       tile_step<8>(smem_u32(sm.ks[j & 1]), smem_u32(sm.vs[j & 1]), qf, o, m_r, l_r, c2, lane,
-                   [&](int key) { return base + key >= NS; });
+                   [&](int, int key) { return base + key >= NS; });
       __syncthreads();
     }
     if (n_sp == 0) {
@@ -207,13 +228,30 @@ __global__ void __launch_bounds__(SW * 32)
     }
     ++nsel;
   }
+  // Slots this lane touches: in the gather (slot (lane >> 3) + 4 it) and in
+  // the score fragment (keys 2 (lane & 3) + {0, 1} + {0, 8}).  Their (row,
+  // column) inside a block depend only on P, so they are computed once.
+  int ldr[4], ldc[4], mdr[4], mdc[4];
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int sl = (lane >> 3) + 4 * it;
+    ldr[it] = sl < d.P * d.P ? sl / d.P : kMaxPool;
+    ldc[it] = sl % d.P;
+    const int km = (it >> 1) * 8 + 2 * (lane & 3) + (it & 1);
+    mdr[it] = km < d.P * d.P ? km / d.P : kMaxPool;
+    mdc[it] = km % d.P;
+  }
   auto load_blk = [&](int stage, long long beta) {
-    for (int i = lane; i < 16 * 8; i += 32) {
-      const int slot = i >> 3, c = i & 7;
-      const long long t = block_slot_token(d, beta, slot);
-      const long long off = (t >= 0 ? t : 0) * row + h * kHeadDim + c * 8;
-      cp_async16(smem_u32(sm.kb[warp][stage]) + swz(slot, c), k + off, t >= 0);
-      cp_async16(smem_u32(sm.vb[warp][stage]) + swz(slot, c), v + off, t >= 0);
+    const BlockGeo g = block_geo(d, beta);
+    const int c = lane & 7;
+#pragma unroll
+    for (int it = 0; it < 4; ++it) {
+      const int sl = (lane >> 3) + 4 * it;
+      const bool ok = ldr[it] < g.nr && ldc[it] < g.nc;
+      const long long t = ok ? g.base + (long long)ldr[it] * d.Wp + ldc[it] : 0;
+      const long long off = t * row + h * kHeadDim + c * 8;
+      cp_async16(smem_u32(sm.kb[warp][stage]) + swz(sl, c), k + off, ok);
+      cp_async16(smem_u32(sm.vb[warp][stage]) + swz(sl, c), v + off, ok);
     }
   };
 #pragma unroll
@@ -226,10 +264,10 @@ __global__ void __launch_bounds__(SW * 32)
     cp_async_commit();
     cp_async_wait<SSTAGE - 1>();
     __syncwarp();
-    const long long beta = sm.sel[warp][i];
+    const BlockGeo g = block_geo(d, sm.sel[warp][i]);
     const int st = i % SSTAGE;
     tile_step<2>(smem_u32(sm.kb[warp][st]), smem_u32(sm.vb[warp][st]), qf, o, m_r, l_r, c2, lane,
-                 [&](int key) { return block_slot_token(d, beta, key) < 0; });
+                 [&](int m, int) { return !(mdr[m] < g.nr && mdc[m] < g.nc); });
     __syncwarp();
   }
   if (!live) return;
@@ -280,9 +318,10 @@ cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const b
                             const float* w, const float* oc, bf16* out, float* lse,
                             const float* o_spec, const float* lse_spec, unsigned* err,
                             cudaStream_t st) {
-  const size_t smem = sizeof(SelSmem);
-  cudaError_t e =
-      cudaFuncSetAttribute(selected_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const bool own_specials = d.NS > 0 && o_spec == nullptr;
+  const size_t smem = own_specials ? sizeof(SelSmem) : kSmemNoSpecials;
+  cudaError_t e = cudaFuncSetAttribute(selected_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sizeof(SelSmem));
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((d.Tc + SW - 1) / SW), (unsigned)d.H);
   selected_kernel<<<grid, SW * 32, smem, st>>>(d, q, k, v, ks, vs, sel, qc32, w, oc, out, lse, o_spec,

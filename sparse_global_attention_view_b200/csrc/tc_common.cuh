@@ -132,6 +132,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 // ---------------------------------------------------------------------------
+// per-warpgroup register reallocation (all warps of the warpgroup execute it)
+
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
+// ---------------------------------------------------------------------------
 // tcgen05.mma
 
 // Shared-memory matrix descriptor: start address, leading / stride byte
@@ -152,7 +164,7 @@ __device__ __forceinline__ uint64_t sdesc_mn(uint32_t saddr) { return sdesc(sadd
 
 // Instruction descriptor: fp32 accumulator, A/B format (1 = bf16, 2 = tf32),
 // A/B major (0 = K, 1 = MN), N >> 3 at bit 17, M >> 4 at bit 24.
-constexpr uint32_t idesc(int m, int n, uint32_t fmt, uint32_t a_mn, uint32_t b_mn) {
+__host__ __device__ constexpr uint32_t idesc(int m, int n, uint32_t fmt, uint32_t a_mn, uint32_t b_mn) {
   return (1u << 4) | (fmt << 7) | (fmt << 10) | (a_mn << 15) | (b_mn << 16) |
          ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }

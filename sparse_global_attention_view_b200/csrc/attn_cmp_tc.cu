@@ -43,9 +43,8 @@ constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16
 constexpr uint32_t OFF_Q = 0;                        // 2 sub-tiles (d 0-31, 32-63)
 constexpr uint32_t OFF_K = OFF_Q + 2 * kSub;         // ST x 2 sub-tiles
 constexpr uint32_t OFF_V = OFF_K + ST * 2 * kSub;    // ST x bf16 tile
-constexpr uint32_t OFF_HS = OFF_V + ST * kSub;       // heap scores [kMaxK][128]
-constexpr uint32_t OFF_HI = OFF_HS + kMaxK * TQ * 4; // heap ids
-constexpr uint32_t OFF_CS = OFF_HI + kMaxK * TQ * 4; // candidate scores [kBuf][128]
+constexpr uint32_t OFF_HS = OFF_V + ST * kSub;       // heap keys [kMaxK][128] (8 bytes)
+constexpr uint32_t OFF_CS = OFF_HS + kMaxK * TQ * 8; // candidate scores [kBuf][128]
 constexpr uint32_t OFF_CC = OFF_CS + kBuf * TQ * 4;  // candidate entry indices
 constexpr uint32_t OFF_BAR = OFF_CC + kBuf * TQ * 4;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;
@@ -64,50 +63,61 @@ constexpr uint32_t kCols = 512;
 constexpr int kLaunchRegs = 168, kRegsLow = 56, kRegsHigh = 224;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 
-// The K best (score, block id) pairs of one row: a binary min-heap in shared
-// memory ([slot][row] layout, so the 128 rows hit distinct banks), worst pair
-// at the root.  Worst = smallest score, and among equal scores the largest id.
+// The K best (score, block id) pairs of one row: a 4-ary min-heap in shared
+// memory of packed 64-bit keys, [slot][row] layout so the 128 rows hit
+// distinct banks.  key = (order-preserving bits of the score) << 32 |
+// (0x7fffffff - id): a larger key is a better pair (higher score, or equal
+// score and lower id), so the root holds the worst pair.  Four children per
+// node keep a sift to 3 levels of 4 independent loads.
+__device__ __forceinline__ uint32_t order_bits(float s) {
+  const uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float order_value(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
 struct Heap {
-  float* hs;
-  int* hi;
+  unsigned long long* hk;
   int r, K, cnt;
-  float tau;  // raw score a candidate must beat (-inf until the heap is full)
+  float tau;  // score a candidate must beat (-inf until the heap is full)
 
-  __device__ __forceinline__ bool worse(float s1, int i1, float s2, int i2) const {
-    return s1 < s2 || (s1 == s2 && i1 > i2);
-  }
-  __device__ __forceinline__ void sift(int p, float s, int id) {
+  __device__ __forceinline__ unsigned long long at(int i) const { return hk[i * TQ + r]; }
+  __device__ __forceinline__ void put(int i, unsigned long long k) { hk[i * TQ + r] = k; }
+  __device__ __forceinline__ void sift(int p, unsigned long long key) {
     while (true) {
-      int c = 2 * p + 1;
-      if (c >= K) break;
-      float cs = hs[c * TQ + r];
-      int ci = hi[c * TQ + r];
-      if (c + 1 < K) {
-        const float s2 = hs[(c + 1) * TQ + r];
-        const int i2 = hi[(c + 1) * TQ + r];
-        if (worse(s2, i2, cs, ci)) cs = s2, ci = i2, c = c + 1;
+      const int c0 = 4 * p + 1;
+      if (c0 >= K) break;
+      unsigned long long m = at(c0);
+      int mc = c0;
+#pragma unroll
+      for (int t = 1; t < 4; ++t) {
+        if (c0 + t < K) {
+          const unsigned long long x = at(c0 + t);
+          if (x < m) m = x, mc = c0 + t;
+        }
       }
-      if (!worse(cs, ci, s, id)) break;
-      hs[p * TQ + r] = cs;
-      hi[p * TQ + r] = ci;
-      p = c;
+      if (m >= key) break;
+      put(p, m);
+      p = mc;
     }
-    hs[p * TQ + r] = s;
-    hi[p * TQ + r] = id;
+    put(p, key);
   }
   __device__ __forceinline__ void push(float s, int id) {
+    const unsigned long long key =
+        ((unsigned long long)order_bits(s) << 32) | (uint32_t)(0x7fffffff - id);
     if (cnt < K) {
-      hs[cnt * TQ + r] = s;
-      hi[cnt * TQ + r] = id;
+      put(cnt, key);
       if (++cnt == K) {
-        for (int p = K / 2 - 1; p >= 0; --p) sift(p, hs[p * TQ + r], hi[p * TQ + r]);
-        tau = hs[r];
+        for (int p = (K - 2) / 4; p >= 0; --p) sift(p, at(p));
+        tau = order_value((uint32_t)(at(0) >> 32));
       }
-    } else {
-      sift(0, s, id);
-      tau = hs[r];
+      return;
     }
+    sift(0, key);
+    tau = order_value((uint32_t)(at(0) >> 32));
   }
+  __device__ __forceinline__ int id_of(int i) const { return 0x7fffffff - (int)(uint32_t)at(i); }
+  __device__ __forceinline__ float score_of(int i) const { return order_value((uint32_t)(at(i) >> 32)); }
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -345,18 +355,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     float* cb_s = reinterpret_cast<float*>(sp + OFF_CS);
     int* cb_e = reinterpret_cast<int*>(sp + OFF_CC);
-    Heap top{reinterpret_cast<float*>(sp + OFF_HS), reinterpret_cast<int*>(sp + OFF_HI), r, d.K, 0, -CUDART_INF_F};
+    Heap top{reinterpret_cast<unsigned long long*>(sp + OFF_HS), r, d.K, 0, -CUDART_INF_F};
     const int E = d.E, S = d.S, Bf = d.Bf;
     const int ntok = (int)n_k;
+    (void)ntok;
     int nb = 0;  // candidates waiting in this row's buffer
     // Insert the buffered candidates.  All lanes run this together, so one
     // round of insertions serves every row of the warp at once.
+    const float inv_e = 1.f / (float)E;
     auto flush = [&]() {
       for (int n = 0; n < nb; ++n) {
         const float v = cb_s[n * TQ + r];
         if (!(v > top.tau)) continue;
+        // entry e -> frame f, position i; the float quotient is off by at most one
         const int e = cb_e[n * TQ + r];
-        const int f = e / E, i = e - f * E;
+        int f = (int)((float)e * inv_e);
+        int i = e - f * E;
+        if (i < 0) i += E, --f;
+        if (i >= E) i -= E, ++f;
         if (i >= S) top.push(v, f * Bf + (i - S));  // special entries are never ranked
       }
       nb = 0;
@@ -423,17 +439,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (cand_s != nullptr) {
         for (int k = 0; k < d.K; ++k) {
           const bool have = k < top.cnt;
-          cand_s[cb + k] = have ? top.hs[k * TQ + r] * d.scale : -CUDART_INF_F;
-          cand_i[cb + k] = have ? top.hi[k * TQ + r] : -1;
+          cand_s[cb + k] = have ? top.score_of(k) * d.scale : -CUDART_INF_F;
+          cand_i[cb + k] = have ? top.id_of(k) : -1;
         }
       }
       if (sel != nullptr) {
         // the heap holds exactly this row's top-K: write its ids in ascending
         // order (rank of each id among the row's distinct ids), then -1 padding
         for (int k = 0; k < top.cnt; ++k) {
-          const int me = top.hi[k * TQ + r];
+          const int me = top.id_of(k);
           int rank = 0;
-          for (int k2 = 0; k2 < top.cnt; ++k2) rank += top.hi[k2 * TQ + r] < me;
+          for (int k2 = 0; k2 < top.cnt; ++k2) rank += top.id_of(k2) < me;
           sel[cb + rank] = me;
         }
         for (int k = top.cnt; k < d.K; ++k) sel[cb + k] = -1;

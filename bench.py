@@ -79,6 +79,11 @@ def dense_flops(z, H, D) -> int:
     return 4 * z.T * z.T * H * D
 
 
+def frame_flops(z, H, D) -> int:
+    # every token against the L tokens of its own frame: QK^T and PV
+    return 4 * z.T * z.L * H * D
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 
@@ -266,6 +271,8 @@ def main() -> None:
     ap.add_argument("--no-dense", action="store_true", help="skip the dense global attention baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
     ap.add_argument("--dense-steps", type=int, default=1)
+    ap.add_argument("--no-frame", action="store_true", help="skip the frame attention leg")
+    ap.add_argument("--frame-steps", type=int, default=5)
     ap.add_argument("--cpu-entries", type=int, default=48, help="query blocks in the cpu_baseline sample")
     ap.add_argument("--ref-entries", type=int, default=16, help="query blocks per reference-arm step")
     args = ap.parse_args()
@@ -438,6 +445,30 @@ def main() -> None:
                  "steps": args.dense_steps}
         del dout
 
+    # ---- frame attention (attention within each frame) on the same inputs ----
+    frame = None
+    if not args.no_frame:
+        fout = torch.empty_like(q)
+        for _ in range(2):
+            G.frame_attn(shape, q, k, v, fout, layer.ws, stream)
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.frame_steps):
+            G.frame_attn(shape, q, k, v, fout, layer.ws, stream)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        G.check_device_error(layer.ws)
+        fms = max_over_ranks(f0.elapsed_time(f1) / args.frame_steps)
+        tf = frame_flops(z, H, D) / (fms / 1e3) / 1e12
+        frame = {"ms_per_layer": round(fms, 3), "tokens_per_s": job_value(world, z.T, fms),
+                 "tflops": round(tf, 1), "frac_bf16_peak": round(tf / P["bf16_tflops"], 4),
+                 "kernel": "tcgen05/TMEM + TMA flash attention, one key segment per frame",
+                 "steps": args.frame_steps}
+        del fout
+
     # ---- the CPU oracle on a bounded sample, and parity of the sampled rows ----
     cpu = None
     parity = None
@@ -472,7 +503,8 @@ def main() -> None:
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded scene model, random projections)",
         "config": workload_config(wl, l2), "roofline": roofline, "stages": stages, "cpu_baseline": cpu,
-        "e2e": e2e, "gpu_launches": launches, "clocks": clk, "dense_baseline": dense, "parity": parity,
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk, "dense_baseline": dense, "frame_attention": frame,
+        "parity": parity,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -180,6 +180,16 @@ gsa_status dense_global_attn(const gsa_shape* shape, const gsa_bf16* q, const gs
                              const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream);
 
 /*
+ * Frame attention ("AVGGT: Rethinking Global Attention for Accelerating
+ * VGGT", section 2.2: the early global layers of VGGT converted to attention
+ * within each frame, O((NL)^2) -> O(N L^2)): every token attends only to the
+ * S + Hp*Wp tokens of its own frame.  out = softmax(scale * q k_f^T) v_f per
+ * frame f and head; same layouts, ownership and errors as dense_global_attn.
+ */
+gsa_status frame_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                      const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream);
+
+/*
  * dense_global_attn on the warp-level tensor-core instruction (mma.sync
  * m16n8k16), the pre-tcgen05 path; kept as a measured baseline for the
  * tcgen05 kernel.  Same arguments and result.

@@ -27,5 +27,6 @@ from .gsa_oracle import (  # noqa: F401
     combine,
     gsa_layer,
     dense_attention,
+    frame_attention,
     selection_is_valid_top_k,
 )

@@ -494,6 +494,25 @@ def dense_attention(geo: Geometry, Q, K, V, rows=None, max_bytes: int = 1 << 30)
     return out
 
 
+def frame_attention(geo: Geometry, Q, K, V, rows=None) -> np.ndarray:
+    """softmax(q K_f^T / sqrt(D)) V_f where K_f, V_f are the S + Hp*Wp tokens of
+    the query's own frame f, for fine query ``rows``.
+
+    "AVGGT: Rethinking Global Attention for Accelerating VGGT", section 2.2:
+    the early global attention layers are converted to frame attention, which
+    attends within each frame only.
+    """
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, geo.H, geo.D))
+    frame = rows // geo.L
+    for f in np.unique(frame):
+        idx = np.nonzero(frame == f)[0]
+        keys = slice(int(f) * geo.L, (int(f) + 1) * geo.L)
+        k, v = f64(K, keys), f64(V, keys)
+        out[idx] = weighted_values(softmax(qk_logits(f64(Q, rows[idx]), k, geo.sm_scale)), v)
+    return out
+
+
 # ----------------------------------------------------------------------------
 # selection checks used by parity tests
 

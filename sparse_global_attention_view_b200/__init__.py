@@ -16,6 +16,7 @@ from .api import (  # noqa: F401
     forward,
     forward_noalloc,
     forward_timed,
+    frame_attn,
     gate_combine,
     new_workspace,
     pool_kv,

@@ -78,6 +78,7 @@ SIGNATURES = {
     "gsa_gate_combine": [P_SHAPE] + [c_vp] * 7,
     "dense_global_attn": [P_SHAPE] + [c_vp] * 6,
     "dense_global_attn_mma": [P_SHAPE] + [c_vp] * 6,
+    "frame_attn": [P_SHAPE] + [c_vp] * 6,
     "gsa_forward": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp],
     "gsa_forward_timed": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp, ctypes.POINTER(c_i32), c_vp],
     "gsa_workspace_offsets": [P_SHAPE, ctypes.POINTER(GsaWsOffsets)],

@@ -162,6 +162,15 @@ def dense_global_attn(shape, q, k, v, out, ws, stream=None):
         _ptr(out, BF16, tok, "out"), _ws(ws), _stream(stream)), "dense_global_attn")
 
 
+def frame_attn(shape, q, k, v, out, ws, stream=None):
+    """Attention of every token over the tokens of its own frame only."""
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    check(load().frame_attn(
+        ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(out, BF16, tok, "out"), _ws(ws), _stream(stream)), "frame_attn")
+
+
 def dense_global_attn_mma(shape, q, k, v, out, ws, stream=None):
     """dense_global_attn on the warp-level mma.sync path (the measured baseline)."""
     z = derive(shape)

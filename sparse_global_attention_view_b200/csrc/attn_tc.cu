@@ -68,8 +68,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
-  const long long m0 = (long long)blockIdx.x * (NQT * TQ);
-  const int nt = (int)((a.n_k + TK - 1) / TK);
+  // Segments: with seg_len > 0 the rows and keys are cut into consecutive
+  // segments of seg_len tokens (frames) and every query attends only to the
+  // keys of its own segment; seg_ctas CTAs cover one segment's queries.
+  long long m0, key0, n_keys, q_end;
+  if (a.seg_len > 0) {
+    const long long f = blockIdx.x / a.seg_ctas, cx = blockIdx.x % a.seg_ctas;
+    key0 = f * a.seg_len;
+    m0 = key0 + cx * (NQT * TQ);
+    n_keys = a.seg_len;
+    q_end = min(key0 + a.seg_len, a.n_q);
+  } else {
+    key0 = 0;
+    m0 = (long long)blockIdx.x * (NQT * TQ);
+    n_keys = a.n_k;
+    q_end = a.n_q;
+  }
+  const int nt = (int)((n_keys + TK - 1) / TK);
 
   if (tid == 0) {
     mbar_init(bar(B_Q), 1);
@@ -109,8 +124,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < nt; ++j) {
         const int s = j % ST;
         if (j >= ST && !mbar_wait(bar(B_KVE + s), ((j / ST) - 1) & 1, abort_flag, a.err)) break;
-        const int c1 = a.kv_head_major ? j * TK : h;
-        const int c2 = a.kv_head_major ? h : j * TK;
+        const int kj = (int)(key0 + (long long)j * TK);
+        const int c1 = a.kv_head_major ? kj : h;
+        const int c2 = a.kv_head_major ? h : kj;
         mbar_expect_tx(bar(B_KF + s), kTile);
         tma_load_3d(sK + s * kTile, &tk, bar(B_KF + s), 0, c1, c2);
         mbar_expect_tx(bar(B_VF + s), kTile);
@@ -200,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + 32 * c, sv[c]);
       tmem_wait_ld();
-      const long long rem = a.n_k - (long long)j * TK;
+      const long long rem = n_keys - (long long)j * TK;
       if (rem < TK) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -259,7 +275,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       fence_after_sync();
       const long long row = m0 + t * TQ + q4 * 32 + lane;
-      const bool store = row < a.n_q;
+      const bool store = row < q_end;
       const float inv = 1.f / l;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -367,8 +383,17 @@ cudaError_t launch_attn_tc(const AttnTcArgs& a, const bf16* q, const bf16* k, co
   e = cudaFuncGetAttributes(&fa, attn_tc_kernel);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  dim3 grid((unsigned)((a.n_q + NQT * TQ - 1) / (NQT * TQ)), (unsigned)a.H);
-  attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, a);
+  AttnTcArgs b = a;
+  unsigned gx;
+  if (a.seg_len > 0) {
+    b.seg_ctas = (a.seg_len + NQT * TQ - 1) / (NQT * TQ);
+    gx = (unsigned)(((a.n_q + a.seg_len - 1) / a.seg_len) * b.seg_ctas);
+  } else {
+    b.seg_ctas = 1;
+    gx = (unsigned)((a.n_q + NQT * TQ - 1) / (NQT * TQ));
+  }
+  dim3 grid(gx, (unsigned)a.H);
+  attn_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, b);
   return cudaGetLastError();
 }
 

@@ -272,6 +272,31 @@ gsa_status dense_global_attn(const gsa_shape* shape, const gsa_bf16* q, const gs
   a.lse_row = a.lse_head = 0;
   a.err = (unsigned*)ws;
   a.kv_head_major = 0;
+  a.seg_len = 0;
+  return cuda_status(gsa::launch_attn_tc(a, (const bf16*)q, (const bf16*)k, (const bf16*)v, d.T,
+                                         as_stream(stream)));
+}
+
+gsa_status frame_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
+                      const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(out) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  gsa::AttnTcArgs a;
+  a.n_q = a.n_k = d.T;
+  a.H = d.H;
+  a.c2 = d.scale_log2;
+  a.out = out;
+  a.out_f32 = 0;
+  a.o_row = (long long)d.H * gsa::kHeadDim;
+  a.o_head = gsa::kHeadDim;
+  a.lse = nullptr;
+  a.lse_row = a.lse_head = 0;
+  a.err = (unsigned*)ws;
+  a.kv_head_major = 0;
+  a.seg_len = d.L;
   return cuda_status(gsa::launch_attn_tc(a, (const bf16*)q, (const bf16*)k, (const bf16*)v, d.T,
                                          as_stream(stream)));
 }
@@ -386,6 +411,7 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
     a.lse_head = 1;
     a.err = (unsigned*)ws;
     a.kv_head_major = 1;
+    a.seg_len = 0;
     if (!step(gsa::launch_attn_tc(a, (const bf16*)q, ks, vs, d.NS, s), 5)) return GSA_ERR_CUDA;
   } else if (!mark(5)) {
     return GSA_ERR_CUDA;

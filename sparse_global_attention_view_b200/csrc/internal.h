@@ -46,6 +46,8 @@ struct AttnTcArgs {
   long long lse_row, lse_head;
   unsigned* err;  // device error word
   int kv_head_major;
+  long long seg_len;   // > 0: attention within consecutive segments of this many tokens
+  long long seg_ctas;  // set by the launcher
 };
 cudaError_t launch_attn_tc(const AttnTcArgs& a, const bf16* q, const bf16* k, const bf16* v,
                            long long kv_rows, cudaStream_t st);

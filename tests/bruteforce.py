@@ -125,3 +125,18 @@ def dense_bruteforce(Q, K, V):
     scale = 1.0 / math.sqrt(D)
     return [[_attend(Q[t][h], [K[j][h] for j in range(T)], [V[j][h] for j in range(T)], scale)
              for h in range(H)] for t in range(T)]
+
+
+def frame_bruteforce(Q, K, V, tokens_per_frame):
+    """Attention of every token over the tokens of its own frame only."""
+    T = len(Q)
+    H = len(Q[0])
+    D = len(Q[0][0])
+    scale = 1.0 / math.sqrt(D)
+    out = []
+    for t in range(T):
+        start = (t // tokens_per_frame) * tokens_per_frame
+        keys = range(start, start + tokens_per_frame)
+        out.append([_attend(Q[t][h], [K[j][h] for j in keys], [V[j][h] for j in keys], scale)
+                    for h in range(H)])
+    return out

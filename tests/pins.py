@@ -251,6 +251,23 @@ def pin_row_subset():
           O.dense_attention(geo, x.q, x.k, x.v)[rows], what="row subset dense")
 
 
+def pin_frame_attention():
+    """Frame attention: one frame = dense attention; several frames = torch's
+    SDPA applied to each frame's slice; and the independent brute force."""
+    geo1, x1 = micro(N=1, S=2, Hp=4, Wp=5, H=2, D=16)
+    close(O.frame_attention(geo1, x1.q, x1.k, x1.v), sdpa_dense(x1.q, x1.k, x1.v), what="frame(N=1)")
+    geo, x = micro(N=3, S=1, Hp=3, Wp=4, H=2, D=8)
+    got = O.frame_attention(geo, x.q, x.k, x.v)
+    L = geo.L
+    want = np.concatenate([sdpa_dense(x.q[f * L:(f + 1) * L], x.k[f * L:(f + 1) * L], x.v[f * L:(f + 1) * L])
+                           for f in range(geo.N)])
+    close(got, want, what="frame vs per-frame sdpa")
+    Q, K, V = (t.to(torch.float64).tolist() for t in (x.q, x.k, x.v))
+    close(got, bruteforce.frame_bruteforce(Q, K, V, L), what="frame brute force")
+    rows = np.array([0, L - 1, L, 2 * L + 3])
+    close(O.frame_attention(geo, x.q, x.k, x.v, rows=rows), got[rows], what="frame row subset")
+
+
 def all_pins(fixture_path):
     return {
         "block_structure": lambda: pin_block_structure(fixture_path),
@@ -267,4 +284,5 @@ def all_pins(fixture_path):
         "bruteforce_dense": pin_bruteforce_dense,
         "frame_permutation": pin_frame_permutation,
         "row_subset": pin_row_subset,
+        "frame_attention": pin_frame_attention,
     }

@@ -147,6 +147,29 @@ def test_dense_full(name):
     PT.assert_close(out, ref, f"{name} dense")
 
 
+@pytest.mark.parametrize("name", ["tiny", "p3_ragged", "p2_onehead", "nine_tokens", "one_frame"])
+def test_frame_attention_full(name):
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    out = torch.full_like(st.q, float("nan"))
+    G.frame_attn(shape, st.q, st.k, st.v, out, st.ws)
+    ref = O.frame_attention(geo, x.q, x.k, x.v)
+    assert PT.zeros_fail(ref)
+    PT.assert_close(out, ref, f"{name} frame attention")
+
+
+@pytest.mark.parametrize("name", ["small"])
+def test_frame_attention_sampled(name):
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    out = torch.full_like(st.q, float("nan"))
+    G.frame_attn(shape, st.q, st.k, st.v, out, st.ws)
+    rows = sample_rows(geo.T, 512, seed=4, forced=PT.forced_rows(geo))
+    PT.assert_close(out[torch.as_tensor(rows).cuda()], O.frame_attention(geo, x.q, x.k, x.v, rows=rows),
+                    f"{name} frame attention sampled")
+    assert not torch.isnan(out).any()
+
+
 @pytest.mark.parametrize("name", ["tiny", "p3_ragged", "nine_tokens"])
 def test_dense_warp_mma_baseline(name):
     import sparse_global_attention_view_b200 as G

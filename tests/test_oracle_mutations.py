@@ -78,6 +78,18 @@ def _block_rows_cols_short(self, br, bc):
             range(self.P * bc, min(self.P * bc + self.P, self.Wp)))
 
 
+def _frame_attention_next_frame(geo, Q, K, V, rows=None):
+    # attends to the following frame's tokens (wrong key range)
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.empty((rows.size, geo.H, geo.D))
+    for n, t in enumerate(rows):
+        f = (int(t) // geo.L + 1) % geo.N
+        keys = slice(f * geo.L, (f + 1) * geo.L)
+        out[n] = O.weighted_values(O.softmax(O.qk_logits(O.f64(Q, [t]), O.f64(K, keys), geo.sm_scale)),
+                                   O.f64(V, keys))[0]
+    return out
+
+
 def _gate_wrong_sign(geo, Qc_rows, w):
     return 1.0 - _orig["gate"](geo, Qc_rows, w)
 
@@ -97,6 +109,7 @@ MUTATIONS = {
     "last block row loses a patch row": ("Geometry.block_rows_cols", _block_rows_cols_short),
     "gate sigmoid of -z": ("gate", _gate_wrong_sign),
     "softmax scale 1/D": ("Geometry.sm_scale", property(lambda self: 1.0 / self.D)),
+    "frame attention over the next frame": ("frame_attention", _frame_attention_next_frame),
 }
 
 

@@ -29,11 +29,18 @@ Where the pages are silent, the readings used here are:
     up-sampling is nearest (each fine token takes its block's output);
   * special tokens are singleton entries of the compressed sequence (they
     are not pooled), take part in compressed attention as queries and keys,
-    are not top-K candidates, and are always attended to by the selection
-    branch;
+    and are not top-K candidates;
+  * the always-kept set of the selection branch is, by default ("specials"),
+    every special token of every frame; the "reference" reading of the
+    Speed3R-VGGT adaptation keeps instead the whole reference frame (frame
+    0: its specials and patches) plus the camera token (special slot 0) of
+    every other frame, and frame 0's blocks are then not top-K candidates
+    (they are attended to already); the register tokens (slots >= 1) of
+    frames 1..N-1 then take part in the compression branch only;
   * the score ranked by top-K is the scaled logit (q_mean . k_mean) / sqrt(D);
     selection is per head and per query block; ties go to the lower block id;
-    K_eff = min(K, number of patch blocks);
+    K_eff = min(K, number of candidate blocks), which is 0 for one frame in
+    the "reference" reading;
   * a selected partial edge block contributes only its valid tokens;
   * one softmax scale 1/sqrt(D) for every attention;
   * the gate is g = sigmoid(q_mean . w_h) per (query block, head); g weights
@@ -47,6 +54,7 @@ full-size workloads never need a float64 copy of the whole tensor.
 from __future__ import annotations
 
 import dataclasses
+import functools
 import math
 
 import numpy as np
@@ -80,6 +88,7 @@ class Geometry:
     P: int
     K: int
     scale: float | None = None
+    keep: str = "specials"  # "specials" | "reference"
 
     @property
     def L(self) -> int:
@@ -114,8 +123,14 @@ class Geometry:
         return self.N * self.Bf
 
     @property
+    def B0(self) -> int:
+        """First top-K candidate block: frame 0's blocks are excluded when
+        frame 0 is kept whole."""
+        return self.Bf if self.keep == "reference" else 0
+
+    @property
     def K_eff(self) -> int:
-        return min(self.K, self.NB)
+        return min(self.K, self.NB - self.B0)
 
     @property
     def sm_scale(self) -> float:
@@ -142,7 +157,10 @@ class Geometry:
         f, j = divmod(int(beta), self.Bf)
         br, bc = divmod(j, self.Bw)
         rows, cols = self.block_rows_cols(br, bc)
-        return np.array([self.patch_token(f, r, c) for r in rows for c in cols], dtype=np.int64)
+        # patch_token(f, r, c) for r in rows, c in cols (row-major)
+        r = np.arange(rows.start, rows.stop, dtype=np.int64)
+        c = np.arange(cols.start, cols.stop, dtype=np.int64)
+        return (f * self.L + self.S + r[:, None] * self.Wp + c[None, :]).ravel()
 
     def entry_of_block(self, beta: int) -> int:
         f, j = divmod(int(beta), self.Bf)
@@ -162,18 +180,43 @@ class Geometry:
         return self.block_tokens(f * self.Bf + (j - self.S))
 
     def special_tokens(self) -> np.ndarray:
-        return np.array([self.special_token(f, j) for f in range(self.N) for j in range(self.S)],
-                        dtype=np.int64)
+        return _special_tokens(self)
+
+    def kept_tokens(self) -> np.ndarray:
+        """Token ids the selection branch always attends to, each listed once."""
+        return _kept_tokens(self)
 
     def patch_block_entries(self) -> np.ndarray:
-        """Compressed-sequence index of every patch block, in block-id order."""
-        return np.array([self.entry_of_block(b) for b in range(self.NB)], dtype=np.int64)
+        """Compressed-sequence index of every patch block, in block-id order
+        (entry_of_block over all ids)."""
+        beta = np.arange(self.NB, dtype=np.int64)
+        return (beta // self.Bf) * self.E + self.S + beta % self.Bf
+
+
+@functools.lru_cache(maxsize=64)
+def _special_tokens(geo: Geometry) -> np.ndarray:
+    ids = np.array([geo.special_token(f, j) for f in range(geo.N) for j in range(geo.S)], dtype=np.int64)
+    ids.flags.writeable = False
+    return ids
+
+
+@functools.lru_cache(maxsize=64)
+def _kept_tokens(geo: Geometry) -> np.ndarray:
+    if geo.keep == "specials":
+        return _special_tokens(geo)
+    assert geo.keep == "reference", geo.keep
+    frame0 = list(range(geo.L))
+    cameras = [geo.special_token(f, 0) for f in range(1, geo.N)] if geo.S > 0 else []
+    ids = np.array(frame0 + cameras, dtype=np.int64)
+    ids.flags.writeable = False
+    return ids
 
 
 def geometry_of(workload, **overrides) -> Geometry:
     """Geometry of a ``synthetic.Workload`` (fields copied by name)."""
     g = Geometry(N=workload.n_frames, S=workload.n_special, Hp=workload.hp, Wp=workload.wp,
-                 H=workload.n_heads, D=workload.head_dim, P=workload.pool, K=workload.top_k)
+                 H=workload.n_heads, D=workload.head_dim, P=workload.pool, K=workload.top_k,
+                 keep="reference" if getattr(workload, "keep", 0) == 1 else "specials")
     return dataclasses.replace(g, **overrides) if overrides else g
 
 
@@ -189,7 +232,7 @@ def f64(x, rows=None) -> np.ndarray:
         elif isinstance(rows, slice):
             t = x[rows]
         else:
-            t = x[torch.as_tensor(np.asarray(rows), dtype=torch.long)]
+            t = x[torch.as_tensor(np.array(rows, dtype=np.int64))]
         return t.to(torch.float64).numpy()
     a = np.asarray(x)
     return (a if rows is None else a[rows]).astype(np.float64)
@@ -198,15 +241,17 @@ def f64(x, rows=None) -> np.ndarray:
 def f64_head(x, rows, h: int) -> np.ndarray:
     """Exact float64 copy of ``x[rows, h]``: [len(rows), D]."""
     if isinstance(x, torch.Tensor):
-        return x[torch.as_tensor(np.asarray(rows), dtype=torch.long), h].to(torch.float64).numpy()
+        return x[torch.as_tensor(np.array(rows, dtype=np.int64)), h].to(torch.float64).numpy()
     return np.asarray(x)[np.asarray(rows), h].astype(np.float64)
 
 
 def softmax(z: np.ndarray, axis: int = -1) -> np.ndarray:
-    """Textbook softmax, shifted by the maximum for range (exact in real arithmetic)."""
-    m = np.max(z, axis=axis, keepdims=True)
-    e = np.exp(z - m)
-    return e / np.sum(e, axis=axis, keepdims=True)
+    """Textbook softmax, shifted by the maximum for range (exact in real
+    arithmetic); float64 torch CPU ops, which use every core."""
+    t = torch.from_numpy(np.asarray(z, dtype=np.float64))
+    m = torch.amax(t, dim=axis, keepdim=True)
+    e = torch.exp(t - m)
+    return (e / torch.sum(e, dim=axis, keepdim=True)).numpy()
 
 
 # ----------------------------------------------------------------------------
@@ -283,40 +328,57 @@ def guide_scores(geo: Geometry, logits: np.ndarray) -> np.ndarray:
     produces a score matrix S_guide that identifies the most relevant regions.
     Column beta is patch block beta; special entries are not candidates.
     """
-    return logits[..., geo.patch_block_entries()]
+    idx = torch.from_numpy(geo.patch_block_entries())
+    return torch.from_numpy(logits).index_select(-1, idx).numpy()
+
+
+def largest_values(x: np.ndarray, k: int) -> np.ndarray:
+    """The k largest values along the last axis, in descending order:
+    [..., k] (torch.topk as the selection routine; only values are used, so
+    its order among equal values does not matter)."""
+    return torch.topk(torch.from_numpy(x), k, dim=-1, sorted=True).values.numpy()
 
 
 def top_k_blocks(geo: Geometry, guide: np.ndarray) -> np.ndarray:
     """Top-K patch blocks per (query, head): [rows, H, K] ascending ids, -1 pad.
 
     Speed3R, technical summary 2.1, selection branch: the K most relevant
-    token regions for each query by the compressed branch's scores.  Blocks
-    are ranked by (-score, block id), so equal scores go to the lower id; the
-    first K_eff = min(K, NB) are kept.  (The candidates are first narrowed to
-    the blocks scoring at least the K-th largest score, which cannot change
-    the ranking's first K_eff entries.)
+    token regions for each query by the compressed branch's scores.  The
+    candidates are the blocks beta >= B0; they are ranked by (-score, block
+    id), so equal scores go to the lower id; the first K_eff are kept.  (The
+    candidates are first narrowed to the blocks scoring at least the K-th
+    largest score, which cannot change the ranking's first K_eff entries.)
     """
     rows, H, NB = guide.shape
     k = geo.K_eff
     sel = np.full((rows, H, geo.K), -1, dtype=np.int64)
-    kth = -np.partition(-guide, k - 1, axis=-1)[..., k - 1]
-    for a in range(rows):
-        for h in range(H):
-            g = guide[a, h]
-            cand = np.nonzero(g >= kth[a, h])[0]
-            ranked = cand[np.lexsort((cand, -g[cand]))]
-            sel[a, h, :k] = np.sort(ranked[:k])
+    if k == 0:
+        return sel
+    cg = guide[..., geo.B0:]
+    kth = largest_values(cg, k)[..., k - 1]
+    # every (row, head) has at least k candidates (those tied at the threshold too)
+    r, h, c = np.nonzero(cg >= kth[..., None])
+    # rank within each (row, head) by score descending, then block id ascending
+    order = np.lexsort((c, -cg[r, h, c], h, r))
+    r, h, c = r[order], h[order], c[order]
+    first = np.ones(r.size, dtype=bool)
+    first[1:] = (r[1:] != r[:-1]) | (h[1:] != h[:-1])
+    start = np.flatnonzero(first)
+    rank = np.arange(r.size) - np.repeat(start, np.diff(np.append(start, r.size)))
+    chosen = (geo.B0 + c[rank < k]).reshape(rows, H, k)
+    sel[..., :k] = np.sort(chosen, axis=-1)
     return sel
 
 
 def top_k_gap(geo: Geometry, guide: np.ndarray) -> np.ndarray:
     """s_(K) - s_(K+1) per (query, head), the K-th minus the (K+1)-th largest
-    score (inf when every block is selected)."""
-    if geo.K_eff >= guide.shape[-1]:
+    score among the candidate blocks (inf when every candidate is selected)."""
+    cg = guide[..., geo.B0:]
+    if geo.K_eff >= cg.shape[-1]:
         return np.full(guide.shape[:-1], np.inf)
     k = geo.K_eff
-    part = -np.partition(-guide, (k - 1, k), axis=-1)
-    return part[..., k - 1] - part[..., k]
+    top = largest_values(cg, k + 1)
+    return top[..., k - 1] - top[..., k]
 
 
 # ----------------------------------------------------------------------------
@@ -324,16 +386,13 @@ def top_k_gap(geo: Geometry, guide: np.ndarray) -> np.ndarray:
 
 
 def selected_keys(geo: Geometry, sel_row: np.ndarray) -> np.ndarray:
-    """Key token ids for one (query block, head): valid tokens of the selected
-    blocks, then every special token of every frame (listed once).
+    """Token ids of the selected regions for one (query block, head): the valid
+    tokens of the selected blocks.
 
     Speed3R, technical summary 2.1 (selection branch: fine-grained attention on
-    only the selected key/value regions) and 2.2 (Speed3R-VGGT keeps the
-    reference-frame / camera-token information in the selection branch; here
-    every special token is always attended to).
+    only the selected key/value regions).
     """
     parts = [geo.block_tokens(b) for b in sel_row if b >= 0]
-    parts.append(geo.special_tokens())
     return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
 
 
@@ -342,13 +401,20 @@ def selected_attention(geo: Geometry, Q, K, V, sel: np.ndarray, rows: np.ndarray
     """O_sel for fine query tokens ``rows``: [len(rows), H, D].
 
     ``sel`` is [len(entries), H, K] (the top-K of each compressed entry) and
-    row t uses the selection of its own entry (its query block).  One softmax
-    runs over the whole key set of selected_keys().
+    row t uses the selection of its own entry (its query block).  The key set
+    is selected_keys() plus the always-kept tokens (``Geometry.kept_tokens``;
+    Speed3R technical summary 2.2, Speed3R-VGGT keeps the reference-frame /
+    camera-token information in the selection branch), and one softmax runs
+    over all of it.  The kept keys are the same for every query, so their
+    logits are computed once for all rows.
     """
     pos = {int(a): i for i, a in enumerate(entries)}
     rows = np.asarray(rows, dtype=np.int64)
     out = np.empty((rows.size, geo.H, geo.D), dtype=np.float64)
     q_all = f64(Q, rows)
+    kept = geo.kept_tokens()
+    k_kept, v_kept = f64(K, kept), f64(V, kept)  # [NK, H, D]
+    s_kept = qk_logits(q_all, k_kept, geo.sm_scale)  # [rows, H, NK]
     by_entry: dict[int, list[int]] = {}
     for i, t in enumerate(rows):
         by_entry.setdefault(geo.entry_of_token(int(t)), []).append(i)
@@ -357,8 +423,9 @@ def selected_attention(geo: Geometry, Q, K, V, sel: np.ndarray, rows: np.ndarray
             keys = selected_keys(geo, sel[pos[a], h])
             k = f64_head(K, keys, h)
             v = f64_head(V, keys, h)
-            s = q_all[idx, h] @ k.T * geo.sm_scale
-            out[idx, h] = softmax(s, axis=-1) @ v
+            s = np.concatenate([q_all[idx, h] @ k.T * geo.sm_scale, s_kept[idx, h]], axis=-1)
+            p = softmax(s, axis=-1)
+            out[idx, h] = p[:, :keys.size] @ v + p[:, keys.size:] @ v_kept[:, h]
     return out
 
 
@@ -412,6 +479,10 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
         Qc, Kc, Vc = pool(geo, Q), pool(geo, K), pool(geo, V)
     else:
         Qc, Kc, Vc = pooled
+    # the same [Tc, H, D] values, stored heads-first once, so that the per-chunk
+    # heads_first() calls below are free
+    Kc_keys = heads_first(Kc).transpose(1, 0, 2)
+    Vc_keys = heads_first(Vc).transpose(1, 0, 2)
     entries = np.array(sorted({geo.entry_of_token(int(t)) for t in rows}), dtype=np.int64)
     nE = entries.size
     o_cmp = np.empty((nE, geo.H, geo.D))
@@ -427,7 +498,7 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     step = max(1, chunk_elems // (geo.H * geo.Tc))
     for e0 in range(0, nE, step):
         e1 = min(nE, e0 + step)
-        o, logits = compressed_attention(geo, Qc[entries[e0:e1]], Kc, Vc)
+        o, logits = compressed_attention(geo, Qc[entries[e0:e1]], Kc_keys, Vc_keys)
         o_cmp[e0:e1] = o
         guide = guide_scores(geo, logits)
         sel[e0:e1] = top_k_blocks(geo, guide)
@@ -435,11 +506,8 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
         if keep_guide:
             guide_all[e0:e1] = guide
         if other is not None:
-            for i in range(e0, e1):
-                for h in range(geo.H):
-                    sel_exact[i, h] = np.array_equal(other[i, h], sel[i, h])
-                    sel_valid[i, h] = selection_is_valid_top_k(geo, guide[i - e0, h], other[i, h],
-                                                               tie_window)
+            sel_exact[e0:e1] = np.all(other[e0:e1] == sel[e0:e1], axis=-1)
+            sel_valid[e0:e1] = selection_valid_top_k(geo, guide, other[e0:e1], tie_window)
     sel_used = sel if other is None else other
     o_sel = selected_attention(geo, Q, K, V, sel_used, rows, entries)
     g = gate(geo, Qc[entries], w)
@@ -517,21 +585,38 @@ def frame_attention(geo: Geometry, Q, K, V, rows=None) -> np.ndarray:
 # selection checks used by parity tests
 
 
+def selection_valid_top_k(geo: Geometry, guide: np.ndarray, chosen: np.ndarray,
+                          window: float) -> np.ndarray:
+    """[rows, H] bool: ``chosen[r, h]`` (ids, -1 pad) is a top-K of ``guide[r, h]``
+    ([rows, H, NB] S_guide) up to ``window``.
+
+    A set is accepted when it has K_eff distinct ids among the candidate blocks
+    and no unchosen candidate beats a chosen one by ``window`` or more.  With
+    window 0 and no ties this is exactly the oracle's own top-K.
+    """
+    cg = guide[..., geo.B0:]
+    n_c = cg.shape[-1]
+    chosen = np.asarray(chosen, dtype=np.int64)
+    used = chosen >= 0
+    ids = np.where(used, chosen - geo.B0, 0)
+    ok = used.sum(axis=-1) == geo.K_eff
+    ok &= np.all(~used | ((ids >= 0) & (ids < n_c)), axis=-1)
+    srt = np.sort(np.where(used, chosen, -1), axis=-1)
+    ok &= ~np.any((srt[..., 1:] == srt[..., :-1]) & (srt[..., 1:] >= 0), axis=-1)
+    # padding (and out-of-range ids, already rejected) point at a spare last column
+    ids = np.where(used & (ids >= 0) & (ids < n_c), ids, n_c)
+    ext = torch.full(cg.shape[:-1] + (n_c + 1,), -np.inf, dtype=torch.float64)
+    ext[..., :n_c] = torch.from_numpy(cg)
+    ids_t = torch.from_numpy(ids)
+    picked = torch.gather(ext, -1, ids_t).numpy()
+    lo = np.where(ids < n_c, picked, np.inf).min(axis=-1, initial=np.inf)  # weakest chosen
+    ext.scatter_(-1, ids_t, -np.inf)
+    hi = ext.amax(dim=-1).numpy()                                          # strongest unchosen
+    return ok & (hi - lo < window)
+
+
 def selection_is_valid_top_k(geo: Geometry, guide_row: np.ndarray, chosen: np.ndarray,
                              window: float) -> bool:
-    """True if ``chosen`` (ids, -1 pad) is a top-K of ``guide_row`` up to ``window``.
-
-    A set is accepted when it has K_eff distinct valid ids and no unchosen
-    block beats a chosen one by more than ``window``.  With window 0 and no
-    ties this is exactly the oracle's own top-K.
-    """
-    ids = np.asarray([b for b in chosen if b >= 0], dtype=np.int64)
-    if ids.size != geo.K_eff or np.unique(ids).size != ids.size:
-        return False
-    if ids.min(initial=0) < 0 or ids.max(initial=0) >= guide_row.size:
-        return False
-    if ids.size == guide_row.size:
-        return True
-    mask = np.zeros(guide_row.size, dtype=bool)
-    mask[ids] = True
-    return bool(guide_row[~mask].max() - guide_row[mask].min() < window)
+    """selection_valid_top_k for one (row, head)."""
+    return bool(selection_valid_top_k(geo, np.asarray(guide_row)[None, None],
+                                      np.asarray(chosen)[None, None], window)[0, 0])

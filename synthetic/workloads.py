@@ -46,6 +46,9 @@ class Workload:
     kind: str  # "gaussian" | "scene"
     sigma: float = 0.3
     second_table_frac: float = 0.0
+    # always-kept set of the selection branch (a layer option, not an input
+    # property): 0 every special token, 1 frame 0 whole + each camera token
+    keep: int = 0
 
     @property
     def tokens_per_frame(self) -> int:

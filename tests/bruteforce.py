@@ -50,8 +50,14 @@ def layout(N, S, Hp, Wp, P):
     return frames
 
 
-def gsa_bruteforce(Q, K, V, w, N, S, Hp, Wp, P, topk):
-    """Q, K, V: nested lists [T][H][D] of floats; w: [H][D].  Returns dict."""
+def gsa_bruteforce(Q, K, V, w, N, S, Hp, Wp, P, topk, keep="specials"):
+    """Q, K, V: nested lists [T][H][D] of floats; w: [H][D].  Returns dict.
+
+    keep="specials": every special token is always attended to.
+    keep="reference": every token of frame 0 and the first special token of
+    each later frame are always attended to, and only the blocks of frames
+    1..N-1 are ranked.
+    """
     H = len(Q[0])
     D = len(Q[0][0])
     scale = 1.0 / math.sqrt(D)
@@ -62,14 +68,23 @@ def gsa_bruteforce(Q, K, V, w, N, S, Hp, Wp, P, topk):
     block_entry = []
     block_tokens = []
     all_specials = []
-    for specials, blocks in frames:
+    block_frame = []
+    for f, (specials, blocks) in enumerate(frames):
         for t in specials:
             entries.append([t])
             all_specials.append(t)
         for toks in blocks:
             block_entry.append(len(entries))
             block_tokens.append(toks)
+            block_frame.append(f)
             entries.append(toks)
+    if keep == "specials":
+        always = all_specials
+        rankable = list(range(len(block_entry)))
+    else:
+        per = S + Hp * Wp
+        always = list(range(per)) + [f * per for f in range(1, N) if S > 0]
+        rankable = [beta for beta in range(len(block_entry)) if block_frame[beta] > 0]
 
     def mean_of(X, toks, h):
         return [sum(X[t][h][d] for t in toks) / len(toks) for d in range(D)]
@@ -86,7 +101,8 @@ def gsa_bruteforce(Q, K, V, w, N, S, Hp, Wp, P, topk):
             o_cmp[a][h] = _attend(qc[a][h], [kc[b][h] for b in range(n_e)],
                                   [vc[b][h] for b in range(n_e)], scale)
             scored = []
-            for beta, b in enumerate(block_entry):
+            for beta in rankable:
+                b = block_entry[beta]
                 scored.append((-(_dot(qc[a][h], kc[b][h]) * scale), beta))
             scored.sort()
             chosen = sorted(beta for _, beta in scored[:min(topk, len(scored))])
@@ -111,7 +127,7 @@ def gsa_bruteforce(Q, K, V, w, N, S, Hp, Wp, P, topk):
             keys = []
             for beta in sel[a][h]:
                 keys.extend(block_tokens[beta])
-            keys.extend(all_specials)
+            keys.extend(always)
             o_sel[t][h] = _attend(Q[t][h], [K[j][h] for j in keys], [V[j][h] for j in keys], scale)
             g = gates[a][h]
             out[t][h] = [g * x + (1.0 - g) * y for x, y in zip(o_cmp[a][h], o_sel[t][h])]

@@ -17,10 +17,10 @@ from synthetic import Workload, generate
 TOL = 1e-11
 
 
-def micro(N=2, S=1, Hp=6, Wp=7, H=2, D=8, P=4, K=2, seed=5):
+def micro(N=2, S=1, Hp=6, Wp=7, H=2, D=8, P=4, K=2, seed=5, keep="specials"):
     wl = Workload("micro", N, S, Hp, Wp, H, D, P, K, seed, "gaussian")
     x = generate(wl)
-    geo = O.Geometry(N=N, S=S, Hp=Hp, Wp=Wp, H=H, D=D, P=P, K=K)
+    geo = O.Geometry(N=N, S=S, Hp=Hp, Wp=Wp, H=H, D=D, P=P, K=K, keep=keep)
     return geo, x
 
 
@@ -268,6 +268,51 @@ def pin_frame_attention():
     close(O.frame_attention(geo, x.q, x.k, x.v, rows=rows), got[rows], what="frame row subset")
 
 
+def pin_reference_one_frame():
+    """Reference-frame keep, one frame: nothing is ranked (K_eff = 0) and the
+    selection branch attends to the whole frame, i.e. it is dense attention."""
+    geo, x = micro(N=1, S=3, Hp=6, Wp=5, H=2, D=8, P=2, K=4, keep="reference")
+    assert geo.K_eff == 0
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    assert (res["sel"] == -1).all()
+    close(res["o_sel"], sdpa_dense(x.q, x.k, x.v), what="reference keep, one frame")
+
+
+def pin_reference_k_all():
+    """Reference-frame keep with every candidate block selected: the key set is
+    every token except the register tokens (special slots >= 1) of frames
+    1..N-1, so the selection branch is SDPA under that key mask; with one
+    special token per frame it is plain dense attention."""
+    geo, x = micro(N=3, S=3, Hp=5, Wp=6, H=2, D=8, P=4, K=64, keep="reference")
+    assert geo.K_eff == geo.NB - geo.Bf
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    L = geo.L
+    allowed = torch.ones(geo.T, dtype=torch.bool)
+    for f in range(1, geo.N):
+        allowed[f * L + 1:f * L + geo.S] = False
+    t = lambda z: z.to(torch.float64).permute(1, 0, 2).unsqueeze(0)  # noqa: E731
+    mask = allowed[None, None, None, :].expand(1, geo.H, geo.T, geo.T)
+    want = torch.nn.functional.scaled_dot_product_attention(t(x.q), t(x.k), t(x.v), attn_mask=mask)
+    close(res["o_sel"], want.squeeze(0).permute(1, 0, 2).numpy(), what="reference keep, K = all")
+    geo1, x1 = micro(N=3, S=1, Hp=5, Wp=6, H=2, D=8, P=4, K=64, keep="reference")
+    res1 = O.gsa_layer(geo1, x1.q, x1.k, x1.v, x1.w)
+    close(res1["o_sel"], sdpa_dense(x1.q, x1.k, x1.v), what="reference keep, S=1, K = all")
+
+
+def pin_reference_bruteforce():
+    """Reference-frame keep on a small input with K below the candidate count:
+    the whole layer against the independent brute force."""
+    geo, x = micro(N=3, S=2, Hp=6, Wp=7, H=2, D=8, P=4, K=3, keep="reference")
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+    Q, K, V, W = (t.to(torch.float64).tolist() for t in (x.q, x.k, x.v, x.w))
+    bf = bruteforce.gsa_bruteforce(Q, K, V, W, geo.N, geo.S, geo.Hp, geo.Wp, geo.P, geo.K,
+                                   keep="reference")
+    assert res["sel"].tolist() == bf["sel"], "brute force selection (reference keep)"
+    assert (res["sel"][res["sel"] >= 0] >= geo.Bf).all(), "frame 0 blocks are not ranked"
+    close(res["o_sel"], bf["o_sel"], what="brute force o_sel (reference keep)")
+    close(res["out"], bf["out"], what="brute force out (reference keep)")
+
+
 def all_pins(fixture_path):
     return {
         "block_structure": lambda: pin_block_structure(fixture_path),
@@ -285,4 +330,7 @@ def all_pins(fixture_path):
         "frame_permutation": pin_frame_permutation,
         "row_subset": pin_row_subset,
         "frame_attention": pin_frame_attention,
+        "reference_one_frame": pin_reference_one_frame,
+        "reference_k_all": pin_reference_k_all,
+        "reference_bruteforce": pin_reference_bruteforce,
     }

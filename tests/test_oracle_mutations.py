@@ -43,13 +43,18 @@ def _top_k_ties_high(geo, guide):
     return sel
 
 
-def _selected_keys_without_specials(geo, sel_row):
-    parts = [geo.block_tokens(b) for b in sel_row if b >= 0]
-    return np.concatenate(parts)
+def _kept_nothing(self):
+    return np.zeros(0, dtype=np.int64)
 
 
-def _selected_keys_specials_twice(geo, sel_row):
-    return np.concatenate([_orig["selected_keys"](geo, sel_row), geo.special_tokens()])
+def _kept_twice(self):
+    once = _orig["Geometry.kept_tokens"](self)
+    return np.concatenate([once, once])
+
+
+def _selected_keys_drop_last_block(geo, sel_row):
+    chosen = [b for b in sel_row if b >= 0][:-1]
+    return _orig["selected_keys"](geo, np.asarray(chosen, dtype=np.int64))
 
 
 def _combine_swapped(g, o_cmp_up, o_sel):
@@ -90,18 +95,35 @@ def _frame_attention_next_frame(geo, Q, K, V, rows=None):
     return out
 
 
+def _kept_all_specials_of_later_frames(self):
+    # reference keep that also keeps the register tokens of frames 1..N-1
+    if self.keep != "reference":
+        return _orig["Geometry.kept_tokens"](self)
+    later = [self.special_token(f, j) for f in range(1, self.N) for j in range(self.S)]
+    return np.array(list(range(self.L)) + later, dtype=np.int64)
+
+
+def _kept_camera_from_last_slot(self):
+    if self.keep != "reference":
+        return _orig["Geometry.kept_tokens"](self)
+    cams = [self.special_token(f, self.S - 1) for f in range(1, self.N)] if self.S > 0 else []
+    return np.array(list(range(self.L)) + cams, dtype=np.int64)
+
+
 def _gate_wrong_sign(geo, Qc_rows, w):
     return 1.0 - _orig["gate"](geo, Qc_rows, w)
 
 
 _orig = {n: getattr(O, n) for n in ("pool", "compressed_attention", "selected_keys", "combine", "gate")}
+_orig["Geometry.kept_tokens"] = O.Geometry.kept_tokens
 
 MUTATIONS = {
     "pool divides partial blocks by P*P": ("pool", _pool_full_denominator),
     "compressed branch multiplies by K instead of V": ("compressed_attention", _compressed_values_are_keys),
     "ties go to the higher block id": ("top_k_blocks", _top_k_ties_high),
-    "selection drops the special tokens": ("selected_keys", _selected_keys_without_specials),
-    "selection lists special tokens twice": ("selected_keys", _selected_keys_specials_twice),
+    "selection drops the always-kept tokens": ("Geometry.kept_tokens", _kept_nothing),
+    "selection lists the always-kept tokens twice": ("Geometry.kept_tokens", _kept_twice),
+    "selection drops its last selected block": ("selected_keys", _selected_keys_drop_last_block),
     "gate weights the selection branch": ("combine", _combine_swapped),
     "combine drops the (1 - g) factor": ("combine", _combine_no_one_minus),
     "special entries ranked as candidates": ("guide_scores", _guide_counts_specials),
@@ -110,6 +132,9 @@ MUTATIONS = {
     "gate sigmoid of -z": ("gate", _gate_wrong_sign),
     "softmax scale 1/D": ("Geometry.sm_scale", property(lambda self: 1.0 / self.D)),
     "frame attention over the next frame": ("frame_attention", _frame_attention_next_frame),
+    "reference keep still ranks frame 0's blocks": ("Geometry.B0", property(lambda self: 0)),
+    "reference keep keeps every register token": ("Geometry.kept_tokens", _kept_all_specials_of_later_frames),
+    "reference keep takes the camera from the last slot": ("Geometry.kept_tokens", _kept_camera_from_last_slot),
 }
 
 

@@ -238,6 +238,13 @@ def f64(x, rows=None) -> np.ndarray:
     return (a if rows is None else a[rows]).astype(np.float64)
 
 
+def f64_head_all(x, h: int) -> np.ndarray:
+    """Exact float64 copy of head h of every row of ``x``: [rows, D]."""
+    if isinstance(x, torch.Tensor):
+        return x[:, h].to(torch.float64).numpy()
+    return np.asarray(x)[:, h].astype(np.float64)
+
+
 def f64_head(x, rows, h: int) -> np.ndarray:
     """Exact float64 copy of ``x[rows, h]``: [len(rows), D]."""
     if isinstance(x, torch.Tensor):
@@ -247,8 +254,15 @@ def f64_head(x, rows, h: int) -> np.ndarray:
 
 def softmax(z: np.ndarray, axis: int = -1) -> np.ndarray:
     """Textbook softmax, shifted by the maximum for range (exact in real
-    arithmetic); float64 torch CPU ops, which use every core."""
-    t = torch.from_numpy(np.asarray(z, dtype=np.float64))
+    arithmetic).  Large arrays go through float64 torch CPU ops, which use
+    every core; small ones stay in NumPy (a torch call costs more than the
+    arithmetic there)."""
+    z = np.asarray(z, dtype=np.float64)
+    if z.size < (1 << 20):
+        m = np.max(z, axis=axis, keepdims=True)
+        e = np.exp(z - m)
+        return e / np.sum(e, axis=axis, keepdims=True)
+    t = torch.from_numpy(z)
     m = torch.amax(t, dim=axis, keepdim=True)
     e = torch.exp(t - m)
     return (e / torch.sum(e, dim=axis, keepdim=True)).numpy()
@@ -418,11 +432,11 @@ def selected_attention(geo: Geometry, Q, K, V, sel: np.ndarray, rows: np.ndarray
     by_entry: dict[int, list[int]] = {}
     for i, t in enumerate(rows):
         by_entry.setdefault(geo.entry_of_token(int(t)), []).append(i)
-    for a, idx in by_entry.items():
-        for h in range(geo.H):
+    for h in range(geo.H):
+        k_h, v_h = f64_head_all(K, h), f64_head_all(V, h)  # [T, D] each
+        for a, idx in by_entry.items():
             keys = selected_keys(geo, sel[pos[a], h])
-            k = f64_head(K, keys, h)
-            v = f64_head(V, keys, h)
+            k, v = k_h[keys], v_h[keys]
             s = np.concatenate([q_all[idx, h] @ k.T * geo.sm_scale, s_kept[idx, h]], axis=-1)
             p = softmax(s, axis=-1)
             out[idx, h] = p[:, :keys.size] @ v + p[:, keys.size:] @ v_kept[:, h]
@@ -529,36 +543,46 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
 # dense global attention (the layer GSA replaces)
 
 
-def dense_attention(geo: Geometry, Q, K, V, rows=None, max_bytes: int = 1 << 30) -> np.ndarray:
+def dense_attention(geo: Geometry, Q, K, V, rows=None, key_chunk: int = 1 << 14,
+                    max_bytes: int = 1 << 30) -> np.ndarray:
     """softmax(q K^T / sqrt(D)) V over all T tokens, for fine query ``rows``.
 
     Speed3R, technical summary 1 (Background): the dense global attention of
     DUSt3R / VGGT-style models, quadratic in the number of tokens.
+
+    Up to ``key_chunk`` keys the whole score row is formed and passed to
+    softmax().  Beyond that the same softmax is written out over key slices in
+    two passes: the row maximum of the scaled logits over all keys first, then
+    sum_j exp(s_j - max) v_j and sum_j exp(s_j - max), divided at the end --
+    the textbook formula, without online rescaling.  Rows are taken in chunks
+    whose logits of one key slice fit in ``max_bytes``.
     """
     rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
     out = np.empty((rows.size, geo.H, geo.D))
-    step = max(1, min(rows.size, max_bytes // max(geo.H * geo.T * 8, 1)))
-    kc = 1 << 16
-    small = geo.T <= kc
-    if small:
+    if geo.T <= key_chunk:
         k_all, v_all = f64(K), f64(V)
+        step = max(1, max_bytes // max(geo.H * geo.T * 8, 1))
+        for r0 in range(0, rows.size, step):
+            r1 = min(rows.size, r0 + step)
+            out[r0:r1] = weighted_values(softmax(qk_logits(f64(Q, rows[r0:r1]), k_all, geo.sm_scale)), v_all)
+        return out
+    step = max(1, max_bytes // (geo.H * key_chunk * 8))
+    slices = [slice(t0, min(geo.T, t0 + key_chunk)) for t0 in range(0, geo.T, key_chunk)]
     for r0 in range(0, rows.size, step):
         r1 = min(rows.size, r0 + step)
         q = f64(Q, rows[r0:r1])
-        if small:
-            out[r0:r1] = weighted_values(softmax(qk_logits(q, k_all, geo.sm_scale)), v_all)
-            continue
-        # the full score row is built key slice by key slice, then one softmax
-        s = np.empty((r1 - r0, geo.H, geo.T))
-        for t0 in range(0, geo.T, kc):
-            t1 = min(geo.T, t0 + kc)
-            s[..., t0:t1] = qk_logits(q, f64(K, slice(t0, t1)), geo.sm_scale)
-        p = softmax(s)
-        acc = np.zeros((r1 - r0, geo.H, geo.D))
-        for t0 in range(0, geo.T, kc):
-            t1 = min(geo.T, t0 + kc)
-            acc += weighted_values(p[..., t0:t1], f64(V, slice(t0, t1)))
-        out[r0:r1] = acc
+        m = torch.full((r1 - r0, geo.H), -np.inf, dtype=torch.float64)
+        for sl in slices:
+            s = torch.from_numpy(qk_logits(q, f64(K, sl), geo.sm_scale))
+            m = torch.maximum(m, s.amax(dim=-1))
+        num = np.zeros((r1 - r0, geo.H, geo.D))
+        den = np.zeros((r1 - r0, geo.H))
+        for sl in slices:
+            s = torch.from_numpy(qk_logits(q, f64(K, sl), geo.sm_scale))
+            e = torch.exp(s - m[..., None])
+            den += e.sum(dim=-1).numpy()
+            num += weighted_values(e.numpy(), f64(V, sl))
+        out[r0:r1] = num / den[..., None]
     return out
 
 

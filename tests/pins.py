@@ -214,6 +214,15 @@ def pin_bruteforce_layer():
     close(res["out"], bf["out"], what="brute force out")
 
 
+def pin_dense_key_slices():
+    """The sliced two-pass form of dense_attention (used for long sequences)
+    equals torch's SDPA: slices of 7 keys over 60 tokens, ragged last slice,
+    row chunks of 3."""
+    geo, x = micro(N=2, S=2, Hp=4, Wp=7, H=2, D=8)
+    got = O.dense_attention(geo, x.q, x.k, x.v, key_chunk=7, max_bytes=3 * geo.H * 7 * 8)
+    close(got, sdpa_dense(x.q, x.k, x.v), what="dense in key slices vs sdpa")
+
+
 def pin_bruteforce_dense():
     geo, x = micro(N=2, S=1, Hp=3, Wp=4, H=2, D=8)
     Q, K, V = (t.to(torch.float64).tolist() for t in (x.q, x.k, x.v))
@@ -330,6 +339,7 @@ def all_pins(fixture_path):
         "frame_permutation": pin_frame_permutation,
         "row_subset": pin_row_subset,
         "frame_attention": pin_frame_attention,
+        "dense_key_slices": pin_dense_key_slices,
         "reference_one_frame": pin_reference_one_frame,
         "reference_k_all": pin_reference_k_all,
         "reference_bruteforce": pin_reference_bruteforce,

@@ -110,11 +110,22 @@ def _kept_camera_from_last_slot(self):
     return np.array(list(range(self.L)) + cams, dtype=np.int64)
 
 
+def _dense_sliced_drops_last_slice(geo, Q, K, V, rows=None, key_chunk=1 << 14, max_bytes=1 << 30):
+    if geo.T <= key_chunk:
+        return _orig["dense_attention"](geo, Q, K, V, rows, key_chunk, max_bytes)
+    # the keys of the ragged last slice are lost
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows)
+    n = (geo.T - 1) // key_chunk * key_chunk
+    k, v = O.f64(K, slice(0, n)), O.f64(V, slice(0, n))
+    return O.weighted_values(O.softmax(O.qk_logits(O.f64(Q, rows), k, geo.sm_scale)), v)
+
+
 def _gate_wrong_sign(geo, Qc_rows, w):
     return 1.0 - _orig["gate"](geo, Qc_rows, w)
 
 
-_orig = {n: getattr(O, n) for n in ("pool", "compressed_attention", "selected_keys", "combine", "gate")}
+_orig = {n: getattr(O, n) for n in ("pool", "compressed_attention", "selected_keys", "combine", "gate",
+                                     "dense_attention")}
 _orig["Geometry.kept_tokens"] = O.Geometry.kept_tokens
 
 MUTATIONS = {
@@ -132,6 +143,7 @@ MUTATIONS = {
     "gate sigmoid of -z": ("gate", _gate_wrong_sign),
     "softmax scale 1/D": ("Geometry.sm_scale", property(lambda self: 1.0 / self.D)),
     "frame attention over the next frame": ("frame_attention", _frame_attention_next_frame),
+    "sliced dense attention drops the ragged last slice": ("dense_attention", _dense_sliced_drops_last_slice),
     "reference keep still ranks frame 0's blocks": ("Geometry.B0", property(lambda self: 0)),
     "reference keep keeps every register token": ("Geometry.kept_tokens", _kept_all_specials_of_later_frames),
     "reference keep takes the camera from the last slot": ("Geometry.kept_tokens", _kept_camera_from_last_slot),

@@ -57,18 +57,21 @@ def peaks() -> dict:
 
 def stage_work(z, H, D, K_eff) -> dict:
     """Per-stage algorithmic work of one layer: (bound, amount, unit)."""
-    T, Tc, NB, NS = z.T, z.Tc, z.NB, z.NS
+    T, Tc, NB, NS, NK = z.T, z.Tc, z.NB, z.NS, z.NK
     return {
-        # read Q, K, V once; write qc32, kc32 (fp32), vc, qc, kc (bf16) and the special copies
-        "pool": ("hbm", 3 * T * H * D * 2 + Tc * H * D * (4 + 4 + 2 + 2 + 2) + 2 * NS * H * D * 2, "bytes"),
+        # read Q, K, V once; write qc32, kc32 (fp32), vc, qc, kc (bf16) and the
+        # head-major copies of the always-kept tokens' K, V (read again when they
+        # are not the specials)
+        "pool": ("hbm", 3 * T * H * D * 2 + Tc * H * D * (4 + 4 + 2 + 2 + 2) + 2 * NK * H * D * 2
+                 + (2 * NK * H * D * 2 if NK != NS else 0), "bytes"),
         # QK^T and PV over the Tc x Tc pooled sequence
         "compressed_attn": ("tensor", 4 * Tc * Tc * H * D, "flop"),
-        # one fp32 dot product of length D per (entry, patch block, head)
-        "block_scores": ("alu", 2 * Tc * NB * H * D, "flop"),
+        # one fp32 dot product of length D per (entry, candidate block, head)
+        "block_scores": ("alu", 2 * Tc * (NB - z.B0) * H * D, "flop"),
         # candidates read once, selection written once
         "topk_merge": ("hbm", H * Tc * K_eff * 8 + H * Tc * K_eff * 4, "bytes"),
-        # QK^T and PV of every token over all N*S special tokens
-        "specials_attn": ("tensor", 4 * T * NS * H * D, "flop"),
+        # QK^T and PV of every token over the NK always-kept tokens
+        "kept_attn": ("tensor", 4 * T * NK * H * D, "flop"),
         # the selected blocks' K and V gathered per (entry, head): K_eff blocks of
         # (at most) 16 tokens x 128 bytes, K and V
         "selected_gate": ("hbm", H * Tc * K_eff * 16 * D * 2 * 2, "bytes"),
@@ -172,7 +175,7 @@ def run_reference(args) -> None:
     if rank != 0:
         return
     torch.set_num_threads(os.cpu_count() or 1)
-    wl = WORKLOADS[args.workload]
+    wl = chosen_workload(args)
     x = generate(wl)
     from oracle import gsa_oracle as O
     geo = O.geometry_of(wl)
@@ -204,12 +207,23 @@ def run_reference(args) -> None:
     print(json.dumps(line), flush=True)
 
 
+def chosen_workload(args):
+    wl = WORKLOADS[args.workload]
+    if args.top_k is not None:
+        wl = wl.with_(top_k=args.top_k)
+    if args.keep:
+        wl = wl.with_(keep=args.keep)
+    return wl
+
+
 def workload_config(wl, l2_note=None) -> dict:
+    kept = ("frame 0 + every camera token always kept" if wl.keep == 1 else "every special token always kept")
     c = {"workload": f"{wl.name}: N={wl.n_frames} frames x ({wl.n_special} special + {wl.hp}x{wl.wp} patches) "
                      f"= {wl.n_tokens} tokens, {wl.n_heads} heads x {wl.head_dim}, pool {wl.pool}x{wl.pool}, "
-                     f"top-K {wl.top_k}, {wl.kind} generator seed {wl.seed}",
+                     f"top-K {wl.top_k}, {kept}, {wl.kind} generator seed {wl.seed}",
          "n_frames": wl.n_frames, "tokens": wl.n_tokens, "heads": wl.n_heads, "head_dim": wl.head_dim,
-         "pool": wl.pool, "top_k": wl.top_k, "parallelism": "replicas (independent scene per rank)"}
+         "pool": wl.pool, "top_k": wl.top_k, "keep": "reference" if wl.keep == 1 else "specials",
+         "parallelism": "replicas (independent scene per rank)"}
     if l2_note:
         c["l2"] = l2_note
     return c
@@ -258,7 +272,7 @@ def job_value(world: int, tokens_per_rank: int, step_ms_max: float) -> float:
 
 
 STAGE_SOURCE = {"pool": "pool.cu", "compressed_attn": "attn_cmp_tc.cu", "block_scores": "topk.cu",
-                "topk_merge": "topk.cu", "specials_attn": "attn_tc.cu", "selected_gate": "selected.cu"}
+                "topk_merge": "topk.cu", "kept_attn": "attn_tc.cu", "selected_gate": "selected.cu"}
 
 
 def main() -> None:
@@ -268,6 +282,9 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["gsa", "reference"], default="gsa")
     ap.add_argument("--workload", choices=list(WORKLOADS), default="pages")
+    ap.add_argument("--top-k", type=int, default=None, help="override the workload's top-K (e.g. 128)")
+    ap.add_argument("--keep", type=int, choices=[0, 1], default=0,
+                    help="always-kept set: 0 every special token, 1 frame 0 + camera tokens")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense global attention baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
     ap.add_argument("--dense-steps", type=int, default=1)
@@ -301,7 +318,7 @@ def main() -> None:
     def max_over_ranks(v: float) -> float:
         return reduce_max(v, dist, torch.device("cuda", local))
 
-    wl = rank_workload(WORKLOADS[args.workload], rank)
+    wl = rank_workload(chosen_workload(args), rank)
     x = generate(wl)
     shape = G.Shape.of(wl)
     z = G.derive(shape)

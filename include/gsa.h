@@ -12,7 +12,11 @@
  *   - S_guide: the pooled scores of each compressed query against every patch
  *     block; the Top-K blocks per (query block, head) are selected;
  *   - selection branch: fine attention of each token over the tokens of its
- *     block's selected blocks plus every special token (always kept);
+ *     block's selected blocks plus an always-kept token set: every special
+ *     token (keep = GSA_KEEP_SPECIALS), or the whole reference frame 0 plus
+ *     the camera token of every frame (keep = GSA_KEEP_REFERENCE, the
+ *     Speed3R-VGGT reading of "reference-frame and camera tokens are always
+ *     kept"; frame 0's blocks are then not top-K candidates);
  *   - gated aggregation: g = sigmoid(q_mean . w_h) per (query block, head),
  *     out = g * up(O_cmp) + (1 - g) * O_sel.
  *
@@ -26,7 +30,12 @@
  * stored [Tc][H][64].  Patch block id beta = f*Bh*Bw + br*Bw + bc (0 <= beta <
  * NB = N*Bh*Bw).  A block at the right/bottom edge holds only the patches that
  * exist; its pooled value is the mean over those.
- * Special-token copies: [H][N*S][64] bf16 (head-major, frame-major).
+ * Always-kept copies: [H][NK][64] bf16 (head-major) of the always-kept tokens'
+ * K / V in token order: NK = N*S (all specials, frame-major) for
+ * GSA_KEEP_SPECIALS; NK = (S + Hp*Wp) + (N-1)*min(S,1) for GSA_KEEP_REFERENCE
+ * (frame 0's tokens, then special slot 0 -- the camera token -- of frames
+ * 1..N-1).  Top-K candidates are the blocks beta >= B0 (B0 = 0, or Bh*Bw for
+ * GSA_KEEP_REFERENCE); K_eff = min(K, NB - B0), which may be 0.
  *
  * Pointers: every buffer pointer is a device pointer (cudaMalloc'd or a slice of
  * one) and must be 16-byte aligned; the caller owns all memory and the library
@@ -79,7 +88,11 @@ typedef struct {
   int32_t pool;      /* P in [1, 4]: P x P average pooling of the patch grid */
   int32_t top_k;     /* K in [1, 128]: selected blocks per (query block, head) */
   float scale;       /* softmax scale; 0 means 1/sqrt(D) */
+  int32_t keep;      /* always-kept set of the selection branch: GSA_KEEP_* */
 } gsa_shape;
+
+#define GSA_KEEP_SPECIALS 0  /* every special token of every frame */
+#define GSA_KEEP_REFERENCE 1 /* frame 0 whole + each frame's camera token (slot 0) */
 
 /* Derived sizes (see the conventions above). */
 typedef struct {
@@ -87,10 +100,12 @@ typedef struct {
   int64_t Tc;    /* compressed entries N*(S+Bh*Bw) */
   int64_t NB;    /* patch blocks N*Bh*Bw (top-K candidates) */
   int64_t NS;    /* special tokens N*S */
+  int64_t NK;    /* always-kept tokens (see keep) */
+  int64_t B0;    /* first top-K candidate block id */
   int32_t L;     /* tokens per frame S+Hp*Wp */
   int32_t E;     /* compressed entries per frame S+Bh*Bw */
   int32_t Bh, Bw, Bf;
-  int32_t K_eff; /* min(K, NB) */
+  int32_t K_eff; /* min(K, NB - B0) */
 } gsa_sizes;
 
 #define GSA_WS_HEADER_BYTES 256
@@ -111,8 +126,8 @@ gsa_status gsa_workspace_init(void* ws, void* stream);
  *   qc32, kc32   [Tc][H][64] fp32  mean of Q / K (scores and the gate use these)
  *   vc           [Tc][H][64] bf16  mean of V (round-to-nearest-even)
  *   qc, kc       [Tc][H][64] bf16  mean of Q / K (may be NULL: not written)
- *   ks, vs       [H][N*S][64] bf16 copies of the special tokens' K / V
- *                (ignored when S == 0; may be NULL: not written)
+ *   ks, vs       [H][NK][64] bf16 copies of the always-kept tokens' K / V
+ *                (ignored when NK == 0; may be NULL: not written)
  * A special token's entry is the token itself.
  */
 gsa_status gsa_pool_kv(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
@@ -124,7 +139,7 @@ gsa_status gsa_pool_kv(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
  * (technical summary 2.1; S_guide on the it page, section 2).
  *   oc [Tc][H][64] fp32: softmax(scale * qc kc^T) vc over all Tc entries.
  *   cand_score / cand_idx [H][Tc][n_split][K]: for every (head, entry) and each
- *   of `n_split` equal slices of the patch-block range, the K largest
+ *   of `n_split` equal slices of the candidate block range [B0, NB), the K largest
  *   S_guide[h][a][beta] = scale * (qc32[a,h] . kc32[entry(beta),h]) of that
  *   slice with their block ids, unordered, padded with (-inf, -1).
  * qc / kc are the bf16 pooled tensors of gsa_pool_kv, qc32 / kc32 the fp32 ones.
@@ -148,9 +163,10 @@ gsa_status gsa_topk_blocks(const gsa_shape* shape, const float* cand_score,
 
 /*
  * Step 5, selected attention (technical summary 2.1, selection branch;
- * 2.2, Speed3R-VGGT keeps the special/camera tokens).  For token t in
- * compressed entry a and head h: one softmax over the valid tokens of the
- * blocks sel[h][a][:] plus all N*S special tokens (ks/vs, NULL when S == 0):
+ * 2.2, Speed3R-VGGT keeps the reference-frame / camera tokens).  For token t
+ * in compressed entry a and head h: one softmax over the valid tokens of the
+ * blocks sel[h][a][:] plus the NK always-kept tokens (ks/vs from gsa_pool_kv,
+ * NULL when NK == 0):
  *   o_sel [T][H][64] bf16, and lse [T][H] fp32 = log sum exp of the scaled
  *   logits (may be NULL).
  */
@@ -200,8 +216,8 @@ gsa_status dense_global_attn_mma(const gsa_shape* shape, const gsa_bf16* q, cons
 /*
  * The whole GSA layer: steps 1-6 enqueued on `stream`, intermediates in `ws`
  * (ws_bytes >= gsa_workspace_size).  w [H][64] fp32 gate vectors; out
- * [T][H][64] bf16.  The attention over the always-kept special tokens runs on
- * the tensor-core attention kernel into the workspace; the selected blocks
+ * [T][H][64] bf16.  The attention over the always-kept tokens runs on the
+ * tensor-core attention kernel into the workspace; the selected blocks
  * continue that softmax in the step-5 kernel, which also applies the gate.
  */
 gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
@@ -214,10 +230,10 @@ gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
  * before the first kernel and events[i+1] after step i, the steps being
  *   0 pooling, 1 compressed attention, 2 S_guide block scores with the
  *   streaming top-K, 3 top-K merge, 4 attention of every token over the
- *   special tokens, 5 attention over the selected blocks, merged with step
- *   4, with the gate.
- * A step fused into another one (or absent, such as step 4 without special
- * tokens) records an empty interval.  If `n_launched` is not NULL it receives
+ *   always-kept tokens, 5 attention over the selected blocks, merged with
+ *   step 4, with the gate.
+ * A step fused into another one (or absent, such as step 4 when NK == 0)
+ * records an empty interval.  If `n_launched` is not NULL it receives
  * the number of kernels enqueued.
  */
 #define GSA_FORWARD_STEPS 6
@@ -229,8 +245,8 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
 /* Byte offsets of gsa_forward's intermediates inside its workspace (host only),
  * for inspecting them after a call: the buffers of gsa_pool_kv (qc32, kc32, vc,
  * qc, kc, ks, vs), oc, the candidates (n_split lists per row), sel, and the
- * special-token segment's fp32 output [T][H][64] and lse [T][H] (empty when
- * S == 0). */
+ * always-kept segment's fp32 output [T][H][64] and lse [T][H] (empty when
+ * NK == 0). */
 typedef struct {
   size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cand_score, cand_idx, sel, o_spec, lse_spec, total;
   int32_t n_split;

@@ -38,7 +38,12 @@ class GsaShape(ctypes.Structure):
         ("pool", c_i32),
         ("top_k", c_i32),
         ("scale", c_f32),
+        ("keep", c_i32),
     ]
+
+
+KEEP_SPECIALS = 0
+KEEP_REFERENCE = 1
 
 
 class GsaSizes(ctypes.Structure):
@@ -47,6 +52,8 @@ class GsaSizes(ctypes.Structure):
         ("Tc", ctypes.c_int64),
         ("NB", ctypes.c_int64),
         ("NS", ctypes.c_int64),
+        ("NK", ctypes.c_int64),
+        ("B0", ctypes.c_int64),
         ("L", c_i32),
         ("E", c_i32),
         ("Bh", c_i32),
@@ -62,7 +69,7 @@ class GsaWsOffsets(ctypes.Structure):
                                       "total")] + [("n_split", c_i32)]
 
 
-FORWARD_STEPS = ("pool", "compressed_attn", "block_scores", "topk_merge", "specials_attn", "selected_gate")
+FORWARD_STEPS = ("pool", "compressed_attn", "block_scores", "topk_merge", "kept_attn", "selected_gate")
 
 P_SHAPE = ctypes.POINTER(GsaShape)
 

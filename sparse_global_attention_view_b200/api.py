@@ -33,15 +33,17 @@ class Shape:
     pool: int = 4
     top_k: int = 16
     scale: float = 0.0
+    keep: int = 0  # 0: every special token always kept; 1: frame 0 + camera tokens
 
     def c(self) -> GsaShape:
         return GsaShape(self.n_frames, self.n_special, self.hp, self.wp, self.n_heads,
-                        self.head_dim, self.pool, self.top_k, float(self.scale))
+                        self.head_dim, self.pool, self.top_k, float(self.scale), self.keep)
 
     @staticmethod
     def of(workload) -> "Shape":
         return Shape(workload.n_frames, workload.n_special, workload.hp, workload.wp,
-                     workload.n_heads, workload.head_dim, workload.pool, workload.top_k)
+                     workload.n_heads, workload.head_dim, workload.pool, workload.top_k,
+                     keep=getattr(workload, "keep", 0))
 
 
 def derive(shape: Shape) -> GsaSizes:
@@ -99,7 +101,7 @@ def pool_kv(shape, q, k, v, qc32, kc32, vc, qc=None, kc=None, ks=None, vs=None, 
     z = derive(shape)
     tok = z.T * shape.n_heads * shape.head_dim
     ent = z.Tc * shape.n_heads * shape.head_dim
-    spc = z.NS * shape.n_heads * shape.head_dim
+    spc = z.NK * shape.n_heads * shape.head_dim
     check(load().gsa_pool_kv(
         ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
         _ptr(qc32, F32, ent, "qc32"), _ptr(kc32, F32, ent, "kc32"), _ptr(vc, BF16, ent, "vc"),
@@ -133,8 +135,8 @@ def topk_blocks(shape, cand_score, cand_idx, n_split, sel, ws, stream=None):
 def selected_attn(shape, q, k, v, ks, vs, sel, o_sel, lse=None, ws=None, stream=None):
     z = derive(shape)
     tok = z.T * shape.n_heads * shape.head_dim
-    spc = z.NS * shape.n_heads * shape.head_dim
-    need_sp = z.NS > 0
+    spc = z.NK * shape.n_heads * shape.head_dim
+    need_sp = z.NK > 0
     check(load().gsa_selected_attn(
         ctypes.byref(shape.c()), _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
         _ptr(ks, BF16, spc, "ks", not need_sp), _ptr(vs, BF16, spc, "vs", not need_sp),
@@ -234,11 +236,11 @@ def workspace_view(ws, shape, name: str) -> torch.Tensor:
     H, D, K = shape.n_heads, shape.head_dim, shape.top_k
     spec = {
         "qc32": (F32, (z.Tc, H, D)), "kc32": (F32, (z.Tc, H, D)), "vc": (BF16, (z.Tc, H, D)),
-        "qc": (BF16, (z.Tc, H, D)), "kc": (BF16, (z.Tc, H, D)), "ks": (BF16, (H, z.NS, D)),
-        "vs": (BF16, (H, z.NS, D)), "oc": (F32, (z.Tc, H, D)),
+        "qc": (BF16, (z.Tc, H, D)), "kc": (BF16, (z.Tc, H, D)), "ks": (BF16, (H, z.NK, D)),
+        "vs": (BF16, (H, z.NK, D)), "oc": (F32, (z.Tc, H, D)),
         "cand_score": (F32, (H, z.Tc, o.n_split, K)), "cand_idx": (I32, (H, z.Tc, o.n_split, K)),
         "sel": (I32, (H, z.Tc, K)),
-        "o_spec": (F32, (z.T if z.NS else 0, H, D)), "lse_spec": (F32, (z.T if z.NS else 0, H)),
+        "o_spec": (F32, (z.T if z.NK else 0, H, D)), "lse_spec": (F32, (z.T if z.NK else 0, H)),
     }[name]
     dtype, shp = spec
     n = 1

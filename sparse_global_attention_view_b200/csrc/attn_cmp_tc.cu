@@ -13,15 +13,18 @@
 //   warps 8-11  streaming top-K, one thread per query row.
 // S(j+1) is computed while both warpgroups work on S(j): the softmax writes
 // P(j) to its own TMEM columns, so the raw scores stay readable until the
-// top-K warpgroup has loaded them.  Each top-K thread compares its row's raw
-// scores (in registers) with the row's current K-th best: 16-column and then
-// 4-column maxima are tested with warp votes, so the warp only touches the
-// columns where some of its 32 rows have a candidate.  Candidates go to a
-// per-row buffer in shared memory; when any row's buffer is half full the warp
-// inserts all buffered candidates in lockstep (one round of insertions serves
-// every row) into the rows' heaps of K best (score, block id) pairs; special
-// entries are never ranked.  Columns arrive in ascending block order and only a
-// strictly larger score displaces the root, so equal scores keep the lower id.
+// top-K warpgroup has loaded them.  Each top-K thread reads its row's raw
+// scores 16 columns at a time (two TMEM loads in flight, so the scan loop stays
+// short in code) and compares them with the row's current K-th best: a warp
+// vote on the 16-column maximum skips the groups where none of its 32 rows has
+// a candidate.  Candidates go to a per-row buffer in shared memory; when any
+// row's buffer is half full the warp inserts all buffered candidates in
+// lockstep (one round of insertions serves every row) into the rows' heaps of
+// K best (score, block id) pairs; special entries are never ranked.  Columns
+// arrive in ascending block order and only a strictly larger score displaces
+// the root, so equal scores keep the lower id.  The softmax keeps eight
+// independent max and sum chains: one warp per sub-partition runs it, so
+// dependency latency, not throughput, is what it must avoid.
 #include <math_constants.h>
 
 #include "internal.h"
@@ -119,6 +122,22 @@ struct Heap {
   __device__ __forceinline__ int id_of(int i) const { return 0x7fffffff - (int)(uint32_t)at(i); }
   __device__ __forceinline__ float score_of(int i) const { return order_value((uint32_t)(at(i) >> 32)); }
 };
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+// Wait for this thread's TMEM loads; the registers are passed through so that
+// no use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                 "+r"(r[14]), "+r"(r[15])
+               :
+               : "memory");
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_cmp_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
@@ -278,11 +297,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      float mx = -CUDART_INF_F;
+      // eight independent max chains keep the single softmax warp of each
+      // sub-partition from stalling on one 128-long dependency chain
+      float mq[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int u = 0; u < 8; ++u) mq[u] = __uint_as_float(sv[0][u]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
+      for (int k = 8; k < 128; ++k) mq[k & 7] = fmaxf(mq[k & 7], __uint_as_float(sv[k >> 5][k & 31]));
+      const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                             fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
       const bool need = mxs > m_used + 8.f;
       if (__any_sync(0xffffffffu, need)) {
@@ -310,21 +333,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = mxs;
         }
       }
-      float sum = 0.f;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = exp2f(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
-          const float p1 = exp2f(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used));
-          sum += p0 + p1;
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used));
+          ps[i & 7] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(p_addr + 16 * c, pk);
       }
       tmem_wait_st();
-      l += sum;
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       fence_before_sync();
       mbar_arrive(bar(B_PF + b));
     }
@@ -356,9 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* cb_s = reinterpret_cast<float*>(sp + OFF_CS);
     int* cb_e = reinterpret_cast<int*>(sp + OFF_CC);
     Heap top{reinterpret_cast<unsigned long long*>(sp + OFF_HS), r, d.K, 0, -CUDART_INF_F};
-    const int E = d.E, S = d.S, Bf = d.Bf;
+    const int E = d.E, S = d.S, Bf = d.Bf, B0 = (int)d.B0;
     const int ntok = (int)n_k;
-    (void)ntok;
     int nb = 0;  // candidates waiting in this row's buffer
     // Insert the buffered candidates.  All lanes run this together, so one
     // round of insertions serves every row of the warp at once.
@@ -373,9 +395,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         int i = e - f * E;
         if (i < 0) i += E, --f;
         if (i >= E) i -= E, ++f;
-        if (i >= S) top.push(v, f * Bf + (i - S));  // special entries are never ranked
+        // special entries are never ranked, nor blocks below B0 (frame 0 when
+        // it is kept whole)
+        if (i >= S && f * Bf + (i - S) >= B0) top.push(v, f * Bf + (i - S));
       }
       nb = 0;
+    };
+    // One 16-column group of the score tile: candidates are the columns that
+    // beat the row's K-th best; the warp only scans groups where some of its
+    // rows has one.
+    auto group = [&](const uint32_t (&g)[16], int q, int e0, int lim) {
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        v[i] = (16 * q + i < lim) ? __uint_as_float(g[i]) : -CUDART_INF_F;
+      float m[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) m[u] = fmaxf(fmaxf(v[u], v[u + 4]), fmaxf(v[u + 8], v[u + 12]));
+      const float m16 = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+      if (__any_sync(0xffffffffu, m16 > top.tau)) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (v[i] > top.tau) {
+            cb_s[nb * TQ + r] = v[i];
+            cb_e[nb * TQ + r] = e0 + 16 * q + i;
+            ++nb;
+          }
+        }
+        if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush();
+      }
     };
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -385,51 +433,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       fence_after_sync();
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tbase + lane_off + b * 128 + 32 * c, sv[c]);
-      tmem_wait_ld();
-      fence_before_sync();
-      mbar_arrive(bar(B_SR + b));  // the tensor core may overwrite this buffer now
+      const uint32_t s_addr = tbase + lane_off + b * 128;
       const int e0 = j * TK;
-      if (ntok - e0 < TK) {
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (32 * c + i >= ntok - e0) sv[c][i] = __float_as_uint(-CUDART_INF_F);
-      }
-      // A column is a candidate for a row if it beats that row's K-th best.
-      // The vote keeps control flow uniform: only columns where some row of
-      // the warp has a candidate cost more than the compare and the vote.
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        float m4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float x = -CUDART_INF_F;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) x = fmaxf(x, __uint_as_float(sv[q >> 1][(q & 1) * 16 + 4 * u + i]));
-          m4[u] = x;
+      const int lim = ntok - e0;
+      uint32_t g0[16], g1[16];
+      tmem_ld16(s_addr, g0);
+#pragma unroll 1
+      for (int q = 0; q < 8; q += 2) {
+        tmem_wait_ld16(g0);
+        tmem_ld16(s_addr + 16 * (q + 1), g1);
+        group(g0, q, e0, lim);
+        tmem_wait_ld16(g1);
+        if (q + 2 < 8) {
+          tmem_ld16(s_addr + 16 * (q + 2), g0);
+        } else {
+          fence_before_sync();
+          mbar_arrive(bar(B_SR + b));  // the tensor core may overwrite this buffer now
         }
-        const float m16 = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        if (__any_sync(0xffffffffu, m16 > top.tau)) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            if (__any_sync(0xffffffffu, m4[u] > top.tau)) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const float v = __uint_as_float(sv[q >> 1][(q & 1) * 16 + 4 * u + i]);
-                if (v > top.tau) {
-                  cb_s[nb * TQ + r] = v;
-                  cb_e[nb * TQ + r] = e0 + 16 * q + 4 * u + i;
-                  ++nb;
-                }
-              }
-            }
-          }
-          if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush();
-        }
+        group(g1, q + 1, e0, lim);
       }
     }
     if (__all_sync(0xffffffffu, ok)) flush();

@@ -13,7 +13,10 @@ namespace gsa {
 struct Dims {
   int N, S, Hp, Wp, H, P, K, Keff;
   int L, E, Bh, Bw, Bf;
+  int keep;          // GSA_KEEP_SPECIALS or GSA_KEEP_REFERENCE
   long long T, Tc, NB, NS;
+  long long NK;      // always-kept tokens of the selection branch
+  long long B0;      // first top-K candidate block (Bf when frame 0 is kept whole)
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
 };
@@ -56,6 +59,17 @@ __device__ __forceinline__ long long block_slot_token(const Dims& d, long long b
   int r = br * d.P + slot / d.P, c = bc * d.P + slot % d.P;
   if (r >= d.Hp || c >= d.Wp) return -1;
   return f * d.L + d.S + (long long)r * d.Wp + c;
+}
+
+// Token id of always-kept token i (0 <= i < NK): special i (frame-major) for
+// GSA_KEEP_SPECIALS; frame 0's token i, then frame (i - L + 1)'s camera token
+// (special slot 0) for GSA_KEEP_REFERENCE.
+__host__ __device__ __forceinline__ long long kept_token(const Dims& d, long long i) {
+  if (d.keep == GSA_KEEP_SPECIALS) {
+    const long long f = i / d.S;
+    return f * d.L + (i - f * d.S);
+  }
+  return i < d.L ? i : (i - d.L + 1) * d.L;
 }
 
 // Token id held in slot `slot` of compressed entry a (a special entry holds its

@@ -23,6 +23,7 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
   if (s->n_frames < 1 || s->n_special < 0 || s->hp < 1 || s->wp < 1 || s->n_heads < 1 ||
       s->head_dim < 1 || s->pool < 1 || s->top_k < 1)
     return GSA_ERR_INVALID_ARG;
+  if (s->keep != GSA_KEEP_SPECIALS && s->keep != GSA_KEEP_REFERENCE) return GSA_ERR_INVALID_ARG;
   if (!(s->scale >= 0.f) || isinf(s->scale)) return GSA_ERR_INVALID_ARG;
   if (s->head_dim != gsa::kHeadDim || s->pool > gsa::kMaxPool || s->top_k > gsa::kMaxTopK ||
       s->n_heads > 128)
@@ -32,8 +33,11 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
   const long long Bf = Bh * Bw, E = s->n_special + Bf;
   const long long N = s->n_frames;
   const long long T = N * L, Tc = N * E, NB = N * Bf, NS = N * s->n_special;
+  const bool ref = s->keep == GSA_KEEP_REFERENCE;
+  const long long NK = ref ? L + (N - 1) * (s->n_special > 0 ? 1 : 0) : NS;
+  const long long B0 = ref ? Bf : 0;
   // token / block ids are int32 on the device, grids are at most 2^31-1 wide
-  if (L > INT32_MAX || T > INT32_MAX || NB + NS > INT32_MAX) return GSA_ERR_INVALID_ARG;
+  if (L > INT32_MAX || T > INT32_MAX || NB + NS + NK > INT32_MAX) return GSA_ERR_INVALID_ARG;
   Dims t;
   t.N = s->n_frames;
   t.S = s->n_special;
@@ -42,7 +46,10 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
   t.H = s->n_heads;
   t.P = s->pool;
   t.K = s->top_k;
-  t.Keff = (int)(NB < s->top_k ? NB : s->top_k);
+  t.Keff = (int)(NB - B0 < s->top_k ? NB - B0 : s->top_k);
+  t.keep = s->keep;
+  t.NK = NK;
+  t.B0 = B0;
   t.L = (int)L;
   t.E = (int)E;
   t.Bh = (int)Bh;
@@ -60,6 +67,8 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
     z->Tc = Tc;
     z->NB = NB;
     z->NS = NS;
+    z->NK = NK;
+    z->B0 = B0;
     z->L = t.L;
     z->E = t.E;
     z->Bh = t.Bh;
@@ -78,7 +87,8 @@ int forward_splits(const Dims& d) {
   long long ns = (2 * 148 + row_ctas - 1) / row_ctas;
   if (ns < 1) ns = 1;
   if (ns > 16) ns = 16;
-  if (ns > d.NB) ns = d.NB;
+  if (ns > d.NB - d.B0) ns = d.NB - d.B0;
+  if (ns < 1) ns = 1;
   while (ns > 1 && ns * d.K > kMaxCandidates) --ns;
   return (int)ns;
 }
@@ -92,7 +102,7 @@ Layout forward_layout(const Dims& d) {
   Layout l;
   l.n_split = forward_splits(d);
   const size_t ent = (size_t)d.Tc * d.H * gsa::kHeadDim;
-  const size_t spc = (size_t)d.NS * d.H * gsa::kHeadDim;
+  const size_t spc = (size_t)d.NK * d.H * gsa::kHeadDim;
   // the fused compressed kernel writes the selection directly: no candidate lists
   const size_t cand = gsa::compressed_tc_supported(d) ? 0 : (size_t)d.H * d.Tc * l.n_split * d.K;
   size_t o = GSA_WS_HEADER_BYTES;
@@ -112,8 +122,8 @@ Layout forward_layout(const Dims& d) {
   l.cs = take(cand * 4);
   l.ci = take(cand * 4);
   l.sel = take((size_t)d.H * d.Tc * d.K * 4);
-  // the special-token segment of the selection branch: normalised output and lse
-  const size_t tok_heads = d.NS > 0 ? (size_t)d.T * d.H : 0;
+  // the always-kept segment of the selection branch: normalised output and lse
+  const size_t tok_heads = d.NK > 0 ? (size_t)d.T * d.H : 0;
   l.ospec = take(tok_heads * gsa::kHeadDim * 4);
   l.lspec = take(tok_heads * 4);
   l.total = o;
@@ -169,7 +179,7 @@ gsa_status gsa_pool_kv(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
       !dev_ptr(vc) || !opt_ptr(qc) || !opt_ptr(kc) || !opt_ptr(ks) || !opt_ptr(vs) || !dev_ptr(ws))
     return GSA_ERR_INVALID_ARG;
   if ((ks == nullptr) != (vs == nullptr)) return GSA_ERR_INVALID_ARG;
-  if (d.NS == 0) ks = vs = nullptr;
+  if (d.NK == 0) ks = vs = nullptr;
   return cuda_status(gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32,
                                       (bf16*)vc, (bf16*)qc, (bf16*)kc, (bf16*)ks, (bf16*)vs,
                                       as_stream(stream)));
@@ -233,7 +243,7 @@ gsa_status gsa_selected_attn(const gsa_shape* shape, const gsa_bf16* q, const gs
   if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(sel) || !dev_ptr(o_sel) ||
       !opt_ptr(lse) || !dev_ptr(ws))
     return GSA_ERR_INVALID_ARG;
-  if (d.NS > 0 && (!dev_ptr(ks) || !dev_ptr(vs))) return GSA_ERR_INVALID_ARG;
+  if (d.NK > 0 && (!dev_ptr(ks) || !dev_ptr(vs))) return GSA_ERR_INVALID_ARG;
   return cuda_status(gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v,
                                           (const bf16*)ks, (const bf16*)vs, sel, nullptr, nullptr,
                                           nullptr, (bf16*)o_sel, lse, nullptr, nullptr,
@@ -345,8 +355,8 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
   bf16* vc = (bf16*)(base + l.vc);
   bf16* qc = (bf16*)(base + l.qc);
   bf16* kc = (bf16*)(base + l.kc);
-  bf16* ks = d.NS > 0 ? (bf16*)(base + l.ks) : nullptr;
-  bf16* vs = d.NS > 0 ? (bf16*)(base + l.vs) : nullptr;
+  bf16* ks = d.NK > 0 ? (bf16*)(base + l.ks) : nullptr;
+  bf16* vs = d.NK > 0 ? (bf16*)(base + l.vs) : nullptr;
   float* oc = (float*)(base + l.oc);
   float* cs = (float*)(base + l.cs);
   int* ci = (int*)(base + l.ci);
@@ -393,13 +403,13 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
   if (!fused && !step(gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s), 4)) return GSA_ERR_CUDA;
   float* ospec = nullptr;
   float* lspec = nullptr;
-  if (d.NS > 0) {
-    // the always-kept special tokens: every token attends to all N*S of them
+  if (d.NK > 0) {
+    // the always-kept tokens: every token attends to all NK of them
     ospec = (float*)(base + l.ospec);
     lspec = (float*)(base + l.lspec);
     gsa::AttnTcArgs a;
     a.n_q = d.T;
-    a.n_k = d.NS;
+    a.n_k = d.NK;
     a.H = d.H;
     a.c2 = d.scale_log2;
     a.out = ospec;
@@ -412,7 +422,7 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
     a.err = (unsigned*)ws;
     a.kv_head_major = 1;
     a.seg_len = 0;
-    if (!step(gsa::launch_attn_tc(a, (const bf16*)q, ks, vs, d.NS, s), 5)) return GSA_ERR_CUDA;
+    if (!step(gsa::launch_attn_tc(a, (const bf16*)q, ks, vs, d.NK, s), 5)) return GSA_ERR_CUDA;
   } else if (!mark(5)) {
     return GSA_ERR_CUDA;
   }

@@ -1,5 +1,6 @@
 // Step 1: P x P average pooling of the patch grid of every frame, plus the
-// special-token copies (Speed3R technical summary 2.1, compression branch).
+// head-major copies of the always-kept tokens' K / V (Speed3R technical
+// summary 2.1, compression branch; 2.2, Speed3R-VGGT).
 //
 // One CTA per patch block (or per special token), H*8 threads, each thread
 // owning 8 consecutive channels (16 bytes) of a token's [H][64] row, so every
@@ -81,7 +82,7 @@ __global__ void pool_kernel(Dims d, const bf16* __restrict__ q, const bf16* __re
     *reinterpret_cast<uint4*>(vc + o) = pack8_bf16(sv);
     if (qc) *reinterpret_cast<uint4*>(qc + o) = pack8_bf16(sq);
     if (kc) *reinterpret_cast<uint4*>(kc + o) = pack8_bf16(sk);
-  } else {
+  } else if (id < d.NB + d.NS) {
     const long long s = id - d.NB;  // special index f*S + j
     const long long f = s / d.S;
     const int j = (int)(s - f * d.S);
@@ -100,12 +101,21 @@ __global__ void pool_kernel(Dims d, const bf16* __restrict__ q, const bf16* __re
     *reinterpret_cast<uint4*>(vc + o) = uv;
     if (qc) *reinterpret_cast<uint4*>(qc + o) = uq;
     if (kc) *reinterpret_cast<uint4*>(kc + o) = uk;
-    if (ks) {
+    if (ks && d.keep == GSA_KEEP_SPECIALS) {
+      // the specials are the always-kept tokens, in this order
       const int h = tid >> 3, dd = (tid & 7) * 8;
-      const long long so = ((long long)h * d.NS + s) * kHeadDim + dd;
+      const long long so = ((long long)h * d.NK + s) * kHeadDim + dd;
       *reinterpret_cast<uint4*>(ks + so) = uk;
       *reinterpret_cast<uint4*>(vs + so) = uv;
     }
+  } else {
+    // GSA_KEEP_REFERENCE: head-major copy of always-kept token i
+    const long long i = id - d.NB - d.NS;
+    const long long off = kept_token(d, i) * row + tid * 8;
+    const int h = tid >> 3, dd = (tid & 7) * 8;
+    const long long so = ((long long)h * d.NK + i) * kHeadDim + dd;
+    *reinterpret_cast<uint4*>(ks + so) = __ldg(reinterpret_cast<const uint4*>(k + off));
+    *reinterpret_cast<uint4*>(vs + so) = __ldg(reinterpret_cast<const uint4*>(v + off));
   }
 }
 
@@ -114,7 +124,9 @@ __global__ void pool_kernel(Dims d, const bf16* __restrict__ q, const bf16* __re
 cudaError_t launch_pool(const Dims& d, const bf16* q, const bf16* k, const bf16* v, float* qc32,
                         float* kc32, bf16* vc, bf16* qc, bf16* kc, bf16* ks, bf16* vs,
                         cudaStream_t st) {
-  const long long n = d.NB + d.NS;
+  // patch blocks, specials, and (reference-frame mode, when copies are wanted)
+  // the always-kept tokens
+  const long long n = d.NB + d.NS + (ks != nullptr && d.keep == GSA_KEEP_REFERENCE ? d.NK : 0);
   if (n > 0) {
     pool_kernel<<<(unsigned)n, d.H * 8, 0, st>>>(d, q, k, v, qc32, kc32, vc, qc, kc, ks, vs);
   }

@@ -4,8 +4,9 @@
 // One warp per (compressed entry a, head h): the entry's <=16 fine tokens are
 // the 16 rows of one m16n8k16 tile.  Each warp runs a single online softmax
 // over two key segments:
-//   1. all N*S special tokens, in 64-key tiles shared by the CTA's 4 warps
-//      (cp.async double buffer from the head-major copy ks/vs);
+//   1. the NK always-kept tokens (all N*S specials, or frame 0 plus every
+//      camera token), in 64-key tiles shared by the CTA's 4 warps (cp.async
+//      double buffer from the head-major copy ks/vs);
 //   2. the entry's selected blocks, one 16-slot block per step, gathered by
 //      the warp itself (16 token rows of 128 bytes straight from K/V, a
 //      3-stage cp.async pipeline per warp; patches outside the grid are
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(SW * 32)
   };
 
   // ---- segment 1: the special tokens ----
-  const long long NS = d.NS;
+  const long long NS = d.NK;  // the always-kept tokens
   if (o_spec != nullptr) {
     // state of a softmax over the specials alone, computed by another kernel
 #pragma unroll
@@ -318,7 +319,7 @@ cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const b
                             const float* w, const float* oc, bf16* out, float* lse,
                             const float* o_spec, const float* lse_spec, unsigned* err,
                             cudaStream_t st) {
-  const bool own_specials = d.NS > 0 && o_spec == nullptr;
+  const bool own_specials = d.NK > 0 && o_spec == nullptr;
   const size_t smem = own_specials ? sizeof(SelSmem) : kSmemNoSpecials;
   cudaError_t e = cudaFuncSetAttribute(selected_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sizeof(SelSmem));

@@ -33,8 +33,9 @@ __global__ void __launch_bounds__(TK_ROWS)
   const long long a = (long long)blockIdx.x * TK_ROWS + tid;
   const bool active = a < d.Tc;
   const long long row = (long long)d.H * kHeadDim;
-  const long long per = (d.NB + n_split - 1) / n_split;
-  const long long b0 = (long long)sp * per;
+  // candidate blocks [B0, NB), cut into n_split slices
+  const long long per = (d.NB - d.B0 + n_split - 1) / n_split;
+  const long long b0 = d.B0 + (long long)sp * per;
   const long long b1 = b0 + per < d.NB ? b0 + per : d.NB;
 
   float q[64];

@@ -88,8 +88,8 @@ class Stages:
         self.vc = torch.empty((z.Tc, H, D), **b16)
         self.qc = torch.empty((z.Tc, H, D), **b16)
         self.kc = torch.empty((z.Tc, H, D), **b16)
-        self.ks = torch.empty((H, z.NS, D), **b16) if z.NS else None
-        self.vs = torch.empty((H, z.NS, D), **b16) if z.NS else None
+        self.ks = torch.empty((H, z.NK, D), **b16) if z.NK else None
+        self.vs = torch.empty((H, z.NK, D), **b16) if z.NK else None
         self.oc = torch.empty((z.Tc, H, D), **f32)
         self.n_split = n_split
         self.cs = torch.empty((H, z.Tc, n_split, shape.top_k), **f32)

@@ -76,14 +76,18 @@ def shape(**kw):
 
 @pytest.mark.parametrize("kw", [
     dict(), dict(n_special=0, hp=16, wp=16, n_heads=2, top_k=4), dict(pool=1, hp=5, wp=7),
-    dict(pool=3, hp=10, wp=11, n_special=1), dict(top_k=128, n_frames=1), dict(pool=2, hp=1, wp=9)])
+    dict(pool=3, hp=10, wp=11, n_special=1), dict(top_k=128, n_frames=1), dict(pool=2, hp=1, wp=9),
+    dict(keep=1), dict(keep=1, n_frames=1), dict(keep=1, n_special=0, top_k=128),
+    dict(keep=1, n_frames=40, top_k=128, pool=1, hp=3, wp=3)])
 def test_derive_matches_oracle_geometry(lib, kw):
     from sparse_global_attention_view_b200 import derive
     s = shape(**kw)
     z = derive(s)
-    g = O.Geometry(N=s.n_frames, S=s.n_special, Hp=s.hp, Wp=s.wp, H=s.n_heads, D=64, P=s.pool, K=s.top_k)
+    g = O.Geometry(N=s.n_frames, S=s.n_special, Hp=s.hp, Wp=s.wp, H=s.n_heads, D=64, P=s.pool, K=s.top_k,
+                   keep="reference" if s.keep == 1 else "specials")
     assert (z.T, z.Tc, z.NB, z.NS, z.L, z.E, z.Bh, z.Bw, z.Bf, z.K_eff) == \
         (g.T, g.Tc, g.NB, g.NS, g.L, g.E, g.Bh, g.Bw, g.Bf, g.K_eff)
+    assert (z.NK, z.B0) == (g.kept_tokens().size, g.B0)
 
 
 def test_workspace_size_grows_with_frames(lib):
@@ -98,6 +102,7 @@ def test_workspace_size_grows_with_frames(lib):
     (dict(head_dim=32), 2), (dict(pool=5), 2), (dict(top_k=129), 2), (dict(n_heads=129), 2),
     (dict(n_frames=0), 1), (dict(hp=0), 1), (dict(top_k=0), 1), (dict(pool=0), 1),
     (dict(n_special=-1), 1), (dict(scale=-1.0), 1), (dict(scale=float("nan")), 1),
+    (dict(keep=2), 1), (dict(keep=-1), 1),
     (dict(n_frames=2_000_000), 1)])
 def test_bad_shapes_are_rejected(lib, kw, status):
     from sparse_global_attention_view_b200 import _lib

@@ -32,6 +32,15 @@ CASES = {
     "one_frame": Workload("one_frame", 1, 5, 37, 37, 4, 64, 4, 16, 11, "gaussian"),
     # nine tokens: a single, mostly empty 128-row query tile and key tile
     "nine_tokens": Workload("nine_tokens", 1, 3, 2, 3, 2, 64, 2, 2, 12, "gaussian"),
+    # reference-frame keep (frame 0 whole + camera tokens; frame 0 not ranked)
+    "ref_small": WORKLOADS["small"].with_(name="ref_small", keep=1),
+    "ref_p3_ragged": Workload("ref_p3_ragged", 3, 2, 10, 11, 2, 64, 3, 5, 7, "gaussian", keep=1),
+    # one frame: nothing to rank (K_eff = 0), the kept set is the whole frame
+    "ref_one_frame": Workload("ref_one_frame", 1, 5, 37, 37, 4, 64, 4, 16, 11, "gaussian", keep=1),
+    # no specials: the kept set is frame 0's patches alone
+    "ref_nospecial": Workload("ref_nospecial", 3, 0, 9, 10, 2, 64, 2, 6, 13, "gaussian", keep=1),
+    # test-time K = 128 (above the fused kernel's heap): the split scorer path
+    "k128_small": WORKLOADS["small"].with_(name="k128_small", top_k=128),
 }
 
 _cache = {}
@@ -67,10 +76,13 @@ def test_pool(name):
     # bf16 round-to-nearest of the mean: within half an ulp (2^-8 relative bounds it)
     np.testing.assert_allclose(st.vc.cpu().double().numpy(), res["vc"], rtol=2.0 ** -8, atol=1e-30)
     np.testing.assert_allclose(st.qc.cpu().double().numpy(), res["qc"], rtol=2.0 ** -8, atol=1e-30)
-    if geo.NS:
-        spec = torch.as_tensor(geo.special_tokens())
-        assert torch.equal(st.ks.cpu(), x.k[spec].permute(1, 0, 2))
-        assert torch.equal(st.vs.cpu(), x.v[spec].permute(1, 0, 2))
+    kept = geo.kept_tokens()
+    if kept.size:
+        kept = torch.as_tensor(np.array(kept))
+        assert torch.equal(st.ks.cpu(), x.k[kept].permute(1, 0, 2))
+        assert torch.equal(st.vs.cpu(), x.v[kept].permute(1, 0, 2))
+    else:
+        assert st.ks is None
 
 
 @pytest.mark.parametrize("name", NAMES)
@@ -193,13 +205,25 @@ def test_dense_sampled(name):
 
 # ---- the 100, 300 and 1000-frame workloads on sampled rows -----------------
 
-BIG = {"medium": 384, "large": 256, "pages": 128}
+# 4096 sampled query rows (plus the forced edge / special rows) on each
+BIG = {"medium": 4096, "large": 4096, "pages": 4096}
+BIG_VARIANTS = {
+    # reference-frame keep, and test-time K = 128, on the 100-frame workload
+    "medium_ref": (WORKLOADS["medium"].with_(name="medium_ref", keep=1), 1024),
+    "medium_k128": (WORKLOADS["medium"].with_(name="medium_k128", top_k=128), 1024),
+}
 
 
-@pytest.mark.parametrize("name", list(BIG))
+def _big(name):
+    if name in BIG_VARIANTS:
+        return BIG_VARIANTS[name]
+    return WORKLOADS[name], BIG[name]
+
+
+@pytest.mark.parametrize("name", list(BIG) + list(BIG_VARIANTS))
 def test_big_workload_sampled(name):
     import sparse_global_attention_view_b200 as G
-    wl = WORKLOADS[name]
+    wl, n_rows = _big(name)
     x = generate(wl)
     geo = O.geometry_of(wl)
     shape = G.Shape.of(wl)
@@ -211,7 +235,7 @@ def test_big_workload_sampled(name):
     torch.cuda.synchronize()
     G.check_device_error(layer.ws)
     assert not torch.isnan(out).any()
-    rows = sample_rows(geo.T, BIG[name], seed=2, forced=PT.forced_rows(geo))
+    rows = sample_rows(geo.T, n_rows, seed=2, forced=PT.forced_rows(geo))
     res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows, sel_override=st.sel_by_entry())
     PT.assert_selection(res, name)
     idx = torch.as_tensor(rows).cuda()
@@ -223,7 +247,10 @@ def test_big_workload_sampled(name):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("name", ["medium"])
+DENSE_ROWS = {"medium": 1024, "large": 512, "pages": 128}
+
+
+@pytest.mark.parametrize("name", list(DENSE_ROWS))
 def test_big_dense_sampled(name):
     import sparse_global_attention_view_b200 as G
     wl = WORKLOADS[name]
@@ -234,6 +261,11 @@ def test_big_dense_sampled(name):
     ws = G.new_workspace(None)
     out = torch.full_like(q, float("nan"))
     G.dense_global_attn(shape, q, k, v, out, ws)
-    rows = sample_rows(geo.T, 64, seed=3, forced=PT.forced_rows(geo))
+    torch.cuda.synchronize()
+    G.check_device_error(ws)
+    assert not torch.isnan(out).any()
+    rows = sample_rows(geo.T, DENSE_ROWS[name], seed=3, forced=PT.forced_rows(geo))
     ref = O.dense_attention(geo, x.q, x.k, x.v, rows=rows)
     PT.assert_close(out[torch.as_tensor(rows).cuda()], ref, f"{name} dense sampled")
+    del q, k, v, out
+    torch.cuda.empty_cache()

@@ -4,7 +4,10 @@
 //
 // One CTA = one 128-row tile of compressed queries of one head, 12 warps:
 //   warp 0      TMA producer: the fp32 pooled query tile once, then a 2-stage
-//               ring of 128-entry key tiles (fp32 pooled K, bf16 pooled V);
+//               ring of 128-entry fp32 pooled-K tiles, each stage refilled as
+//               soon as the QK^T product that read it is complete;
+//   warp 3      TMA producer of the 2-stage ring of bf16 pooled-V tiles, each
+//               stage refilled once its PV product is complete;
 //   warp 1      MMA issuer: S = Qc Kc^T with kind::tf32 from the fp32 means
 //               (the top-K ranking needs better than bf16 scores), into one of
 //               two TMEM score buffers, then O += P Vc (bf16, P from TMEM);
@@ -13,16 +16,19 @@
 //   warps 8-11  streaming top-K, one thread per query row.
 // S(j+1) is computed while both warpgroups work on S(j): the softmax writes
 // P(j) to its own TMEM columns, so the raw scores stay readable until the
-// top-K warpgroup has loaded them.  Each top-K thread reads its row's raw
-// scores 16 columns at a time (two TMEM loads in flight, so the scan loop stays
-// short in code) and compares them with the row's current K-th best: a warp
-// vote on the 16-column maximum skips the groups where none of its 32 rows has
-// a candidate.  Candidates go to a per-row buffer in shared memory; when any
-// row's buffer is half full the warp inserts all buffered candidates in
-// lockstep (one round of insertions serves every row) into the rows' heaps of
-// K best (score, block id) pairs; special entries are never ranked.  Columns
-// arrive in ascending block order and only a strictly larger score displaces
-// the root, so equal scores keep the lower id.  The softmax keeps eight
+// top-K warpgroup is done with them.  The softmax already forms the maxima of
+// the tile's eight 16-column groups; it compares them with each row's current
+// K-th best score (published in shared memory by the top-K thread) and hands
+// the top-K warp an 8-bit mask of the groups that may hold a candidate.  The
+// top-K warp reads from TMEM only the groups flagged for any of its 32 rows
+// and releases the score buffer after its last read, so once the heaps are
+// full most tiles cost it one mask load.  Candidates (columns that beat the
+// row's K-th best) go to a per-row buffer in shared memory; when any row's
+// buffer is half full the warp inserts all buffered candidates in lockstep
+// (one round of insertions serves every row) into the rows' heaps of K best
+// (score, block id) pairs; special entries are never ranked.  Columns arrive
+// in ascending block order and only a strictly larger score displaces the
+// root, so equal scores keep the lower id.  The softmax keeps eight
 // independent max and sum chains: one warp per sub-partition runs it, so
 // dependency latency, not throughput, is what it must avoid.
 #include <math_constants.h>
@@ -50,12 +56,18 @@ constexpr uint32_t OFF_HS = OFF_V + ST * kSub;       // heap keys [kMaxK][128] (
 constexpr uint32_t OFF_CS = OFF_HS + kMaxK * TQ * 8; // candidate scores [kBuf][128]
 constexpr uint32_t OFF_CC = OFF_CS + kBuf * TQ * 4;  // candidate entry indices
 constexpr uint32_t OFF_BAR = OFF_CC + kBuf * TQ * 4;
-constexpr uint32_t OFF_MISC = OFF_BAR + 256;
+constexpr uint32_t OFF_TAU = OFF_BAR + 256;          // each row's K-th best score [128]
+constexpr uint32_t OFF_MASK = OFF_TAU + TQ * 4;      // candidate-group masks [2][128] bytes
+constexpr uint32_t OFF_MISC = OFF_MASK + 2 * TQ;
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
-constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + ST, B_KVE = B_VF + ST, B_SF = B_KVE + ST,
-              B_PF = B_SF + 2, B_SR = B_PF + 2, B_OD = B_SR + 2, B_OF = B_OD + 1, B_DRAIN = B_OF + 1,
-              B_COUNT = B_DRAIN + 1;
+// KE / VE: a K / V stage is free again (the QK^T resp. PV product that read it
+// is complete); MR: the softmax has published the candidate-group masks of
+// score buffer b.
+constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + ST, B_KE = B_VF + ST, B_VE = B_KE + ST,
+              B_SF = B_VE + ST, B_PF = B_SF + 2, B_SR = B_PF + 2, B_MR = B_SR + 2, B_OD = B_MR + 2,
+              B_OF = B_OD + 1, B_DRAIN = B_OF + 1, B_COUNT = B_DRAIN + 1;
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 constexpr uint32_t kCols = 512;
 // Register split: the block is launched with kLaunchRegs per thread; the
@@ -164,12 +176,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < ST; ++s) {
       mbar_init(bar(B_KF + s), 1);
       mbar_init(bar(B_VF + s), 1);
-      mbar_init(bar(B_KVE + s), 1);
+      mbar_init(bar(B_KE + s), 1);
+      mbar_init(bar(B_VE + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar(B_SF + b), 1);
       mbar_init(bar(B_PF + b), TQ);
-      mbar_init(bar(B_SR + b), TQ);  // top-K warpgroup has read S buffer b
+      mbar_init(bar(B_SR + b), TQ);  // top-K warpgroup is done with S buffer b
+      mbar_init(bar(B_MR + b), TQ);
     }
     mbar_init(bar(B_OD), 1);
     mbar_init(bar(B_OF), 1);
@@ -177,6 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  volatile float* tau_s = reinterpret_cast<volatile float*>(sp + OFF_TAU);
+  volatile uint8_t* mask_s = sp + OFF_MASK;
+  if (tid < TQ) tau_s[tid] = -CUDART_INF_F;
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), kCols);
     tmem_relinquish();
@@ -190,31 +207,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dec<kRegsLow>();
   }
   if (warp == 0) {
+    // TMA producer of the query tile and the K ring: a K stage is refilled as
+    // soon as the QK^T product that read it is complete
     if (lane == 0) {
       prefetch_tmap(&tq);
       prefetch_tmap(&tk);
-      prefetch_tmap(&tv);
       mbar_expect_tx(bar(B_Q), 2 * kSub);
       for (int half = 0; half < 2; ++half)
         tma_load_3d(sQ + half * kSub, &tq, bar(B_Q), 32 * half, h, (int)m0);
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
         const int s = j % ST;
-        if (j >= ST && !mbar_wait(bar(B_KVE + s), ((j / ST) - 1) & 1, abort_flag, err)) break;
+        if (j >= ST && !mbar_wait(bar(B_KE + s), ((j / ST) - 1) & 1, abort_flag, err)) break;
         mbar_expect_tx(bar(B_KF + s), 2 * kSub);
         for (int half = 0; half < 2; ++half)
           tma_load_3d(sK + (2 * s + half) * kSub, &tk, bar(B_KF + s), 32 * half, h, j * TK);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        volatile int never = 0;
+        mbar_wait(bar(B_Q), 0, &never, err);
+        for (int j = issued - 1; j >= 0 && j >= issued - ST; --j)
+          mbar_wait(bar(B_KF + j % ST), (j / ST) & 1, &never, err);
+      }
+    }
+  } else if (warp == 3) {
+    // TMA producer of the V ring: a V stage is refilled once its PV product is complete
+    if (lane == 0) {
+      prefetch_tmap(&tv);
+      int issued = 0;
+      for (int j = 0; j < nt; ++j) {
+        const int s = j % ST;
+        if (j >= ST && !mbar_wait(bar(B_VE + s), ((j / ST) - 1) & 1, abort_flag, err)) break;
         mbar_expect_tx(bar(B_VF + s), kSub);
         tma_load_3d(sV + s * kSub, &tv, bar(B_VF + s), 0, h, j * TK);
         issued = j + 1;
       }
       if (*abort_flag) {
         volatile int never = 0;
-        mbar_wait(bar(B_Q), 0, &never, err);
-        for (int j = issued - 1; j >= 0 && j >= issued - ST; --j) {
-          mbar_wait(bar(B_KF + j % ST), (j / ST) & 1, &never, err);
+        for (int j = issued - 1; j >= 0 && j >= issued - ST; --j)
           mbar_wait(bar(B_VF + j % ST), (j / ST) & 1, &never, err);
-        }
       }
     }
   } else if (warp == 1) {
@@ -228,6 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_tf32_ss(tbase + b * 128, sdesc_k(sQ + off), sdesc_k(sK + 2 * s * kSub + off), id_qk, kk > 0);
         }
         mma_commit(bar(B_SF + b));
+        mma_commit(bar(B_KE + s));
       };
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag, err) && mbar_wait(bar(B_KF), 0, abort_flag, err);
       if (ok) {
@@ -254,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16_ts(tbase + 256, tbase + 320 + b * 64 + kk * 8, sdesc_mn(sV + s * kSub + kk * 2048), id_pv,
                       (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(B_OD));
-        mma_commit(bar(B_KVE + s));
+        mma_commit(bar(B_VE + s));
       }
       if (ok) {
         mma_commit(bar(B_OF));
@@ -297,13 +330,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      // eight independent max chains keep the single softmax warp of each
-      // sub-partition from stalling on one 128-long dependency chain
+      // the maxima of the eight 16-column groups: eight independent chains keep
+      // the single softmax warp of each sub-partition from stalling on one
+      // 128-long dependency chain
       float mq[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mq[u] = __uint_as_float(sv[0][u]);
+      for (int q = 0; q < 8; ++q) mq[q] = __uint_as_float(sv[q >> 1][(q & 1) * 16]);
 #pragma unroll
-      for (int k = 8; k < 128; ++k) mq[k & 7] = fmaxf(mq[k & 7], __uint_as_float(sv[k >> 5][k & 31]));
+      for (int i = 1; i < 16; ++i)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mq[q] = fmaxf(mq[q], __uint_as_float(sv[q >> 1][(q & 1) * 16 + i]));
+      {
+        // tell the top-K warp which groups may hold a candidate for this row:
+        // those whose maximum beats the row's K-th best so far (a stale, lower
+        // threshold only flags more groups)
+        const float tau = tau_s[r];
+        uint32_t msk = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) msk |= (mq[q] > tau ? 1u : 0u) << q;
+        mask_s[b * TQ + r] = (uint8_t)msk;
+        mbar_arrive(bar(B_MR + b));
+      }
       const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
                              fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
@@ -400,6 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i >= S && f * Bf + (i - S) >= B0) top.push(v, f * Bf + (i - S));
       }
       nb = 0;
+      tau_s[r] = top.tau;
     };
     // One 16-column group of the score tile: candidates are the columns that
     // beat the row's K-th best; the warp only scans groups where some of its
@@ -428,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + b), (j >> 1) & 1, abort_flag, err))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MR + b), (j >> 1) & 1, abort_flag, err))) {
         ok = false;
         break;
       }
@@ -436,21 +484,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t s_addr = tbase + lane_off + b * 128;
       const int e0 = j * TK;
       const int lim = ntok - e0;
-      uint32_t g0[16], g1[16];
-      tmem_ld16(s_addr, g0);
-#pragma unroll 1
-      for (int q = 0; q < 8; q += 2) {
-        tmem_wait_ld16(g0);
-        tmem_ld16(s_addr + 16 * (q + 1), g1);
-        group(g0, q, e0, lim);
-        tmem_wait_ld16(g1);
-        if (q + 2 < 8) {
-          tmem_ld16(s_addr + 16 * (q + 2), g0);
-        } else {
+      // the groups flagged by the softmax for any of the warp's 32 rows
+      uint32_t G = __reduce_or_sync(0xffffffffu, (uint32_t)mask_s[b * TQ + r]);
+      bool released = false;
+      while (G != 0) {
+        const int q = __ffs(G) - 1;
+        G &= G - 1;
+        uint32_t g[16];
+        tmem_ld16(s_addr + 16 * q, g);
+        tmem_wait_ld16(g);
+        if (G == 0) {
           fence_before_sync();
           mbar_arrive(bar(B_SR + b));  // the tensor core may overwrite this buffer now
+          released = true;
         }
-        group(g1, q + 1, e0, lim);
+        group(g, q, e0, lim);
+      }
+      if (!released) {
+        fence_before_sync();
+        mbar_arrive(bar(B_SR + b));
       }
     }
     if (__all_sync(0xffffffffu, ok)) flush();

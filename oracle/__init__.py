@@ -28,5 +28,8 @@ from .gsa_oracle import (  # noqa: F401
     gsa_layer,
     dense_attention,
     frame_attention,
+    sga_sampled,
+    sga_key_tokens,
+    sga_attention,
     selection_is_valid_top_k,
 )

@@ -606,6 +606,78 @@ def frame_attention(geo: Geometry, Q, K, V, rows=None) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
+# AVGGT subsampled global attention (SGA)
+
+
+def sga_sampled(geo: Geometry, sub_h: int, sub_w: int) -> np.ndarray:
+    """Bool [Hp, Wp]: the patch positions whose keys and values SGA keeps.
+
+    "AVGGT: Rethinking Global Attention for Accelerating VGGT", section 2.2
+    (SGA): patch tokens are sampled uniformly on the 2D grid, one per
+    sub_h x sub_w window; read here as the window's first (top-left) patch.
+    """
+    keep = np.zeros((geo.Hp, geo.Wp), dtype=bool)
+    keep[::sub_h, ::sub_w] = True
+    return keep
+
+
+def sga_key_tokens(geo: Geometry, sub_h: int, sub_w: int) -> np.ndarray:
+    """Token ids of the kept keys, frame by frame: the S specials (all kept),
+    then the sampled patches row-major."""
+    grid = np.flatnonzero(sga_sampled(geo, sub_h, sub_w).ravel())
+    per = np.concatenate([np.arange(geo.S), geo.S + grid])
+    return (np.arange(geo.N)[:, None] * geo.L + per[None, :]).ravel()
+
+
+def sga_attention(geo: Geometry, Q, K, V, sub_h: int, sub_w: int, rows=None) -> np.ndarray:
+    """SGA output for fine query ``rows``: [len(rows), H, D].
+
+    AVGGT section 2.2: every query is kept; the keys/values are the special
+    tokens plus the sampled patches; each token's own key/value (the diagonal)
+    is kept as well, once; the dropped columns are replaced by a single pair
+    (mean of the dropped keys, mean of the dropped values) -- read here as one
+    more ordinary key, with no weight for how many columns it stands for.  One
+    softmax runs over [kept keys, own key if dropped, mean key].
+    """
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
+    kept = sga_key_tokens(geo, sub_h, sub_w)
+    is_kept = np.zeros(geo.T, dtype=bool)
+    is_kept[kept] = True
+    dropped = np.flatnonzero(~is_kept)
+    q = f64(Q, rows)
+    k_own, v_own = f64(K, rows), f64(V, rows)
+    k_kept, v_kept = f64(K, kept), f64(V, kept)
+    if dropped.size:
+        k_mean = np.zeros((geo.H, geo.D))
+        v_mean = np.zeros((geo.H, geo.D))
+        for t0 in range(0, dropped.size, 1 << 16):
+            part = dropped[t0:t0 + (1 << 16)]
+            k_mean += f64(K, part).sum(axis=0)
+            v_mean += f64(V, part).sum(axis=0)
+        k_mean /= dropped.size
+        v_mean /= dropped.size
+    out = np.empty((rows.size, geo.H, geo.D))
+    step = max(1, (1 << 27) // max(geo.H * (kept.size + 2), 1))
+    for r0 in range(0, rows.size, step):
+        r1 = min(rows.size, r0 + step)
+        qq = q[r0:r1]
+        s_kept = qk_logits(qq, k_kept, geo.sm_scale)                               # [r, H, NK]
+        s_own = np.sum(qq * k_own[r0:r1], axis=-1) * geo.sm_scale                  # [r, H]
+        s_own = np.where(is_kept[rows[r0:r1]][:, None], -np.inf, s_own)
+        if dropped.size:
+            s_mean = np.sum(qq * k_mean[None], axis=-1) * geo.sm_scale            # [r, H]
+        else:
+            s_mean = np.full(s_own.shape, -np.inf)
+        p = softmax(np.concatenate([s_kept, s_own[..., None], s_mean[..., None]], axis=-1))
+        o = weighted_values(p[..., :kept.size], v_kept)
+        o += p[..., kept.size, None] * v_own[r0:r1]
+        if dropped.size:
+            o += p[..., kept.size + 1, None] * v_mean[None]
+        out[r0:r1] = o
+    return out
+
+
+# ----------------------------------------------------------------------------
 # selection checks used by parity tests
 
 

@@ -156,3 +156,38 @@ def frame_bruteforce(Q, K, V, tokens_per_frame):
         out.append([_attend(Q[t][h], [K[j][h] for j in keys], [V[j][h] for j in keys], scale)
                     for h in range(H)])
     return out
+
+
+def sga_bruteforce(Q, K, V, tokens_per_frame, n_special, hp, wp, sub_h, sub_w):
+    """Subsampled global attention: keys are every special token and the patch
+    at the top-left of every sub_h x sub_w window, plus the query's own token,
+    plus one key/value pair holding the means over all other patch tokens."""
+    T = len(Q)
+    H = len(Q[0])
+    D = len(Q[0][0])
+    scale = 1.0 / math.sqrt(D)
+    keep = set()
+    for t in range(T):
+        i = t % tokens_per_frame
+        if i < n_special:
+            keep.add(t)
+        else:
+            r, c = divmod(i - n_special, wp)
+            if r % sub_h == 0 and c % sub_w == 0:
+                keep.add(t)
+    dropped = [t for t in range(T) if t not in keep]
+    out = []
+    for t in range(T):
+        row = []
+        for h in range(H):
+            keys = [K[j][h] for j in sorted(keep)]
+            vals = [V[j][h] for j in sorted(keep)]
+            if t not in keep:
+                keys.append(K[t][h])
+                vals.append(V[t][h])
+            if dropped:
+                keys.append([sum(K[j][h][d] for j in dropped) / len(dropped) for d in range(D)])
+                vals.append([sum(V[j][h][d] for j in dropped) / len(dropped) for d in range(D)])
+            row.append(_attend(Q[t][h], keys, vals, scale))
+        out.append(row)
+    return out

@@ -322,6 +322,26 @@ def pin_reference_bruteforce():
     close(res["out"], bf["out"], what="brute force out (reference keep)")
 
 
+def pin_sga():
+    """AVGGT SGA: with windows of 1 x 1 nothing is dropped (no mean pair, the
+    diagonal is already a key), so it is dense attention; on a ragged grid it
+    matches the independent brute force; and the kept key ids follow the grid."""
+    geo, x = micro(N=2, S=2, Hp=5, Wp=7, H=2, D=8)
+    close(O.sga_attention(geo, x.q, x.k, x.v, 1, 1), sdpa_dense(x.q, x.k, x.v), what="sga 1x1 = dense")
+    Q, K, V = (t.to(torch.float64).tolist() for t in (x.q, x.k, x.v))
+    for sh, sw in ((2, 3), (3, 2), (5, 7)):
+        got = O.sga_attention(geo, x.q, x.k, x.v, sh, sw)
+        want = bruteforce.sga_bruteforce(Q, K, V, geo.L, geo.S, geo.Hp, geo.Wp, sh, sw)
+        close(got, want, what=f"sga {sh}x{sw} brute force")
+    rows = np.array([0, 3, 9, geo.L + 2, geo.T - 1])
+    close(O.sga_attention(geo, x.q, x.k, x.v, 2, 3, rows=rows),
+          O.sga_attention(geo, x.q, x.k, x.v, 2, 3)[rows], what="sga row subset")
+    ids = O.sga_key_tokens(geo, 2, 3)
+    per_frame = geo.S + 3 * 3  # rows 0,2,4 x cols 0,3,6
+    assert ids.size == geo.N * per_frame
+    assert list(ids[:per_frame]) == [0, 1, 2, 5, 8, 16, 19, 22, 30, 33, 36]
+
+
 def all_pins(fixture_path):
     return {
         "block_structure": lambda: pin_block_structure(fixture_path),
@@ -340,6 +360,7 @@ def all_pins(fixture_path):
         "row_subset": pin_row_subset,
         "frame_attention": pin_frame_attention,
         "dense_key_slices": pin_dense_key_slices,
+        "sga": pin_sga,
         "reference_one_frame": pin_reference_one_frame,
         "reference_k_all": pin_reference_k_all,
         "reference_bruteforce": pin_reference_bruteforce,

@@ -120,6 +120,42 @@ def _dense_sliced_drops_last_slice(geo, Q, K, V, rows=None, key_chunk=1 << 14, m
     return O.weighted_values(O.softmax(O.qk_logits(O.f64(Q, rows), k, geo.sm_scale)), v)
 
 
+def _sga_centre_sample(geo, sub_h, sub_w):
+    keep = np.zeros((geo.Hp, geo.Wp), dtype=bool)
+    keep[sub_h // 2::sub_h, sub_w // 2::sub_w] = True
+    return keep
+
+
+def _sga_without_mean_pair(geo, Q, K, V, sub_h, sub_w, rows=None):
+    # the dropped columns simply vanish: SGA with the mean pair's logit at -inf
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
+    kept = O.sga_key_tokens(geo, sub_h, sub_w)
+    out = np.empty((rows.size, geo.H, geo.D))
+    for i, t in enumerate(rows):
+        keys = kept if t in set(kept.tolist()) else np.append(kept, t)
+        s_ = O.qk_logits(O.f64(Q, [t]), O.f64(K, keys), geo.sm_scale)
+        out[i] = O.weighted_values(O.softmax(s_), O.f64(V, keys))[0]
+    return out
+
+
+def _sga_diagonal_twice(geo, Q, K, V, sub_h, sub_w, rows=None):
+    # the own key is added even when it is already a sampled key
+    rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
+    kept = O.sga_key_tokens(geo, sub_h, sub_w)
+    is_kept = np.zeros(geo.T, dtype=bool)
+    is_kept[kept] = True
+    dropped = np.flatnonzero(~is_kept)
+    out = np.empty((rows.size, geo.H, geo.D))
+    for i, t in enumerate(rows):
+        keys = np.append(kept, t)
+        k, v = O.f64(K, keys), O.f64(V, keys)
+        if dropped.size:
+            k = np.concatenate([k, O.f64(K, dropped).mean(axis=0, keepdims=True)])
+            v = np.concatenate([v, O.f64(V, dropped).mean(axis=0, keepdims=True)])
+        out[i] = O.weighted_values(O.softmax(O.qk_logits(O.f64(Q, [t]), k, geo.sm_scale)), v)[0]
+    return out
+
+
 def _gate_wrong_sign(geo, Qc_rows, w):
     return 1.0 - _orig["gate"](geo, Qc_rows, w)
 
@@ -144,6 +180,9 @@ MUTATIONS = {
     "softmax scale 1/D": ("Geometry.sm_scale", property(lambda self: 1.0 / self.D)),
     "frame attention over the next frame": ("frame_attention", _frame_attention_next_frame),
     "sliced dense attention drops the ragged last slice": ("dense_attention", _dense_sliced_drops_last_slice),
+    "SGA samples the window centre": ("sga_sampled", _sga_centre_sample),
+    "SGA drops the mean pair": ("sga_attention", _sga_without_mean_pair),
+    "SGA lists a sampled own key twice": ("sga_attention", _sga_diagonal_twice),
     "reference keep still ranks frame 0's blocks": ("Geometry.B0", property(lambda self: 0)),
     "reference keep keeps every register token": ("Geometry.kept_tokens", _kept_all_specials_of_later_frames),
     "reference keep takes the camera from the last slot": ("Geometry.kept_tokens", _kept_camera_from_last_slot),

@@ -290,6 +290,9 @@ def main() -> None:
     ap.add_argument("--dense-steps", type=int, default=1)
     ap.add_argument("--no-frame", action="store_true", help="skip the frame attention leg")
     ap.add_argument("--frame-steps", type=int, default=5)
+    ap.add_argument("--sga-windows", default="4,8",
+                    help="AVGGT SGA legs: comma-separated window sizes s (s x s windows); empty for none")
+    ap.add_argument("--sga-steps", type=int, default=2)
     ap.add_argument("--cpu-entries", type=int, default=48, help="query blocks in the cpu_baseline sample")
     ap.add_argument("--ref-entries", type=int, default=16, help="query blocks per reference-arm step")
     args = ap.parse_args()
@@ -486,6 +489,36 @@ def main() -> None:
                  "steps": args.frame_steps}
         del fout
 
+    # ---- AVGGT subsampled global attention on the same inputs ----
+    sga = None
+    windows = [int(w_) for w_ in args.sga_windows.split(",") if w_.strip()]
+    if windows:
+        sga = {}
+        for sub in windows:
+            ws_sga = G.new_sga_workspace(shape, sub, sub)
+            sout = torch.empty_like(q)
+            G.sga_attn(shape, sub, sub, q, k, v, sout, ws_sga, stream)
+            torch.cuda.synchronize()
+            barrier()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+            for _ in range(args.sga_steps):
+                G.sga_attn(shape, sub, sub, q, k, v, sout, ws_sga, stream)
+            s1.record(stream)
+            torch.cuda.synchronize()
+            barrier()
+            G.check_device_error(ws_sga)
+            sms = max_over_ranks(s0.elapsed_time(s1) / args.sga_steps)
+            nk = z.NS + wl.n_frames * (-(-wl.hp // sub)) * (-(-wl.wp // sub))
+            tf = 4 * z.T * (nk + 2) * H * D / (sms / 1e3) / 1e12
+            sga[f"{sub}x{sub}"] = {"ms_per_layer": round(sms, 3), "tokens_per_s": job_value(world, z.T, sms),
+                                   "kept_keys": nk, "tflops": round(tf, 1),
+                                   "frac_bf16_peak": round(tf / P["bf16_tflops"], 4), "steps": args.sga_steps}
+            del ws_sga, sout
+        sga["kernels"] = ("gather of the kept keys, per-frame sums of the dropped ones, their means, "
+                          "tcgen05/TMEM attention over the kept keys, log-sum-exp merge of the own key "
+                          "and the mean pair")
+
     # ---- the CPU oracle on a bounded sample, and parity of the sampled rows ----
     cpu = None
     parity = None
@@ -520,7 +553,7 @@ def main() -> None:
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded scene model, random projections)",
         "config": workload_config(wl, l2), "roofline": roofline, "stages": stages, "cpu_baseline": cpu,
-        "e2e": e2e, "gpu_launches": launches, "clocks": clk, "dense_baseline": dense, "frame_attention": frame,
+        "e2e": e2e, "gpu_launches": launches, "clocks": clk, "dense_baseline": dense, "frame_attention": frame, "sga": sga,
         "parity": parity,
     }
     if rank == 0:

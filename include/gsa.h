@@ -206,6 +206,29 @@ gsa_status frame_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16*
                       const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream);
 
 /*
+ * Subsampled global attention ("AVGGT: Rethinking Global Attention for
+ * Accelerating VGGT", section 2.2, SGA).  Every query t attends, in one
+ * softmax (scale from `shape`), to
+ *   - every special token,
+ *   - the patch at the top-left of every sub_h x sub_w window of every frame
+ *     (rows 0, sub_h, 2 sub_h, ... and columns 0, sub_w, ... of the grid),
+ *   - its own key/value when it is not one of those (the diagonal),
+ *   - one extra key/value pair: the means of the keys and of the values of
+ *     all patch tokens not sampled (absent when none is dropped), taken as a
+ *     single ordinary key.
+ * Uses n_frames, n_special, hp, wp, n_heads, head_dim, scale of `shape`;
+ * q, k, v, out [T][H][64] bf16.  sub_h, sub_w >= 1 (1 x 1 is dense
+ * attention).  `ws` (ws_bytes >= sga_workspace_size) holds the head-major
+ * copies of the kept keys, the dropped-token means and the fp32 softmax over
+ * the kept keys; its first word is the device error word as for every call.
+ * Returns GSA_ERR_WORKSPACE when ws_bytes is too small.
+ */
+gsa_status sga_workspace_size(const gsa_shape* shape, int32_t sub_h, int32_t sub_w, size_t* bytes);
+gsa_status sga_attn(const gsa_shape* shape, int32_t sub_h, int32_t sub_w, const gsa_bf16* q,
+                    const gsa_bf16* k, const gsa_bf16* v, gsa_bf16* out, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/*
  * dense_global_attn on the warp-level tensor-core instruction (mma.sync
  * m16n8k16), the pre-tcgen05 path; kept as a measured baseline for the
  * tcgen05 kernel.  Same arguments and result.

@@ -17,6 +17,9 @@ from .api import (  # noqa: F401
     forward_noalloc,
     forward_timed,
     frame_attn,
+    sga_workspace_size,
+    new_sga_workspace,
+    sga_attn,
     gate_combine,
     new_workspace,
     pool_kv,

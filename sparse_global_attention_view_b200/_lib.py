@@ -86,6 +86,8 @@ SIGNATURES = {
     "dense_global_attn": [P_SHAPE] + [c_vp] * 6,
     "dense_global_attn_mma": [P_SHAPE] + [c_vp] * 6,
     "frame_attn": [P_SHAPE] + [c_vp] * 6,
+    "sga_workspace_size": [P_SHAPE, c_i32, c_i32, ctypes.POINTER(c_size)],
+    "sga_attn": [P_SHAPE, c_i32, c_i32] + [c_vp] * 5 + [c_size, c_vp],
     "gsa_forward": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp],
     "gsa_forward_timed": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp, ctypes.POINTER(c_i32), c_vp],
     "gsa_workspace_offsets": [P_SHAPE, ctypes.POINTER(GsaWsOffsets)],

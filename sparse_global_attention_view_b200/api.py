@@ -173,6 +173,30 @@ def frame_attn(shape, q, k, v, out, ws, stream=None):
         _ptr(out, BF16, tok, "out"), _ws(ws), _stream(stream)), "frame_attn")
 
 
+def sga_workspace_size(shape, sub_h: int, sub_w: int) -> int:
+    n = ctypes.c_size_t()
+    check(load().sga_workspace_size(ctypes.byref(shape.c()), ctypes.c_int32(sub_h), ctypes.c_int32(sub_w),
+                                    ctypes.byref(n)), "sga_workspace_size")
+    return n.value
+
+
+def new_sga_workspace(shape, sub_h: int, sub_w: int, device=None, stream=None) -> torch.Tensor:
+    """Zero-headed workspace for sga_attn."""
+    ws = torch.empty(sga_workspace_size(shape, sub_h, sub_w), dtype=torch.uint8, device=device or "cuda")
+    check(load().gsa_workspace_init(ctypes.c_void_p(ws.data_ptr()), _stream(stream)), "gsa_workspace_init")
+    return ws
+
+
+def sga_attn(shape, sub_h: int, sub_w: int, q, k, v, out, ws, stream=None):
+    """Subsampled global attention (AVGGT SGA) over sub_h x sub_w windows."""
+    z = derive(shape)
+    tok = z.T * shape.n_heads * shape.head_dim
+    check(load().sga_attn(
+        ctypes.byref(shape.c()), ctypes.c_int32(sub_h), ctypes.c_int32(sub_w),
+        _ptr(q, BF16, tok, "q"), _ptr(k, BF16, tok, "k"), _ptr(v, BF16, tok, "v"),
+        _ptr(out, BF16, tok, "out"), _ws(ws), ctypes.c_size_t(ws.numel()), _stream(stream)), "sga_attn")
+
+
 def dense_global_attn_mma(shape, q, k, v, out, ws, stream=None):
     """dense_global_attn on the warp-level mma.sync path (the measured baseline)."""
     z = derive(shape)

@@ -311,6 +311,63 @@ gsa_status frame_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16*
                                          as_stream(stream)));
 }
 
+namespace {
+
+struct SgaLayout {
+  size_t ks, vs, part, mean, o, lse, total;
+};
+
+SgaLayout sga_layout(const Dims& d, int sub_h, int sub_w) {
+  const gsa::SgaSizes z = gsa::sga_sizes(d, sub_h, sub_w);
+  const size_t row = (size_t)d.H * gsa::kHeadDim;
+  SgaLayout l;
+  size_t o = GSA_WS_HEADER_BYTES;
+  auto take = [&](size_t bytes) {
+    size_t at = o;
+    o += up256(bytes);
+    return at;
+  };
+  l.ks = take((size_t)z.NK * row * 2);
+  l.vs = take((size_t)z.NK * row * 2);
+  l.part = take((size_t)d.N * 2 * row * 4);
+  l.mean = take(2 * row * 4);
+  l.o = take((size_t)d.T * row * 4);
+  l.lse = take((size_t)d.T * d.H * 4);
+  l.total = o;
+  return l;
+}
+
+}  // namespace
+
+gsa_status sga_workspace_size(const gsa_shape* shape, int32_t sub_h, int32_t sub_w, size_t* bytes) {
+  Dims d;
+  if (bytes == nullptr || sub_h < 1 || sub_w < 1) return GSA_ERR_INVALID_ARG;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  *bytes = sga_layout(d, sub_h, sub_w).total;
+  return GSA_OK;
+}
+
+gsa_status sga_attn(const gsa_shape* shape, int32_t sub_h, int32_t sub_w, const gsa_bf16* q,
+                    const gsa_bf16* k, const gsa_bf16* v, gsa_bf16* out, void* ws, size_t ws_bytes,
+                    void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (sub_h < 1 || sub_w < 1) return GSA_ERR_INVALID_ARG;
+  if (!dev_ptr(q) || !dev_ptr(k) || !dev_ptr(v) || !dev_ptr(out) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  const SgaLayout l = sga_layout(d, sub_h, sub_w);
+  if (ws_bytes < l.total) return GSA_ERR_WORKSPACE;
+  char* base = static_cast<char*>(ws);
+  int launched = 0;
+  return cuda_status(gsa::launch_sga(d, sub_h, sub_w, (const bf16*)q, (const bf16*)k, (const bf16*)v,
+                                     (bf16*)out, (bf16*)(base + l.ks), (bf16*)(base + l.vs),
+                                     (float*)(base + l.part), (float*)(base + l.mean),
+                                     (float*)(base + l.o), (float*)(base + l.lse), (unsigned*)ws,
+                                     as_stream(stream), &launched));
+}
+
 gsa_status dense_global_attn_mma(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
                                  const gsa_bf16* v, gsa_bf16* out, void* ws, void* stream) {
   Dims d;

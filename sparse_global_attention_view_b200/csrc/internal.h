@@ -83,6 +83,17 @@ cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const b
                             const float* o_spec, const float* lse_spec, unsigned* err,
                             cudaStream_t st);
 
+// Subsampled global attention (AVGGT SGA): sizes and the five launches.
+struct SgaSizes {
+  int nh, nw;             // sampled patch rows / columns per frame
+  long long NK;           // kept keys: N * (S + nh * nw)
+  long long n_dropped;    // patch tokens whose keys are replaced by the mean pair
+};
+SgaSizes sga_sizes(const Dims& d, int sub_h, int sub_w);
+cudaError_t launch_sga(const Dims& d, int sub_h, int sub_w, const bf16* q, const bf16* k,
+                       const bf16* v, bf16* out, bf16* ks, bf16* vs, float* part, float* mean,
+                       float* o_kept, float* lse, unsigned* err, cudaStream_t st, int* launched);
+
 cudaError_t launch_gate_combine(const Dims& d, const float* qc32, const float* w, const float* oc,
                                 const bf16* o_sel, bf16* out, cudaStream_t st);
 

@@ -182,6 +182,37 @@ def test_frame_attention_sampled(name):
     assert not torch.isnan(out).any()
 
 
+SGA_CASES = [("tiny", 2, 2), ("tiny", 1, 1), ("p3_ragged", 3, 2), ("p2_onehead", 2, 3),
+             ("nine_tokens", 2, 2), ("one_frame", 4, 4), ("ref_nospecial", 3, 3), ("k_all", 9, 9)]
+
+
+@pytest.mark.parametrize("name,sh,sw", SGA_CASES)
+def test_sga_full(name, sh, sw):
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    ws = G.new_sga_workspace(shape, sh, sw)
+    out = torch.full_like(st.q, float("nan"))
+    G.sga_attn(shape, sh, sw, st.q, st.k, st.v, out, ws)
+    torch.cuda.synchronize()
+    G.check_device_error(ws)
+    ref = O.sga_attention(geo, x.q, x.k, x.v, sh, sw)
+    assert PT.zeros_fail(ref)
+    PT.assert_close(out, ref, f"{name} sga {sh}x{sw}")
+    if (sh, sw) == (1, 1):
+        PT.assert_close(out, O.dense_attention(geo, x.q, x.k, x.v), f"{name} sga 1x1 vs dense")
+
+
+def test_sga_workspace_too_small():
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case("tiny")
+    need = G.sga_workspace_size(shape, 2, 2)
+    ws = G.new_workspace(None)  # header only
+    assert ws.numel() < need
+    out = torch.empty_like(st.q)
+    with pytest.raises(G.GsaError):
+        G.sga_attn(shape, 2, 2, st.q, st.k, st.v, out, ws)
+
+
 @pytest.mark.parametrize("name", ["tiny", "p3_ragged", "nine_tokens"])
 def test_dense_warp_mma_baseline(name):
     import sparse_global_attention_view_b200 as G
@@ -268,4 +299,29 @@ def test_big_dense_sampled(name):
     ref = O.dense_attention(geo, x.q, x.k, x.v, rows=rows)
     PT.assert_close(out[torch.as_tensor(rows).cuda()], ref, f"{name} dense sampled")
     del q, k, v, out
+    torch.cuda.empty_cache()
+
+
+SGA_BIG = {"small": (4, 4, 512), "medium": (4, 4, 1024), "pages": (8, 8, 256)}
+
+
+@pytest.mark.parametrize("name", list(SGA_BIG))
+def test_big_sga_sampled(name):
+    import sparse_global_attention_view_b200 as G
+    sh, sw, n_rows = SGA_BIG[name]
+    wl = WORKLOADS[name]
+    x = generate(wl)
+    geo = O.geometry_of(wl)
+    shape = G.Shape.of(wl)
+    q, k, v, w = _dev(x)
+    ws = G.new_sga_workspace(shape, sh, sw)
+    out = torch.full_like(q, float("nan"))
+    G.sga_attn(shape, sh, sw, q, k, v, out, ws)
+    torch.cuda.synchronize()
+    G.check_device_error(ws)
+    assert not torch.isnan(out).any()
+    rows = sample_rows(geo.T, n_rows, seed=5, forced=PT.forced_rows(geo))
+    ref = O.sga_attention(geo, x.q, x.k, x.v, sh, sw, rows=rows)
+    PT.assert_close(out[torch.as_tensor(rows).cuda()], ref, f"{name} sga {sh}x{sw} sampled")
+    del q, k, v, out, ws
     torch.cuda.empty_cache()

@@ -45,7 +45,7 @@ constexpr int TQ = 128;
 constexpr int TK = 128;
 constexpr int ST = 2;
 constexpr int kThreads = 384;
-constexpr int kMaxK = 64;        // heap capacity per row
+constexpr int kMaxK = kFusedTopK;  // heap capacity per row
 constexpr int kBuf = 32;         // candidate buffer entries per row
 constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16) tile: 16 KB
 
@@ -91,6 +91,9 @@ __device__ __forceinline__ uint32_t order_bits(float s) {
 __device__ __forceinline__ float order_value(uint32_t o) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
+__device__ __forceinline__ unsigned long long pair_key(float s, int id) {
+  return ((unsigned long long)order_bits(s) << 32) | (uint32_t)(0x7fffffff - id);
+}
 struct Heap {
   unsigned long long* hk;
   int r, K, cnt;
@@ -117,9 +120,7 @@ struct Heap {
     }
     put(p, key);
   }
-  __device__ __forceinline__ void push(float s, int id) {
-    const unsigned long long key =
-        ((unsigned long long)order_bits(s) << 32) | (uint32_t)(0x7fffffff - id);
+  __device__ __forceinline__ void push(unsigned long long key) {
     if (cnt < K) {
       put(cnt, key);
       if (++cnt == K) {
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_cmp_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const Dims d, float* __restrict__ oc,
                        float* __restrict__ cand_s, int* __restrict__ cand_i, int* __restrict__ sel,
-                       unsigned* err) {
+                       unsigned* err, const CmpPass cp) {
   extern __shared__ __align__(1024) uint8_t cmp_smem_raw[];
   const uint32_t raw = smem_u32(cmp_smem_raw);
   const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 3) {
     // TMA producer of the V ring: a V stage is refilled once its PV product is complete
-    if (lane == 0) {
+    if (lane == 0 && !cp.scores_only) {
       prefetch_tmap(&tv);
       int issued = 0;
       for (int j = 0; j < nt; ++j) {
@@ -278,10 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_after_sync();
           issue_s(s1, b ^ 1);
         }
-        ok = mbar_wait(bar(B_VF + s), (j / ST) & 1, abort_flag, err) &&
+        // (the softmax's arrival on PF(b) also says it has read S(j) from buffer b)
+        ok = (cp.scores_only || mbar_wait(bar(B_VF + s), (j / ST) & 1, abort_flag, err)) &&
              mbar_wait(bar(B_PF + b), (j >> 1) & 1, abort_flag, err);
         if (!ok) break;
         fence_after_sync();
+        if (cp.scores_only) continue;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_bf16_ts(tbase + 256, tbase + 320 + b * 64 + kk * 8, sdesc_mn(sV + s * kSub + kk * 2048), id_pv,
@@ -351,6 +354,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mask_s[b * TQ + r] = (uint8_t)msk;
         mbar_arrive(bar(B_MR + b));
       }
+      if (cp.scores_only) {
+        // ranking pass: no attention; S(j) has been read
+        fence_before_sync();
+        mbar_arrive(bar(B_PF + b));
+        continue;
+      }
       const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
                              fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
@@ -398,8 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_before_sync();
       mbar_arrive(bar(B_PF + b));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF), 0, abort_flag, err));
-    if (ok) {
+    if (ok && !cp.scores_only) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF), 0, abort_flag, err));
+    if (ok && !cp.scores_only) {
       fence_after_sync();
       const long long row = m0 + r;
       const bool store = row < d.Tc;
@@ -428,6 +437,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     Heap top{reinterpret_cast<unsigned long long*>(sp + OFF_HS), r, d.K, 0, -CUDART_INF_F};
     const int E = d.E, S = d.S, Bf = d.Bf, B0 = (int)d.B0;
     const int ntok = (int)n_k;
+    const long long my_row = m0 + r;
+    // a second ranking pass keeps only pairs strictly below the first pass's
+    // K-th best (score, id) key of the row
+    const unsigned long long ub =
+        (cp.ub != nullptr && my_row < d.Tc) ? cp.ub[(long long)h * d.Tc + my_row] : ~0ull;
     int nb = 0;  // candidates waiting in this row's buffer
     // Insert the buffered candidates.  All lanes run this together, so one
     // round of insertions serves every row of the warp at once.
@@ -444,7 +458,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (i >= E) i -= E, ++f;
         // special entries are never ranked, nor blocks below B0 (frame 0 when
         // it is kept whole)
-        if (i >= S && f * Bf + (i - S) >= B0) top.push(v, f * Bf + (i - S));
+        if (i >= S && f * Bf + (i - S) >= B0) {
+          const unsigned long long key = pair_key(v, f * Bf + (i - S));
+          if (key < ub) top.push(key);
+        }
       }
       nb = 0;
       tau_s[r] = top.tau;
@@ -507,6 +524,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (__all_sync(0xffffffffu, ok)) flush();
     const long long row = m0 + r;
+    if (ok && row < d.Tc && cp.root != nullptr)
+      cp.root[(long long)h * d.Tc + row] = top.cnt == d.K ? top.at(0) : 0ull;
     if (ok && row < d.Tc) {
       const long long cb = ((long long)h * d.Tc + row) * d.K;
       if (cand_s != nullptr) {
@@ -543,7 +562,7 @@ bool compressed_tc_supported(const Dims& d) { return d.K <= kMaxK; }
 
 cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* kc32, const bf16* vc,
                                  float* oc, float* cand_score, int* cand_idx, int* sel, unsigned* err,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, const CmpPass& cp) {
   if (!compressed_tc_supported(d)) return cudaErrorInvalidValue;
   const unsigned long long H = (unsigned long long)d.H, Tc = (unsigned long long)d.Tc;
   CUtensorMap mq, mk, mv;
@@ -560,7 +579,7 @@ cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* 
   if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   dim3 grid((unsigned)((d.Tc + TQ - 1) / TQ), (unsigned)d.H);
   attn_cmp_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, d, oc, cand_score, cand_idx, sel,
-                                                         err);
+                                                         err, cp);
   return cudaGetLastError();
 }
 

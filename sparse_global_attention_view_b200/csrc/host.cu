@@ -81,8 +81,12 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
 
 constexpr int kMaxCandidates = 2048;  // n_split * K per row in the merge
 
+// K in (64, 128]: the fused kernel runs twice (top 64, then the next K - 64
+// below the first pass's 64th-best key) and the two selections are merged.
+bool two_pass(const Dims& d) { return d.K > gsa::kFusedTopK && d.K <= 2 * gsa::kFusedTopK; }
+
 int forward_splits(const Dims& d) {
-  if (gsa::compressed_tc_supported(d)) return 1;
+  if (gsa::compressed_tc_supported(d) || two_pass(d)) return 1;
   const long long row_ctas = ((d.Tc + 127) / 128) * d.H;
   long long ns = (2 * 148 + row_ctas - 1) / row_ctas;
   if (ns < 1) ns = 1;
@@ -94,7 +98,7 @@ int forward_splits(const Dims& d) {
 }
 
 struct Layout {
-  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cs, ci, sel, ospec, lspec, total;
+  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cs, ci, sel, ospec, lspec, sel_a, sel_b, root, total;
   int n_split;
 };
 
@@ -104,7 +108,8 @@ Layout forward_layout(const Dims& d) {
   const size_t ent = (size_t)d.Tc * d.H * gsa::kHeadDim;
   const size_t spc = (size_t)d.NK * d.H * gsa::kHeadDim;
   // the fused compressed kernel writes the selection directly: no candidate lists
-  const size_t cand = gsa::compressed_tc_supported(d) ? 0 : (size_t)d.H * d.Tc * l.n_split * d.K;
+  const bool fused = gsa::compressed_tc_supported(d) || two_pass(d);
+  const size_t cand = fused ? 0 : (size_t)d.H * d.Tc * l.n_split * d.K;
   size_t o = GSA_WS_HEADER_BYTES;
   auto take = [&](size_t bytes) {
     size_t at = o;
@@ -126,6 +131,11 @@ Layout forward_layout(const Dims& d) {
   const size_t tok_heads = d.NK > 0 ? (size_t)d.T * d.H : 0;
   l.ospec = take(tok_heads * gsa::kHeadDim * 4);
   l.lspec = take(tok_heads * 4);
+  // the two ranking passes of K in (64, 128]: their selections and the bound
+  const size_t rows2 = two_pass(d) ? (size_t)d.H * d.Tc : 0;
+  l.sel_a = take(rows2 * gsa::kFusedTopK * 4);
+  l.sel_b = take(rows2 * gsa::kFusedTopK * 4);
+  l.root = take(rows2 * 8);
   l.total = o;
   return l;
 }
@@ -429,10 +439,35 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
   };
   if (!mark(0)) return GSA_ERR_CUDA;
   const bool fused = gsa::compressed_tc_supported(d);
+  const bool twice = two_pass(d);
   if (!step(gsa::launch_pool(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, qc32, kc32, vc,
-                             fused ? nullptr : qc, fused ? nullptr : kc, ks, vs, s), 1))
+                             (fused || twice) ? nullptr : qc, (fused || twice) ? nullptr : kc, ks, vs, s),
+            1))
     return GSA_ERR_CUDA;
-  if (fused) {
+  if (twice) {
+    // step 2: attention + the top 64 of every row (and its 64th-best key);
+    // step 3: a ranking-only pass for the next K - 64 below that key (its
+    // heap holds K - 64);
+    // step 4: the ascending union of the two selections
+    Dims d64 = d, drest = d;
+    d64.K = gsa::kFusedTopK;
+    drest.K = d.K - gsa::kFusedTopK;
+    int* sel_a = (int*)(base + l.sel_a);
+    int* sel_b = (int*)(base + l.sel_b);
+    unsigned long long* root = (unsigned long long*)(base + l.root);
+    gsa::CmpPass first, second;
+    first.root = root;
+    second.ub = root;
+    second.scores_only = 1;
+    if (!step(gsa::launch_compressed_tc(d64, qc32, kc32, vc, oc, nullptr, nullptr, sel_a, (unsigned*)ws, s,
+                                        first),
+              2) ||
+        !step(gsa::launch_compressed_tc(drest, qc32, kc32, vc, oc, nullptr, nullptr, sel_b, (unsigned*)ws, s,
+                                        second),
+              3) ||
+        !step(gsa::launch_selection_union(d, sel_a, gsa::kFusedTopK, sel_b, drest.K, sel, s), 4))
+      return GSA_ERR_CUDA;
+  } else if (fused) {
     // steps 1-3 in one kernel (its heaps hold each row's final top-K, written
     // to sel in ascending order); the intervals of steps 2 and 3 stay empty
     if (!step(gsa::launch_compressed_tc(d, qc32, kc32, vc, oc, nullptr, nullptr, sel, (unsigned*)ws, s),
@@ -457,7 +492,8 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
     if (!step(gsa::launch_attn_mma(a, s), 2)) return GSA_ERR_CUDA;
     if (!step(gsa::launch_block_scores_topk(d, qc32, kc32, cs, ci, l.n_split, s), 3)) return GSA_ERR_CUDA;
   }
-  if (!fused && !step(gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s), 4)) return GSA_ERR_CUDA;
+  if (!fused && !twice && !step(gsa::launch_topk_merge(d, cs, ci, l.n_split, sel, s), 4))
+    return GSA_ERR_CUDA;
   float* ospec = nullptr;
   float* lspec = nullptr;
   if (d.NK > 0) {

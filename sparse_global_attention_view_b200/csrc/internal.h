@@ -62,10 +62,24 @@ bool make_tmap_3d(CUtensorMap* m, bool fp32, const void* base, unsigned long lon
 // (one candidate list per row, i.e. n_split = 1); needs K <= 64.  Writes the
 // candidate lists when cand_score/cand_idx are non-null and the final
 // selection (ascending ids, -1 padding) when sel is non-null.
+// A second launch ranks the next K pairs: with `ub` set, only (score, id)
+// keys strictly below ub[h*Tc + row] are candidates; `root` (nullable)
+// receives each row's K-th best key (0 when fewer than K candidates exist);
+// `scores_only` skips the attention (no V, P, PV or oc).
+struct CmpPass {
+  const unsigned long long* ub = nullptr;
+  unsigned long long* root = nullptr;
+  int scores_only = 0;
+};
 bool compressed_tc_supported(const Dims& d);
+constexpr int kFusedTopK = 64;  // heap capacity of one pass of the fused kernel
 cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* kc32, const bf16* vc,
                                  float* oc, float* cand_score, int* cand_idx, int* sel, unsigned* err,
-                                 cudaStream_t st);
+                                 cudaStream_t st, const CmpPass& cp = CmpPass());
+// sel[h][a][0..K) = ascending union of two ascending, -1-padded lists of
+// na and nb ids per row (the two ranking passes), -1 padded.
+cudaError_t launch_selection_union(const Dims& d, const int* sel_a, int na, const int* sel_b, int nb,
+                                   int* sel, cudaStream_t st);
 
 cudaError_t launch_block_scores_topk(const Dims& d, const float* qc32, const float* kc32,
                                      float* cand_score, int* cand_idx, int n_split,

@@ -177,7 +177,39 @@ __global__ void __launch_bounds__(MG_WARPS * 32)
   for (int i = d.Keff + lane; i < d.K; i += 32) dst[i] = -1;
 }
 
+// One thread per (head, entry): merge of two ascending lists (-1 padded).
+__global__ void selection_union_kernel(long long rows, int na, int nb, int K, const int* __restrict__ sel_a,
+                                       const int* __restrict__ sel_b, int* __restrict__ sel) {
+  const long long rid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (rid >= rows) return;
+  const int* a = sel_a + rid * na;
+  const int* b = sel_b + rid * nb;
+  int* o = sel + rid * K;
+  int i = 0, j = 0, n = 0;
+  while (n < K) {
+    const int x = i < na ? a[i] : -1;
+    const int y = j < nb ? b[j] : -1;
+    if (x < 0 && y < 0) break;
+    if (y < 0 || (x >= 0 && x < y)) {
+      o[n++] = x;
+      ++i;
+    } else {
+      o[n++] = y;
+      ++j;
+    }
+  }
+  for (; n < K; ++n) o[n] = -1;
+}
+
 }  // namespace
+
+cudaError_t launch_selection_union(const Dims& d, const int* sel_a, int na, const int* sel_b, int nb,
+                                   int* sel, cudaStream_t st) {
+  const long long rows = (long long)d.H * d.Tc;
+  selection_union_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(rows, na, nb, d.K, sel_a, sel_b,
+                                                                           sel);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_block_scores_topk(const Dims& d, const float* qc32, const float* kc32,
                                      float* cand_score, int* cand_idx, int n_split,

@@ -144,8 +144,37 @@ def test_forward(name):
     out2 = layer(st.q, st.k, st.v, st.w)
     torch.cuda.synchronize()
     G.check_device_error(layer.ws)
-    PT.assert_close(out1, res["out"], f"{name} out (forward)")
     assert torch.equal(out1, out2), "forward must be deterministic"
+    sel_fwd = G.workspace_view(layer.ws, shape, "sel").permute(1, 0, 2).contiguous().cpu().numpy()
+    if not np.array_equal(sel_fwd, st.sel_by_entry()):
+        # K > 64: gsa_forward ranks on the tensor cores in two passes, the
+        # stage call with an fp32 scorer; both are top-K up to the tie window
+        # but may differ inside it, so the oracle takes the forward's own set
+        res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, sel_override=sel_fwd)
+        PT.assert_selection(res, f"{name} forward selection")
+    PT.assert_close(out1, res["out"], f"{name} out (forward)")
+
+
+@pytest.mark.parametrize("name", ["k128_small", "k_all", "ref_small", "small"])
+def test_forward_selection(name):
+    # the selection gsa_forward itself made (for K > 64: two ranking passes of
+    # the fused kernel and their union) must be the oracle's top-K up to the
+    # tie window, and the layer output must match the oracle evaluated with it
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    layer = G.GsaLayer(shape)
+    out = torch.full_like(st.q, float("nan"))
+    layer(st.q, st.k, st.v, st.w, out)
+    torch.cuda.synchronize()
+    G.check_device_error(layer.ws)
+    sel = G.workspace_view(layer.ws, shape, "sel").permute(1, 0, 2).contiguous().cpu().numpy()
+    rows = sample_rows(geo.T, 2048, seed=6, forced=PT.forced_rows(geo))
+    ref = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows, sel_override=sel)
+    PT.assert_selection(ref, f"{name} forward selection")
+    assert (sel[:, :, geo.K_eff:] == -1).all()
+    chosen = sel[:, :, :geo.K_eff]
+    assert (np.diff(chosen, axis=-1) > 0).all(), "ids must be strictly ascending"
+    PT.assert_close(out[torch.as_tensor(rows).cuda()], ref["out"], f"{name} forward out")
 
 
 @pytest.mark.parametrize("name", ["tiny", "p3_ragged", "p1_nospecial", "k_all", "p2_onehead", "nine_tokens"])
@@ -273,6 +302,12 @@ def test_big_workload_sampled(name):
     ent = torch.as_tensor(res["entries"]).cuda()
     PT.assert_close(st.oc[ent], res["o_cmp"], f"{name} o_cmp")
     PT.assert_close(st.o_sel[idx], res["o_sel"], f"{name} o_sel")
+    sel_fwd = G.workspace_view(layer.ws, shape, "sel").permute(1, 0, 2).contiguous().cpu().numpy()
+    if not np.array_equal(sel_fwd, st.sel_by_entry()):
+        # K > 64: the forward's two tensor-core ranking passes and the stage
+        # call's fp32 scorer may pick differently inside the tie window
+        res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows, sel_override=sel_fwd)
+        PT.assert_selection(res, f"{name} forward selection")
     PT.assert_close(out[idx], res["out"], f"{name} out")
     del st, layer
     torch.cuda.empty_cache()

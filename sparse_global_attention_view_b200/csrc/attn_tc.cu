@@ -28,6 +28,30 @@ namespace {
 
 using namespace tc;
 
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^x on the FMA pipe, for a quarter of the softmax's exponentials so that the
+// special-function unit is not the only bound: Cody-Waite range reduction
+// x = j + f, j = round(x) (added to the exponent bits), f in [-1/2, 1/2], and a
+// cubic fitted to 2^f on that interval by iteratively reweighted least squares
+// on Chebyshev nodes (max relative error 7.5e-5 in fp32, below the bf16
+// rounding of P).  x is clamped at -125 (the result is then ~2^-125, i.e. 0 for
+// the softmax).
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const int j = __float_as_int(t) - 0x4B400000;
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(0.055171769f, f, 0.24261113f);
+  p = fmaf(p, f, 0.69326097f);
+  p = fmaf(p, f, 0.99992806f);
+  return __int_as_float(__float_as_int(p) + (j << 23));
+}
+
+
 constexpr int TQ = 128;            // rows per query tile
 constexpr int NQT = 2;             // query tiles per CTA
 constexpr int TK = 128;            // keys per key tile
@@ -224,11 +248,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      float mx = -CUDART_INF_F;
+      // eight independent max / sum chains: each softmax warp owns whole rows,
+      // so a single 128-long dependency chain would leave it stalled
+      float mq[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int u = 0; u < 8; ++u) mq[u] = __uint_as_float(sv[0][u]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[c][i]));
+      for (int k = 8; k < 128; ++k) mq[k & 7] = fmaxf(mq[k & 7], __uint_as_float(sv[k >> 5][k & 31]));
+      const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                             fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
       const bool need = mxs > m_used + 8.f;
       // tcgen05.ld/st are warp-collective: the warp rescales together, with
@@ -253,21 +281,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = mxs;
         }
       }
-      float sum = 0.f;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = exp2f(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
-          const float p1 = exp2f(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used));
-          sum += p0 + p1;
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
+          const float x1 = fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used);
+          const float p1 = (i & 1) ? exp2_fma(x1) : fast_exp2(x1);  // one in four on the FMA pipe
+          ps[i & 7] += p0 + p1;
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(s_addr + 16 * c, pk);
       }
       tmem_wait_st();
-      l += sum;
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       fence_before_sync();
       mbar_arrive(bar(B_PF + t));
     }

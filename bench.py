@@ -216,14 +216,14 @@ def chosen_workload(args):
     return wl
 
 
-def workload_config(wl, l2_note=None) -> dict:
+def workload_config(wl, l2_note=None, parallelism="replicas (independent scene per rank)") -> dict:
     kept = ("frame 0 + every camera token always kept" if wl.keep == 1 else "every special token always kept")
     c = {"workload": f"{wl.name}: N={wl.n_frames} frames x ({wl.n_special} special + {wl.hp}x{wl.wp} patches) "
                      f"= {wl.n_tokens} tokens, {wl.n_heads} heads x {wl.head_dim}, pool {wl.pool}x{wl.pool}, "
                      f"top-K {wl.top_k}, {kept}, {wl.kind} generator seed {wl.seed}",
          "n_frames": wl.n_frames, "tokens": wl.n_tokens, "heads": wl.n_heads, "head_dim": wl.head_dim,
          "pool": wl.pool, "top_k": wl.top_k, "keep": "reference" if wl.keep == 1 else "specials",
-         "parallelism": "replicas (independent scene per rank)"}
+         "parallelism": parallelism}
     if l2_note:
         c["l2"] = l2_note
     return c
@@ -252,9 +252,24 @@ def recorded_traffic(kernel_file: str, workload: str):
     return None
 
 
-def rank_workload(wl, rank: int):
-    """Rank r > 0 runs an independent scene of the same size (seed + 1000 r)."""
+def rank_workload(wl, rank: int, parallel: str = "replicas"):
+    """Replicas: rank r > 0 runs an independent scene of the same size (seed +
+    1000 r).  Heads: every rank holds the same scene and takes its own heads."""
+    if parallel == "heads":
+        return wl
     return wl if rank == 0 else wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def head_slice(world: int, rank: int, n_heads: int) -> tuple[int, int]:
+    """Contiguous heads [h0, h1) of rank r when the heads are split over the
+    ranks as evenly as possible (every head attends independently, so the layer
+    needs no exchange between ranks -- as after a column-parallel QKV
+    projection)."""
+    if world > n_heads:
+        raise ValueError(f"{world} ranks for {n_heads} heads")
+    base, extra = divmod(n_heads, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
 
 
 def reduce_max(value: float, dist, device) -> float:
@@ -266,9 +281,11 @@ def reduce_max(value: float, dist, device) -> float:
     return float(t.item())
 
 
-def job_value(world: int, tokens_per_rank: int, step_ms_max: float) -> float:
-    """Whole-job tokens/s: every rank's tokens over the slowest rank's step time."""
-    return world * tokens_per_rank / (step_ms_max / 1e3)
+def job_value(world: int, tokens_per_rank: int, step_ms_max: float, parallel: str = "replicas") -> float:
+    """Whole-job tokens/s over the slowest rank's step time: every rank's own
+    scene (replicas), or the one scene all ranks share by heads."""
+    tokens = tokens_per_rank if parallel == "heads" else world * tokens_per_rank
+    return tokens / (step_ms_max / 1e3)
 
 
 STAGE_SOURCE = {"pool": "pool.cu", "compressed_attn": "attn_cmp_tc.cu", "block_scores": "topk.cu",
@@ -295,6 +312,8 @@ def main() -> None:
     ap.add_argument("--sga-steps", type=int, default=2)
     ap.add_argument("--cpu-entries", type=int, default=48, help="query blocks in the cpu_baseline sample")
     ap.add_argument("--ref-entries", type=int, default=16, help="query blocks per reference-arm step")
+    ap.add_argument("--parallel", choices=["replicas", "heads"], default="replicas",
+                    help="N > 1: independent scenes per rank (weak scaling) or one scene split by heads (strong)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "gsa":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -321,8 +340,17 @@ def main() -> None:
     def max_over_ranks(v: float) -> float:
         return reduce_max(v, dist, torch.device("cuda", local))
 
-    wl = rank_workload(chosen_workload(args), rank)
+    mode = args.parallel if world > 1 else "replicas"
+    wl = rank_workload(chosen_workload(args), rank, args.parallel)
+    wl_scene = wl
     x = generate(wl)
+    parallelism = "replicas (independent scene per rank)"
+    if mode == "heads":
+        parallelism = f"heads (one scene; {wl.n_heads} heads split over {world} ranks, no exchange in the layer)"
+        h0, h1 = head_slice(world, rank, wl.n_heads)
+        x.q, x.k, x.v = (t[:, h0:h1].contiguous() for t in (x.q, x.k, x.v))
+        x.w = x.w[h0:h1].contiguous()
+        wl = wl.with_(n_heads=h1 - h0)
     shape = G.Shape.of(wl)
     z = G.derive(shape)
     H, D = shape.n_heads, shape.head_dim
@@ -376,7 +404,7 @@ def main() -> None:
     step_ms_local = (start.elapsed_time(stop) / args.steps) if flush is None else \
         statistics.mean(sum(r) for r in per_step)
     step_ms = max_over_ranks(step_ms_local)
-    value = job_value(world, z.T, step_ms)
+    value = job_value(world, z.T, step_ms, mode)
 
     # ---- per-stage roofline from the same timed steps ----
     P = peaks()
@@ -439,7 +467,7 @@ def main() -> None:
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e_steps)
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hw))
     d2h = hout.numel() * hout.element_size()
-    e2e = {"value": job_value(world, z.T, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+    e2e = {"value": job_value(world, z.T, e2e_ms, mode), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
            "path": "pinned host Q/K/V/w -> device, gsa_forward, device -> pinned host out"}
 
@@ -459,7 +487,7 @@ def main() -> None:
         barrier()
         dms = max_over_ranks(d0.elapsed_time(d1) / args.dense_steps)
         tf = dense_flops(z, H, D) / (dms / 1e3) / 1e12
-        dense = {"ms_per_layer": round(dms, 3), "tokens_per_s": job_value(world, z.T, dms),
+        dense = {"ms_per_layer": round(dms, 3), "tokens_per_s": job_value(world, z.T, dms, mode),
                  "tflops": round(tf, 1), "frac_bf16_peak": round(tf / P["bf16_tflops"], 4),
                  "gsa_speedup": round(dms / step_ms, 2), "kernel": "tcgen05/TMEM + TMA flash attention",
                  "steps": args.dense_steps}
@@ -483,7 +511,7 @@ def main() -> None:
         G.check_device_error(layer.ws)
         fms = max_over_ranks(f0.elapsed_time(f1) / args.frame_steps)
         tf = frame_flops(z, H, D) / (fms / 1e3) / 1e12
-        frame = {"ms_per_layer": round(fms, 3), "tokens_per_s": job_value(world, z.T, fms),
+        frame = {"ms_per_layer": round(fms, 3), "tokens_per_s": job_value(world, z.T, fms, mode),
                  "tflops": round(tf, 1), "frac_bf16_peak": round(tf / P["bf16_tflops"], 4),
                  "kernel": "tcgen05/TMEM + TMA flash attention, one key segment per frame",
                  "steps": args.frame_steps}
@@ -511,7 +539,7 @@ def main() -> None:
             sms = max_over_ranks(s0.elapsed_time(s1) / args.sga_steps)
             nk = z.NS + wl.n_frames * (-(-wl.hp // sub)) * (-(-wl.wp // sub))
             tf = 4 * z.T * (nk + 2) * H * D / (sms / 1e3) / 1e12
-            sga[f"{sub}x{sub}"] = {"ms_per_layer": round(sms, 3), "tokens_per_s": job_value(world, z.T, sms),
+            sga[f"{sub}x{sub}"] = {"ms_per_layer": round(sms, 3), "tokens_per_s": job_value(world, z.T, sms, mode),
                                    "kept_keys": nk, "tflops": round(tf, 1),
                                    "frac_bf16_peak": round(tf / P["bf16_tflops"], 4), "steps": args.sga_steps}
             del ws_sga, sout
@@ -550,9 +578,10 @@ def main() -> None:
           "L2 flushed between steps (256 MB write, outside the per-kernel events)")
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "strong" if mode == "heads" else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded scene model, random projections)",
-        "config": workload_config(wl, l2), "roofline": roofline, "stages": stages, "cpu_baseline": cpu,
+        "config": workload_config(wl_scene, l2, parallelism), "roofline": roofline, "stages": stages, "cpu_baseline": cpu,
         "e2e": e2e, "gpu_launches": launches, "clocks": clk, "dense_baseline": dense, "frame_attention": frame, "sga": sga,
         "parity": parity,
     }

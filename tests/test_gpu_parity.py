@@ -39,8 +39,12 @@ CASES = {
     "ref_one_frame": Workload("ref_one_frame", 1, 5, 37, 37, 4, 64, 4, 16, 11, "gaussian", keep=1),
     # no specials: the kept set is frame 0's patches alone
     "ref_nospecial": Workload("ref_nospecial", 3, 0, 9, 10, 2, 64, 2, 6, 13, "gaussian", keep=1),
-    # test-time K = 128 (above the fused kernel's heap): the split scorer path
+    # test-time K = 128 (above the fused kernel's heap): two ranking passes in
+    # gsa_forward, the split scorer in the stage calls
     "k128_small": WORKLOADS["small"].with_(name="k128_small", top_k=128),
+    # an uneven second pass (64 + 36) and the reference keep with K = 128
+    "k100_small": WORKLOADS["small"].with_(name="k100_small", top_k=100),
+    "ref_k128": Workload("ref_k128", 4, 5, 37, 37, 2, 64, 4, 128, 14, "gaussian", keep=1),
 }
 
 _cache = {}
@@ -155,7 +159,7 @@ def test_forward(name):
     PT.assert_close(out1, res["out"], f"{name} out (forward)")
 
 
-@pytest.mark.parametrize("name", ["k128_small", "k_all", "ref_small", "small"])
+@pytest.mark.parametrize("name", ["k128_small", "k100_small", "ref_k128", "k_all", "ref_small", "small"])
 def test_forward_selection(name):
     # the selection gsa_forward itself made (for K > 64: two ranking passes of
     # the fused kernel and their union) must be the oracle's top-K up to the
@@ -360,3 +364,19 @@ def test_big_sga_sampled(name):
     PT.assert_close(out[torch.as_tensor(rows).cuda()], ref, f"{name} sga {sh}x{sw} sampled")
     del q, k, v, out, ws
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name,h0,h1", [("small", 4, 9), ("ref_small", 0, 8), ("k128_small", 11, 16)])
+def test_head_slice_matches_full_layer(name, h0, h1):
+    # head-parallel ranks run gsa_forward on their own heads only: heads are
+    # independent in every step, so a slice of heads gives exactly those
+    # heads of the full layer
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    full = G.GsaLayer(shape)(st.q, st.k, st.v, st.w)
+    wl = CASES[name].with_(n_heads=h1 - h0)
+    part_shape = G.Shape.of(wl)
+    sl = lambda t: t[:, h0:h1].contiguous()  # noqa: E731
+    part = G.GsaLayer(part_shape)(sl(st.q), sl(st.k), sl(st.v), st.w[h0:h1].contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(part, full[:, h0:h1]), "a head slice must reproduce those heads bit for bit"

@@ -20,9 +20,9 @@ step by step in the order the Speed3R pages give the method:
        key/value regions;
     4. gated aggregation -- a learnable sigmoid gate computed from the query
        mixes the two branch outputs;
-  plus the Speed3R-VGGT adaptation ("the selection branch always keeps the
-  reference-frame / camera-token information", section 2.2) and the dense
-  global attention the module replaces (section 1, "Background").
+  plus the Speed3R-VGGT adaptation (section 2.2: the selection branch is made
+  to retain the reference frame and the camera tokens at all times) and the
+  dense global attention the module replaces (section 1, background).
 
 Where the pages are silent, the readings used here are:
   * queries, keys and values are all pooled in the compression branch; the

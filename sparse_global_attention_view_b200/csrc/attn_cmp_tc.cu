@@ -26,7 +26,10 @@
 // row's K-th best) go to a per-row buffer in shared memory; when any row's
 // buffer is half full the warp inserts all buffered candidates in lockstep
 // (one round of insertions serves every row) into the rows' heaps of K best
-// (score, block id) pairs; special entries are never ranked.  Columns arrive
+// (score, block id) pairs; special entries are never ranked.  Once every heap
+// of the warp is full, a round is one predicated three-level replacement of
+// the root per lane (lanes without a candidate walk it without moving), with
+// the next round's candidate loaded during the current one: no lane diverges.  Columns arrive
 // in ascending block order and only a strictly larger score displaces the
 // root, so equal scores keep the lower id.  The softmax keeps eight
 // independent max and sum chains: one warp per sub-partition runs it, so
@@ -120,6 +123,38 @@ struct Heap {
     }
     put(p, key);
   }
+  // Replace the root (the worst pair) of a full heap by `key` and restore the
+  // heap order: a fixed three levels (K <= 64 pairs fit in 1 + 4 + 16 + 64
+  // slots), the four children of a level loaded together and the descent
+  // predicated rather than branched, so every lane of the warp takes the same
+  // path; the new root is tracked in a register.
+  __device__ __forceinline__ void replace_root(unsigned long long key, bool take = true) {
+    if (!take) key = 0ull;  // a lane without a candidate walks the levels without moving
+    int p = 0;
+    bool go = take;
+    unsigned long long root = key;
+#pragma unroll
+    for (int lvl = 0; lvl < 3; ++lvl) {
+      const int c0 = 4 * p + 1;
+      unsigned long long x[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) x[t] = (go && c0 + t < K) ? at(c0 + t) : ~0ull;
+      unsigned long long m = x[0];
+      int mc = c0;
+#pragma unroll
+      for (int t = 1; t < 4; ++t)
+        if (x[t] < m) m = x[t], mc = c0 + t;
+      const bool move = go && m < key;
+      if (move) put(p, m);
+      if (lvl == 0 && move) root = m;
+      p = move ? mc : p;
+      go = move;
+    }
+    if (take) {
+      put(p, key);
+      tau = order_value((uint32_t)(root >> 32));
+    }
+  }
   __device__ __forceinline__ void push(unsigned long long key) {
     if (cnt < K) {
       put(cnt, key);
@@ -129,8 +164,7 @@ struct Heap {
       }
       return;
     }
-    sift(0, key);
-    tau = order_value((uint32_t)(at(0) >> 32));
+    replace_root(key);
   }
   __device__ __forceinline__ int id_of(int i) const { return 0x7fffffff - (int)(uint32_t)at(i); }
   __device__ __forceinline__ float score_of(int i) const { return order_value((uint32_t)(at(i) >> 32)); }
@@ -447,6 +481,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     // round of insertions serves every row of the warp at once.
     const float inv_e = 1.f / (float)E;
     auto flush = [&]() {
+      if (__all_sync(0xffffffffu, top.cnt == d.K)) {
+        // every heap of the warp is full: one predicated replacement per round
+        const int rounds = (int)__reduce_max_sync(0xffffffffu, (unsigned)nb);
+        float v_next = nb > 0 ? cb_s[r] : -CUDART_INF_F;
+        int e_next = nb > 0 ? cb_e[r] : 0;
+        for (int n = 0; n < rounds; ++n) {
+          const bool have = n < nb;
+          const float v = v_next;
+          const int e = e_next;
+          // the next round's candidate is read while this one is inserted
+          v_next = n + 1 < nb ? cb_s[(n + 1) * TQ + r] : -CUDART_INF_F;
+          e_next = n + 1 < nb ? cb_e[(n + 1) * TQ + r] : 0;
+          int f = (int)((float)e * inv_e);
+          int i = e - f * E;
+          if (i < 0) i += E, --f;
+          if (i >= E) i -= E, ++f;
+          const int id = f * Bf + (i - S);
+          const unsigned long long key = pair_key(v, id);
+          const bool take = have && v > top.tau && i >= S && id >= B0 && key < ub;
+          top.replace_root(key, take);
+        }
+        nb = 0;
+        tau_s[r] = top.tau;
+        return;
+      }
       for (int n = 0; n < nb; ++n) {
         const float v = cb_s[n * TQ + r];
         if (!(v > top.tau)) continue;

@@ -143,7 +143,11 @@ gsa_status gsa_pool_kv(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
  *   S_guide[h][a][beta] = scale * (qc32[a,h] . kc32[entry(beta),h]) of that
  *   slice with their block ids, unordered, padded with (-inf, -1).
  * qc / kc are the bf16 pooled tensors of gsa_pool_kv, qc32 / kc32 the fp32 ones.
- * n_split in [1, 64].
+ * n_split in [1, 64], n_split * K <= 2048.  With n_split == 1 and K <= 64 this
+ * runs the fused tcgen05 kernel (scores from tf32 products of qc32 / kc32,
+ * the list of each row being its exact top-K); otherwise warp-level bf16
+ * attention from qc / kc and an fp32 scorer over the slices.  Blocks below
+ * B0 are never candidates.
  */
 gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const gsa_bf16* kc,
                                const gsa_bf16* vc, const float* qc32, const float* kc32,
@@ -238,7 +242,8 @@ gsa_status dense_global_attn_mma(const gsa_shape* shape, const gsa_bf16* q, cons
 
 /*
  * The whole GSA layer: steps 1-6 enqueued on `stream`, intermediates in `ws`
- * (ws_bytes >= gsa_workspace_size).  w [H][64] fp32 gate vectors; out
+ * (ws_bytes >= gsa_workspace_size); K up to 128 (see gsa_forward_timed for
+ * how K > 64 is ranked).  w [H][64] fp32 gate vectors; out
  * [T][H][64] bf16.  The attention over the always-kept tokens runs on the
  * tensor-core attention kernel into the workspace; the selected blocks
  * continue that softmax in the step-5 kernel, which also applies the gate.
@@ -255,6 +260,12 @@ gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
  *   streaming top-K, 3 top-K merge, 4 attention of every token over the
  *   always-kept tokens, 5 attention over the selected blocks, merged with
  *   step 4, with the gate.
+ * For K <= 64 steps 1-3 are one fused kernel (step 1's interval holds it).
+ * For 64 < K <= 128 step 1 is the fused kernel ranking the top 64 (and
+ * recording each row's 64th-best (score, id) key), step 2 a second,
+ * ranking-only pass of it for the next K - 64 pairs strictly below that key,
+ * and step 3 the ascending union of the two selections (Speed3R technical
+ * summary 4: a larger Top-K at test time).
  * A step fused into another one (or absent, such as step 4 when NK == 0)
  * records an empty interval.  If `n_launched` is not NULL it receives
  * the number of kernels enqueued.

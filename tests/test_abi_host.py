@@ -134,6 +134,35 @@ def test_null_and_misaligned_pointers_are_rejected(lib):
     assert lib.gsa_check_device_error(null, st) == 1
     assert lib.gsa_workspace_init(bad, st) == 1
     assert lib.gsa_derive(None, None) == 1
+    assert lib.frame_attn(ctypes.byref(s), p, p, bad, p, p, st) == 1
+    assert lib.sga_attn(ctypes.byref(s), 2, 2, p, p, p, null, p, ctypes.c_size_t(1 << 40), st) == 1
+    assert lib.sga_attn(ctypes.byref(s), 0, 2, p, p, p, p, p, ctypes.c_size_t(1 << 40), st) == 1
+    assert lib.sga_attn(ctypes.byref(s), 2, -1, p, p, p, p, p, ctypes.c_size_t(1 << 40), st) == 1
+
+
+def test_sga_workspace_size(lib):
+    from sparse_global_attention_view_b200 import derive
+    s = shape()
+    n2, n4 = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.sga_workspace_size(ctypes.byref(s.c()), 2, 2, ctypes.byref(n2)) == 0
+    assert lib.sga_workspace_size(ctypes.byref(s.c()), 4, 4, ctypes.byref(n4)) == 0
+    assert n2.value > n4.value > 256 and n2.value % 256 == 0
+    # the fp32 output over the kept keys dominates: T x H x 64 x 4 bytes at least
+    z = derive(s)
+    assert n4.value >= z.T * s.n_heads * 64 * 4
+    assert lib.sga_workspace_size(ctypes.byref(s.c()), 0, 4, ctypes.byref(n4)) == 1
+    assert lib.sga_workspace_size(ctypes.byref(s.c()), 4, 4, None) == 1
+    p = ctypes.c_void_p(FAKE)
+    assert lib.sga_attn(ctypes.byref(s.c()), 4, 4, p, p, p, p, p, ctypes.c_size_t(n4.value - 1),
+                        ctypes.c_void_p(0)) == 3
+
+
+def test_two_pass_workspace_is_larger(lib):
+    # K in (64, 128] keeps two 64-wide selections and a 64-bit bound per row
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    assert lib.gsa_workspace_size(ctypes.byref(shape(top_k=64).c()), ctypes.byref(a)) == 0
+    assert lib.gsa_workspace_size(ctypes.byref(shape(top_k=65).c()), ctypes.byref(b)) == 0
+    assert b.value > a.value
 
 
 def test_small_workspace_is_rejected(lib):

@@ -39,3 +39,19 @@ def test_ranking_and_validity_against_plain_python(keep):
         for r in range(4):
             for h in range(2):
                 assert got[r, h] == _plain_valid(geo, g[r, h], other[r, h], 0.05)
+
+
+@pytest.mark.parametrize("keep", ["specials", "reference"])
+def test_gap_against_plain_sort(keep):
+    # the K-th minus the (K+1)-th largest candidate score, inf when every
+    # candidate is selected; the parity tests' tie window is read from it
+    rng = np.random.default_rng(2)
+    for K in (1, 5, 20, 32):
+        geo = O.Geometry(N=3, S=1, Hp=8, Wp=8, H=2, D=8, P=4, K=K, keep=keep)
+        g = np.round(rng.normal(size=(3, 2, geo.NB)), 2)
+        gap = O.top_k_gap(geo, g)
+        for r in range(3):
+            for h in range(2):
+                cand = sorted(g[r, h, geo.B0:], reverse=True)
+                want = np.inf if geo.K_eff >= len(cand) else cand[geo.K_eff - 1] - cand[geo.K_eff]
+                assert gap[r, h] == want

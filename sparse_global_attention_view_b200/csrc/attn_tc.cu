@@ -1,7 +1,9 @@
 // Exact attention on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
-// Used for the dense global attention (Speed3R technical summary 1) and for
-// the always-kept special-token segment of the selection branch (2.1, 2.2).
+// Used for the dense global attention (Speed3R technical summary 1), the
+// always-kept segment of the selection branch (2.1, 2.2), frame attention
+// (keys restricted to the query's own frame: per-frame key segments; AVGGT
+// 2.2) and the kept keys of subsampled global attention (AVGGT 2.2).
 //
 // One CTA = two 128-row query tiles of one head (TMEM lanes = rows) and 12 warps:
 //   warp 0      TMA producer: Q tiles once, then a 4-stage ring of 128-key K/V
@@ -11,7 +13,8 @@
 //   warp 2      TMEM allocation (512 columns: S_0, S_1, O_0, O_1);
 //   warps 4-11  softmax, one warpgroup per query tile, one thread per row.
 // The MMA thread interleaves the two tiles so one tile's softmax overlaps the
-// other tile's matrix products.  The softmax keeps a stale maximum until a
+// other tile's matrix products.  The softmax keeps eight independent max and
+// sum chains and takes a quarter of its exponentials on the FMA pipe.  The softmax keeps a stale maximum until a
 // tile's maximum exceeds it by 2^8 and only then rescales O (in TMEM), so the
 // common case never waits for the tensor core.  Every mbarrier wait is
 // bounded: on timeout the CTA records kErrTimeout, raises its abort flag, drains

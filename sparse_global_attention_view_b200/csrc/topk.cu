@@ -1,6 +1,7 @@
-// Steps 3-4: S_guide block scores with a streaming Top-K, and the merge of the
-// per-slice candidate lists into the selection (Speed3R technical summary 2.1,
-// selection branch; S_guide on the it page, section 2).
+// Steps 3-4 of the stage calls: S_guide block scores with a streaming Top-K,
+// and the merge of the per-slice candidate lists into the selection (Speed3R
+// technical summary 2.1, selection branch; S_guide on the it page, section 2);
+// and the union of the two ranking passes gsa_forward runs for 64 < K <= 128.
 //
 // Block scores are fp32 dot products of the fp32 pooled query and key means,
 // times the softmax scale.  Each thread owns one compressed query row and

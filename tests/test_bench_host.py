@@ -1,0 +1,54 @@
+"""Host-side helpers of bench.py (no GPU): the head split, the job value of
+both multi-GPU modes, the workload overrides and the per-stage algorithmic work."""
+
+import types
+
+import pytest
+
+import bench
+from synthetic import WORKLOADS
+
+
+@pytest.mark.parametrize("world,heads", [(1, 16), (2, 16), (3, 16), (8, 16), (5, 7), (7, 7)])
+def test_head_slices_partition_the_heads(world, heads):
+    got = [bench.head_slice(world, r, heads) for r in range(world)]
+    assert got[0][0] == 0 and got[-1][1] == heads
+    for (a0, a1), (b0, b1) in zip(got, got[1:]):
+        assert a1 == b0
+    sizes = [h1 - h0 for h0, h1 in got]
+    assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 1
+
+
+def test_more_ranks_than_heads_is_refused():
+    with pytest.raises(ValueError):
+        bench.head_slice(3, 0, 2)
+
+
+def test_job_value_modes():
+    assert bench.job_value(4, 1000, 500.0) == pytest.approx(4 * 1000 / 0.5)
+    assert bench.job_value(4, 1000, 500.0, "heads") == pytest.approx(1000 / 0.5)
+
+
+def test_rank_workloads():
+    wl = WORKLOADS["medium"]
+    assert bench.rank_workload(wl, 0) == wl
+    assert bench.rank_workload(wl, 2).seed == wl.seed + 2000
+    assert bench.rank_workload(wl, 2, "heads") == wl
+
+
+def test_workload_overrides():
+    args = types.SimpleNamespace(workload="pages", top_k=128, keep=1)
+    wl = bench.chosen_workload(args)
+    assert (wl.top_k, wl.keep, wl.n_frames) == (128, 1, 1000)
+    cfg = bench.workload_config(wl)
+    assert cfg["keep"] == "reference" and cfg["top_k"] == 128 and "frame 0" in cfg["workload"]
+
+
+def test_stage_work_at_the_pages_workload():
+    z = types.SimpleNamespace(T=1_374_000, Tc=105_000, NB=100_000, NS=5000, NK=5000, B0=0)
+    work = bench.stage_work(z, 16, 64, 64)
+    assert work["compressed_attn"] == ("tensor", 4 * 105_000 ** 2 * 16 * 64, "flop")
+    assert work["kept_attn"] == ("tensor", 4 * 1_374_000 * 5000 * 16 * 64, "flop")
+    assert work["selected_gate"][1] == 16 * 105_000 * 64 * 16 * 64 * 2 * 2
+    # Q, K, V read once: 3 x 1,374,000 x 16 x 64 x 2 bytes, plus the pooled and kept writes
+    assert work["pool"][1] > 3 * 1_374_000 * 16 * 64 * 2

@@ -55,3 +55,30 @@ def test_gap_against_plain_sort(keep):
                 cand = sorted(g[r, h, geo.B0:], reverse=True)
                 want = np.inf if geo.K_eff >= len(cand) else cand[geo.K_eff - 1] - cand[geo.K_eff]
                 assert gap[r, h] == want
+
+
+def _two_pass(geo, g_row, first):
+    # the first pass keeps the `first` best (score, lower id) pairs and records
+    # the worst of them; the second keeps the next K - first pairs strictly below
+    # that pair in the same order; the selection is their union
+    order = sorted(range(geo.B0, geo.NB), key=lambda b: (-g_row[b], b))
+    top = order[:first]
+    if len(top) < first:
+        return sorted(top)
+    bound = (-g_row[top[-1]], top[-1])
+    rest = [b for b in order if (-g_row[b], b) > bound][:geo.K_eff - first]
+    return sorted(top + rest)
+
+
+@pytest.mark.parametrize("K", [65, 100, 128])
+def test_two_ranking_passes_equal_the_top_k(K):
+    # the reading behind gsa_forward's K > 64 path: ranking the first 64 and then
+    # the next K - 64 strictly below the 64th pair is exactly the top-K, ties to
+    # the lower id included
+    rng = np.random.default_rng(3)
+    for keep in ("specials", "reference"):
+        geo = O.Geometry(N=4, S=1, Hp=20, Wp=20, H=1, D=8, P=4, K=K, keep=keep)
+        g = np.round(rng.normal(size=(6, 1, geo.NB)), 1)  # many ties
+        own = O.top_k_blocks(geo, g)
+        for r in range(6):
+            assert _two_pass(geo, g[r, 0], 64) == [b for b in own[r, 0] if b >= 0]

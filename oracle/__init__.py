@@ -7,12 +7,17 @@ product path (the CUDA library and its Python binding) never imports it.
 Parity status of every function here: pinned by the CPU tests in
 ``tests/test_oracle_pins.py`` (closed forms, library routines, brute force,
 invariants) and ``tests/test_oracle_mutations.py`` (planted mistakes that the
-pins must catch).  No function is unpinned.
+pins must catch).  The chunked and threaded forms the oracle takes at full
+size (``Chunking``) are pinned too, by forcing them on small inputs
+(``chunking``).  No function is unpinned.
 """
 
 from .gsa_oracle import (  # noqa: F401
+    Chunking,
     Geometry,
+    chunking,
     geometry_of,
+    spans,
     f64,
     softmax,
     pool,

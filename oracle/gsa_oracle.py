@@ -53,12 +53,68 @@ full-size workloads never need a float64 copy of the whole tensor.
 
 from __future__ import annotations
 
+import contextlib
 import dataclasses
 import functools
 import math
 
 import numpy as np
 import torch
+
+
+# ----------------------------------------------------------------------------
+# sizes at which the same arithmetic switches to a chunked or threaded form
+
+
+@dataclasses.dataclass(frozen=True)
+class Chunking:
+    """Where the oracle splits work to bound host memory or to use every core.
+
+    None of these changes what is computed, only in which pieces: each form
+    is pinned against the unsplit one and against a library routine or the
+    brute force by forcing tiny values (``chunking``).
+
+    softmax_torch_elems  arrays of at least this many elements go through
+                         float64 torch ops (multi-threaded) instead of NumPy
+    pool_frames          frames pooled per slice of the input
+    layer_chunk_elems    compressed logits [entries, H, Tc] formed at once
+    dense_key_chunk      longer sequences take dense attention's two-pass
+                         form over key slices of this many tokens
+    dense_max_bytes      bytes of logits of one key slice (row chunking)
+    sga_mean_tokens      dropped tokens summed per slice for SGA's mean pair
+    sga_row_elems        logits [rows, H, keys] SGA forms at once
+    """
+
+    softmax_torch_elems: int = 1 << 20
+    pool_frames: int = 32
+    layer_chunk_elems: int = 50_000_000
+    dense_key_chunk: int = 1 << 14
+    dense_max_bytes: int = 1 << 30
+    sga_mean_tokens: int = 1 << 16
+    sga_row_elems: int = 1 << 27
+
+
+CHUNKS = Chunking()
+
+
+def spans(n: int, step: int) -> list[tuple[int, int]]:
+    """(start, stop) of the consecutive slices of range(n), ``step`` long; the
+    last one may be shorter."""
+    step = max(1, int(step))
+    return [(i, min(n, i + step)) for i in range(0, n, step)]
+
+
+@contextlib.contextmanager
+def chunking(**sizes):
+    """Temporarily use other split sizes (tests force every split form with
+    tiny values)."""
+    global CHUNKS
+    old = CHUNKS
+    CHUNKS = dataclasses.replace(old, **sizes)
+    try:
+        yield CHUNKS
+    finally:
+        CHUNKS = old
 
 
 # ----------------------------------------------------------------------------
@@ -254,11 +310,11 @@ def f64_head(x, rows, h: int) -> np.ndarray:
 
 def softmax(z: np.ndarray, axis: int = -1) -> np.ndarray:
     """Textbook softmax, shifted by the maximum for range (exact in real
-    arithmetic).  Large arrays go through float64 torch CPU ops, which use
-    every core; small ones stay in NumPy (a torch call costs more than the
-    arithmetic there)."""
+    arithmetic).  Arrays of ``CHUNKS.softmax_torch_elems`` elements or more go
+    through float64 torch CPU ops, which use every core; smaller ones stay in
+    NumPy (a torch call costs more than the arithmetic there)."""
     z = np.asarray(z, dtype=np.float64)
-    if z.size < (1 << 20):
+    if z.size < CHUNKS.softmax_torch_elems:
         m = np.max(z, axis=axis, keepdims=True)
         e = np.exp(z - m)
         return e / np.sum(e, axis=axis, keepdims=True)
@@ -272,18 +328,20 @@ def softmax(z: np.ndarray, axis: int = -1) -> np.ndarray:
 # step 1: compression by spatial average pooling
 
 
-def pool(geo: Geometry, X, frames_per_chunk: int = 32) -> np.ndarray:
+def pool(geo: Geometry, X, frames_per_chunk: int | None = None) -> np.ndarray:
     """Compressed sequence of X: [Tc, H, D] float64.
 
     Speed3R, technical summary 2.1, compression branch: the tokens are
     down-sampled spatially, e.g. by 4x4 average pooling, into a coarse
     context.  Each patch block's entry is the arithmetic mean over the
     patches the block actually holds (fewer than P*P at the right/bottom
-    edges); each special token is copied as its own entry.
+    edges); each special token is copied as its own entry.  The input is
+    read ``frames_per_chunk`` frames at a time (``CHUNKS.pool_frames``).
     """
-    out = np.empty((geo.Tc, geo.H, geo.D), dtype=np.float64)
-    for f0 in range(0, geo.N, frames_per_chunk):
-        f1 = min(geo.N, f0 + frames_per_chunk)
+    if frames_per_chunk is None:
+        frames_per_chunk = CHUNKS.pool_frames
+    out = np.full((geo.Tc, geo.H, geo.D), np.nan)  # NaN marks anything left unwritten
+    for f0, f1 in spans(geo.N, frames_per_chunk):
         x = f64(X, slice(f0 * geo.L, f1 * geo.L)).reshape(f1 - f0, geo.L, geo.H, geo.D)
         spec = x[:, :geo.S]
         grid = x[:, geo.S:].reshape(f1 - f0, geo.Hp, geo.Wp, geo.H, geo.D)
@@ -424,7 +482,7 @@ def selected_attention(geo: Geometry, Q, K, V, sel: np.ndarray, rows: np.ndarray
     """
     pos = {int(a): i for i, a in enumerate(entries)}
     rows = np.asarray(rows, dtype=np.int64)
-    out = np.empty((rows.size, geo.H, geo.D), dtype=np.float64)
+    out = np.full((rows.size, geo.H, geo.D), np.nan)
     q_all = f64(Q, rows)
     kept = geo.kept_tokens()
     k_kept, v_kept = f64(K, kept), f64(V, kept)  # [NK, H, D]
@@ -469,7 +527,7 @@ def combine(g_rows: np.ndarray, o_cmp_up: np.ndarray, o_sel: np.ndarray) -> np.n
 
 
 def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
-              tie_window: float = 1e-3, chunk_elems: int = 50_000_000, pooled=None) -> dict:
+              tie_window: float = 1e-3, chunk_elems: int | None = None, pooled=None) -> dict:
     """The GSA layer for fine query tokens ``rows`` (all tokens when None).
 
     Returns a dict of float64 arrays:
@@ -486,8 +544,12 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     (no unchosen block beats a chosen one by ``tie_window`` or more).
 
     ``pooled`` = (pool(Q), pool(K), pool(V)) from an earlier call on the same
-    inputs skips recomputing step 1.
+    inputs skips recomputing step 1.  Steps 2-4 run over the entries in
+    chunks whose logits hold about ``chunk_elems`` values
+    (``CHUNKS.layer_chunk_elems``).
     """
+    if chunk_elems is None:
+        chunk_elems = CHUNKS.layer_chunk_elems
     rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
     if pooled is None:
         Qc, Kc, Vc = pool(geo, Q), pool(geo, K), pool(geo, V)
@@ -499,19 +561,19 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     Vc_keys = heads_first(Vc).transpose(1, 0, 2)
     entries = np.array(sorted({geo.entry_of_token(int(t)) for t in rows}), dtype=np.int64)
     nE = entries.size
-    o_cmp = np.empty((nE, geo.H, geo.D))
-    sel = np.empty((nE, geo.H, geo.K), dtype=np.int64)
-    gap = np.empty((nE, geo.H))
+    # NaN (or an id below -1) marks anything a chunk left unwritten
+    o_cmp = np.full((nE, geo.H, geo.D), np.nan)
+    sel = np.full((nE, geo.H, geo.K), -2, dtype=np.int64)
+    gap = np.full((nE, geo.H), np.nan)
     keep_guide = nE * geo.NB * geo.H <= 50_000_000
-    guide_all = np.empty((nE, geo.H, geo.NB)) if keep_guide else None
+    guide_all = np.full((nE, geo.H, geo.NB), np.nan) if keep_guide else None
     other = None
     if sel_override is not None:
         other = np.asarray(sel_override)[entries].astype(np.int64)
         sel_exact = np.zeros((nE, geo.H), dtype=bool)
         sel_valid = np.zeros((nE, geo.H), dtype=bool)
     step = max(1, chunk_elems // (geo.H * geo.Tc))
-    for e0 in range(0, nE, step):
-        e1 = min(nE, e0 + step)
+    for e0, e1 in spans(nE, step):
         o, logits = compressed_attention(geo, Qc[entries[e0:e1]], Kc_keys, Vc_keys)
         o_cmp[e0:e1] = o
         guide = guide_scores(geo, logits)
@@ -543,8 +605,8 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
 # dense global attention (the layer GSA replaces)
 
 
-def dense_attention(geo: Geometry, Q, K, V, rows=None, key_chunk: int = 1 << 14,
-                    max_bytes: int = 1 << 30) -> np.ndarray:
+def dense_attention(geo: Geometry, Q, K, V, rows=None, key_chunk: int | None = None,
+                    max_bytes: int | None = None) -> np.ndarray:
     """softmax(q K^T / sqrt(D)) V over all T tokens, for fine query ``rows``.
 
     Speed3R, technical summary 1 (Background): the dense global attention of
@@ -555,21 +617,22 @@ def dense_attention(geo: Geometry, Q, K, V, rows=None, key_chunk: int = 1 << 14,
     two passes: the row maximum of the scaled logits over all keys first, then
     sum_j exp(s_j - max) v_j and sum_j exp(s_j - max), divided at the end --
     the textbook formula, without online rescaling.  Rows are taken in chunks
-    whose logits of one key slice fit in ``max_bytes``.
+    whose logits of one key slice fit in ``max_bytes``.  (Defaults:
+    ``CHUNKS.dense_key_chunk`` and ``CHUNKS.dense_max_bytes``.)
     """
+    key_chunk = CHUNKS.dense_key_chunk if key_chunk is None else key_chunk
+    max_bytes = CHUNKS.dense_max_bytes if max_bytes is None else max_bytes
     rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
-    out = np.empty((rows.size, geo.H, geo.D))
+    out = np.full((rows.size, geo.H, geo.D), np.nan)
     if geo.T <= key_chunk:
         k_all, v_all = f64(K), f64(V)
         step = max(1, max_bytes // max(geo.H * geo.T * 8, 1))
-        for r0 in range(0, rows.size, step):
-            r1 = min(rows.size, r0 + step)
+        for r0, r1 in spans(rows.size, step):
             out[r0:r1] = weighted_values(softmax(qk_logits(f64(Q, rows[r0:r1]), k_all, geo.sm_scale)), v_all)
         return out
     step = max(1, max_bytes // (geo.H * key_chunk * 8))
-    slices = [slice(t0, min(geo.T, t0 + key_chunk)) for t0 in range(0, geo.T, key_chunk)]
-    for r0 in range(0, rows.size, step):
-        r1 = min(rows.size, r0 + step)
+    slices = [slice(t0, t1) for t0, t1 in spans(geo.T, key_chunk)]
+    for r0, r1 in spans(rows.size, step):
         q = f64(Q, rows[r0:r1])
         m = torch.full((r1 - r0, geo.H), -np.inf, dtype=torch.float64)
         for sl in slices:
@@ -595,7 +658,7 @@ def frame_attention(geo: Geometry, Q, K, V, rows=None) -> np.ndarray:
     attends within each frame only.
     """
     rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
-    out = np.empty((rows.size, geo.H, geo.D))
+    out = np.full((rows.size, geo.H, geo.D), np.nan)
     frame = rows // geo.L
     for f in np.unique(frame):
         idx = np.nonzero(frame == f)[0]
@@ -637,7 +700,9 @@ def sga_attention(geo: Geometry, Q, K, V, sub_h: int, sub_w: int, rows=None) -> 
     is kept as well, once; the dropped columns are replaced by a single pair
     (mean of the dropped keys, mean of the dropped values) -- read here as one
     more ordinary key, with no weight for how many columns it stands for.  One
-    softmax runs over [kept keys, own key if dropped, mean key].
+    softmax runs over [kept keys, own key if dropped, mean key].  The dropped
+    tokens are summed ``CHUNKS.sga_mean_tokens`` at a time and the queries
+    taken in chunks of about ``CHUNKS.sga_row_elems`` logits.
     """
     rows = np.arange(geo.T) if rows is None else np.asarray(rows, dtype=np.int64)
     kept = sga_key_tokens(geo, sub_h, sub_w)
@@ -650,16 +715,15 @@ def sga_attention(geo: Geometry, Q, K, V, sub_h: int, sub_w: int, rows=None) -> 
     if dropped.size:
         k_mean = np.zeros((geo.H, geo.D))
         v_mean = np.zeros((geo.H, geo.D))
-        for t0 in range(0, dropped.size, 1 << 16):
-            part = dropped[t0:t0 + (1 << 16)]
+        for t0, t1 in spans(dropped.size, CHUNKS.sga_mean_tokens):
+            part = dropped[t0:t1]
             k_mean += f64(K, part).sum(axis=0)
             v_mean += f64(V, part).sum(axis=0)
         k_mean /= dropped.size
         v_mean /= dropped.size
-    out = np.empty((rows.size, geo.H, geo.D))
-    step = max(1, (1 << 27) // max(geo.H * (kept.size + 2), 1))
-    for r0 in range(0, rows.size, step):
-        r1 = min(rows.size, r0 + step)
+    out = np.full((rows.size, geo.H, geo.D), np.nan)
+    step = max(1, CHUNKS.sga_row_elems // max(geo.H * (kept.size + 2), 1))
+    for r0, r1 in spans(rows.size, step):
         qq = q[r0:r1]
         s_kept = qk_logits(qq, k_kept, geo.sm_scale)                               # [r, H, NK]
         s_own = np.sum(qq * k_own[r0:r1], axis=-1) * geo.sm_scale                  # [r, H]

@@ -342,6 +342,72 @@ def pin_sga():
     assert list(ids[:per_frame]) == [0, 1, 2, 5, 8, 16, 19, 22, 30, 33, 36]
 
 
+# ---------------------------------------------------------------------------
+# the split forms the oracle takes at full size, forced on micro inputs
+
+
+def _same(a, b, what):
+    """Two runs of the oracle that differ only in how the work is split."""
+    for key in a:
+        if key in b and isinstance(a[key], np.ndarray) and a[key].dtype != bool:
+            close(a[key], b[key], tol=1e-12, what=f"{what}: {key}")
+
+
+def pin_split_layer():
+    """The whole layer with every split form forced: torch's threaded softmax
+    for every softmax, pooling two frames at a time (three frames: a ragged
+    last slice) and steps 2-4 over chunks of five compressed entries (a ragged
+    last chunk) equals the unsplit run and the brute force, for both always-kept
+    readings and for a subset of rows."""
+    for keep in ("specials", "reference"):
+        geo, x = micro(N=3, S=2, Hp=6, Wp=7, H=2, D=8, P=4, K=3, keep=keep)
+        assert geo.N % 2 == 1 and geo.Tc % 5 != 0
+        plain = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+        rows = np.array([0, 2, 9, geo.L + 4, geo.T - 7, geo.T - 1])
+        with O.chunking(softmax_torch_elems=1, pool_frames=2, layer_chunk_elems=5 * geo.H * geo.Tc):
+            split = O.gsa_layer(geo, x.q, x.k, x.v, x.w)
+            sub = O.gsa_layer(geo, x.q, x.k, x.v, x.w, rows=rows)
+        _same(plain, split, f"split layer ({keep})")
+        close(sub["out"], plain["out"][rows], tol=1e-12, what=f"split layer rows ({keep})")
+        Q, K, V, W = (t.to(torch.float64).tolist() for t in (x.q, x.k, x.v, x.w))
+        bf = bruteforce.gsa_bruteforce(Q, K, V, W, geo.N, geo.S, geo.Hp, geo.Wp, geo.P, geo.K, keep=keep)
+        assert split["sel"].tolist() == bf["sel"], f"split layer selection ({keep})"
+        for key in ("o_cmp", "o_sel", "g", "out"):
+            close(split[key], bf[key], what=f"split layer vs brute force ({keep}): {key}")
+
+
+def pin_split_dense():
+    """Dense and frame attention with their split forms forced: rows three at a
+    time through torch's softmax (short sequences), then key slices of seven
+    tokens with rows in chunks of three (long sequences), against torch's SDPA."""
+    geo, x = micro(N=3, S=2, Hp=4, Wp=5, H=2, D=8)
+    want = sdpa_dense(x.q, x.k, x.v)
+    with O.chunking(softmax_torch_elems=1, dense_max_bytes=3 * geo.H * geo.T * 8):
+        close(O.dense_attention(geo, x.q, x.k, x.v), want, what="dense, rows in threes, torch softmax")
+        L = geo.L
+        frames = np.concatenate([sdpa_dense(x.q[f * L:(f + 1) * L], x.k[f * L:(f + 1) * L],
+                                            x.v[f * L:(f + 1) * L]) for f in range(geo.N)])
+        close(O.frame_attention(geo, x.q, x.k, x.v), frames, what="frame attention, torch softmax")
+    with O.chunking(dense_key_chunk=7, dense_max_bytes=3 * geo.H * 7 * 8):
+        close(O.dense_attention(geo, x.q, x.k, x.v), want, what="dense in key slices of 7")
+
+
+def pin_split_sga():
+    """SGA with its split forms forced: the dropped tokens summed five at a time,
+    queries three at a time, torch's softmax; against the unsplit run and the
+    brute force."""
+    geo, x = micro(N=2, S=2, Hp=5, Wp=7, H=2, D=8)
+    Q, K, V = (t.to(torch.float64).tolist() for t in (x.q, x.k, x.v))
+    for sh, sw in ((2, 3), (3, 2)):
+        nk = O.sga_key_tokens(geo, sh, sw).size
+        plain = O.sga_attention(geo, x.q, x.k, x.v, sh, sw)
+        with O.chunking(softmax_torch_elems=1, sga_mean_tokens=5, sga_row_elems=3 * geo.H * (nk + 2)):
+            split = O.sga_attention(geo, x.q, x.k, x.v, sh, sw)
+        close(split, plain, tol=1e-12, what=f"split sga {sh}x{sw}")
+        close(split, bruteforce.sga_bruteforce(Q, K, V, geo.L, geo.S, geo.Hp, geo.Wp, sh, sw),
+              what=f"split sga {sh}x{sw} brute force")
+
+
 def all_pins(fixture_path):
     return {
         "block_structure": lambda: pin_block_structure(fixture_path),
@@ -364,4 +430,7 @@ def all_pins(fixture_path):
         "reference_one_frame": pin_reference_one_frame,
         "reference_k_all": pin_reference_k_all,
         "reference_bruteforce": pin_reference_bruteforce,
+        "split_layer": pin_split_layer,
+        "split_dense": pin_split_dense,
+        "split_sga": pin_split_sga,
     }

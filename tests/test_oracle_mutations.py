@@ -6,10 +6,12 @@ least one pin in ``pins.py`` fail.
 """
 
 import os
+import sys
 import warnings
 
 import numpy as np
 import pytest
+import torch
 
 import pins
 from oracle import gsa_oracle as O
@@ -17,7 +19,7 @@ from oracle import gsa_oracle as O
 FIXTURE = os.path.join(os.path.dirname(__file__), "golden", "block_structure_37x37_p4.txt")
 
 
-def _pool_full_denominator(geo, X, frames_per_chunk=32):
+def _pool_full_denominator(geo, X, frames_per_chunk=None):
     out = _orig["pool"](geo, X, frames_per_chunk)
     # re-weight every block entry as if it always held P*P patches
     for f in range(geo.N):
@@ -160,8 +162,32 @@ def _gate_wrong_sign(geo, Qc_rows, w):
     return 1.0 - _orig["gate"](geo, Qc_rows, w)
 
 
+def _softmax_torch_wrong_axis(z, axis=-1):
+    # the threaded (large-array) form normalises over the first axis
+    z = np.asarray(z, dtype=np.float64)
+    if z.size < O.CHUNKS.softmax_torch_elems:
+        return _orig["softmax"](z, axis)
+    t = torch.from_numpy(z)
+    e = torch.exp(t - torch.amax(t, dim=0, keepdim=True))
+    return (e / torch.sum(e, dim=0, keepdim=True)).numpy()
+
+
+def _spans_mistake(caller, how):
+    """spans() that, only when called from ``caller`` and only when the work is
+    really split, drops the last slice or skips the first element of every
+    slice after the first (an off-by-one at the boundaries)."""
+    def mutated(n, step):
+        out = _orig["spans"](n, step)
+        if sys._getframe(1).f_code.co_name != caller or len(out) < 2:
+            return out
+        if how == "drop_last":
+            return out[:-1]
+        return [(a + (1 if i else 0), b) for i, (a, b) in enumerate(out)]
+    return mutated
+
+
 _orig = {n: getattr(O, n) for n in ("pool", "compressed_attention", "selected_keys", "combine", "gate",
-                                     "dense_attention")}
+                                     "dense_attention", "softmax", "spans")}
 _orig["Geometry.kept_tokens"] = O.Geometry.kept_tokens
 
 MUTATIONS = {
@@ -186,7 +212,12 @@ MUTATIONS = {
     "reference keep still ranks frame 0's blocks": ("Geometry.B0", property(lambda self: 0)),
     "reference keep keeps every register token": ("Geometry.kept_tokens", _kept_all_specials_of_later_frames),
     "reference keep takes the camera from the last slot": ("Geometry.kept_tokens", _kept_camera_from_last_slot),
+    "threaded softmax over the wrong axis": ("softmax", _softmax_torch_wrong_axis),
 }
+# every split loop of the oracle, with each boundary mistake
+for _fn in ("pool", "gsa_layer", "dense_attention", "sga_attention"):
+    for _how, _what in (("drop_last", "drops its last slice"), ("skip", "skips a slice boundary")):
+        MUTATIONS[f"{_fn} {_what} when split"] = ("spans", _spans_mistake(_fn, _how))
 
 
 @pytest.mark.parametrize("name", sorted(MUTATIONS))

@@ -311,10 +311,20 @@ gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out);
  *   without ordering) race on the array and corrupt each other's results:
  *   order them.
  * - Allocates nothing: no cudaMalloc / cudaFree and no allocating library call.
+ * - In-kernel failures (a bounded wait that ran out, a selection id out of
+ *   range) set bits in the array's error word, as they do in a workspace's;
+ *   read them with gsa_noalloc_check_device_error before the next no-alloc
+ *   call on the device, which zeroes the word again.
  */
 #define GSA_NOALLOC_SCRATCH_BYTES (32u << 20)
 gsa_status gsa_forward_noalloc(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
                                const gsa_bf16* v, const float* w, gsa_bf16* out, void* stream);
+
+/* gsa_check_device_error for gsa_forward_noalloc: synchronise `stream`, read
+ * and clear the error word of the fixed array on the current device, and
+ * return GSA_OK, GSA_ERR_TIMEOUT or GSA_ERR_DEVICE_CHECK (GSA_ERR_CUDA if the
+ * array's address cannot be looked up).  Allocates nothing. */
+gsa_status gsa_noalloc_check_device_error(void* stream);
 
 /* Synchronise `stream`, read the device error word in `ws`, clear it, and
  * return GSA_OK, GSA_ERR_TIMEOUT or GSA_ERR_DEVICE_CHECK. */

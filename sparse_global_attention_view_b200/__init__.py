@@ -22,6 +22,7 @@ from .api import (  # noqa: F401
     sga_attn,
     gate_combine,
     new_workspace,
+    noalloc_check_device_error,
     pool_kv,
     selected_attn,
     topk_blocks,

@@ -92,6 +92,7 @@ SIGNATURES = {
     "gsa_forward_timed": [P_SHAPE] + [c_vp] * 6 + [c_size, c_vp, ctypes.POINTER(c_i32), c_vp],
     "gsa_workspace_offsets": [P_SHAPE, ctypes.POINTER(GsaWsOffsets)],
     "gsa_forward_noalloc": [P_SHAPE] + [c_vp] * 6,
+    "gsa_noalloc_check_device_error": [c_vp],
     "gsa_check_device_error": [c_vp, c_vp],
     "gsa_status_string": [c_i32],
 }

@@ -228,6 +228,12 @@ def forward_noalloc(shape, q, k, v, w, out, stream=None) -> None:
         "gsa_forward_noalloc")
 
 
+def noalloc_check_device_error(stream=None) -> None:
+    """Synchronise, then read and clear the error word of the fixed array that
+    ``forward_noalloc`` uses on the current device; raises on a device error."""
+    check(load().gsa_noalloc_check_device_error(_stream(stream)), "gsa_noalloc_check_device_error")
+
+
 def forward_timed(shape, q, k, v, w, out, ws, events, stream=None) -> int:
     """``forward`` recording ``events`` (len(FORWARD_STEPS) + 1 torch.cuda.Event
     with timing, already recorded once so their handles exist) between its

@@ -53,3 +53,12 @@ extern "C" gsa_status gsa_forward_noalloc(const gsa_shape* shape, const gsa_bf16
     return GSA_ERR_CUDA;
   return gsa_forward(shape, q, k, v, w, out, ws, (size_t)GSA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+extern "C" gsa_status gsa_noalloc_check_device_error(void* stream) {
+  // the fixed array's first word is the error word of the last no-alloc call
+  // on the current device (its header was zeroed when that call began)
+  void* ws = nullptr;
+  gsa_status st = scratch_for_current_device(&ws);
+  if (st != GSA_OK) return st;
+  return gsa_check_device_error(ws, stream);
+}

@@ -185,6 +185,16 @@ def test_noalloc_rejects_shapes_beyond_its_scratch(lib):
     assert b"noalloc" in lib.gsa_status_string(7)
 
 
+def test_noalloc_limit_falls_between_four_and_five_vggt_frames(lib):
+    """The fixed array holds the VGGT token layout (5 + 37x37 tokens per frame,
+    16 heads, K = 16) up to 4 frames and no more: a layout change that moves
+    this limit fails here, on the CPU."""
+    from sparse_global_attention_view_b200 import workspace_size
+    from sparse_global_attention_view_b200._lib import NOALLOC_SCRATCH_BYTES
+    assert workspace_size(shape(n_frames=4, top_k=16)) <= NOALLOC_SCRATCH_BYTES
+    assert workspace_size(shape(n_frames=5, top_k=16)) > NOALLOC_SCRATCH_BYTES
+
+
 def test_status_strings(lib):
     for code in range(8):
         assert lib.gsa_status_string(code)

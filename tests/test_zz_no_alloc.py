@@ -47,5 +47,6 @@ def test_noalloc_matches_workspace_forward_on_two_calls(name):
         out = torch.full_like(q, float("nan"))
         G.forward_noalloc(shape, q, k, v, w, out)
         torch.cuda.synchronize()
-        G.check_device_error(layer.ws)
+        G.check_device_error(layer.ws)       # the workspace call
+        G.noalloc_check_device_error()       # the no-alloc call's own error word
         PT.assert_close(out, ref.double().cpu().numpy(), f"{name} noalloc call {call + 1}")

@@ -7,9 +7,11 @@ A step is one whole GSA layer (pooling, compressed attention, S_guide top-K,
 top-K merge, selected attention with the gate) over the workload's tokens, with
 Q/K/V resident in HBM.  The metric is tokens per second of the layer (and ms
 per layer); the dense global attention it replaces is timed in the same run.
-Multi-GPU runs (torchrun, one rank per GPU) give every rank its own scene of the
-same size: there is no exchange inside the layer, so the scaling is weak and
-the value is all ranks' tokens over the slowest rank's time.
+Multi-GPU runs (torchrun, one rank per GPU) split one scene's heads over the
+ranks (every head attends independently, so the layer has no exchange step):
+strong scaling, the scene's tokens over the slowest rank's time.  With
+``--parallel replicas`` every rank runs its own scene of the same size instead
+(weak scaling, all ranks' tokens over the slowest rank's time).
 
 Prints one JSON line on rank 0.
 """
@@ -72,10 +74,24 @@ def stage_work(z, H, D, K_eff) -> dict:
         "topk_merge": ("hbm", H * Tc * K_eff * 8 + H * Tc * K_eff * 4, "bytes"),
         # QK^T and PV of every token over the NK always-kept tokens
         "kept_attn": ("tensor", 4 * T * NK * H * D, "flop"),
-        # the selected blocks' K and V gathered per (entry, head): K_eff blocks of
-        # (at most) 16 tokens x 128 bytes, K and V
-        "selected_gate": ("hbm", H * Tc * K_eff * 16 * D * 2 * 2, "bytes"),
+        # the selected blocks' K and V gathered per (entry, head): K_eff blocks
+        # of (on average) Hp*Wp/Bf valid tokens x 128 bytes, K and V; the bench
+        # replaces this with the exact count of the run's own selection
+        "selected_gate": ("gather", H * Tc * K_eff * (z.T - NS) // max(z.NB, 1) * D * 2 * 2, "bytes"),
     }
+
+
+def selected_bytes(sel, z, shape) -> int:
+    """K and V bytes of the valid tokens of every selected block, summed over
+    all (head, entry) selections: what the selection branch must gather."""
+    Bh = -(-shape.hp // shape.pool)
+    Bw = -(-shape.wp // shape.pool)
+    rows = torch.clamp(shape.hp - torch.arange(Bh) * shape.pool, max=shape.pool)
+    cols = torch.clamp(shape.wp - torch.arange(Bw) * shape.pool, max=shape.pool)
+    per_block = (rows[:, None] * cols[None, :]).reshape(-1).to(sel.device)  # valid tokens by position
+    valid = sel >= 0
+    tokens = torch.where(valid, per_block[torch.where(valid, sel, 0) % (Bh * Bw)], 0)
+    return int(tokens.sum().item()) * shape.head_dim * 2 * 2
 
 
 def dense_flops(z, H, D) -> int:
@@ -172,6 +188,7 @@ def cpu_threads() -> int:
 def run_reference(args) -> None:
     """The float64 CPU oracle as the reference arm (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
     torch.set_num_threads(os.cpu_count() or 1)
@@ -199,7 +216,8 @@ def run_reference(args) -> None:
         "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": layer_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(wl),
+        "data": "synthetic",
+        "config": workload_config(wl, l2_note(wl, world, args.parallel), parallelism_of(wl, world, args.parallel)),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -214,6 +232,28 @@ def chosen_workload(args):
     if args.keep:
         wl = wl.with_(keep=args.keep)
     return wl
+
+
+def inputs_exceed_l2(in_bytes: int) -> bool:
+    """Q/K/V of one rank large enough (4x the 126 MB L2) that no flush is needed."""
+    return in_bytes > 4 * 126 * 2**20
+
+
+def l2_note(wl, world: int = 1, parallel: str = "replicas") -> str:
+    """How the timed region keeps one rank's inputs out of L2."""
+    heads = wl.n_heads
+    if world > 1 and parallel == "heads":
+        heads = -(-wl.n_heads // world)  # the largest head slice
+    in_bytes = 3 * wl.n_tokens * heads * wl.head_dim * 2
+    if inputs_exceed_l2(in_bytes):
+        return f"inputs larger than L2 ({in_bytes / 1e9:.1f} GB of Q/K/V)"
+    return "L2 flushed between steps (256 MB write, outside the per-kernel events)"
+
+
+def parallelism_of(wl, world: int, parallel: str) -> str:
+    if world > 1 and parallel == "heads":
+        return f"heads (one scene; {wl.n_heads} heads split over {world} ranks, no exchange in the layer)"
+    return "replicas (independent scene per rank)"
 
 
 def workload_config(wl, l2_note=None, parallelism="replicas (independent scene per rank)") -> dict:
@@ -312,8 +352,9 @@ def main() -> None:
     ap.add_argument("--sga-steps", type=int, default=2)
     ap.add_argument("--cpu-entries", type=int, default=48, help="query blocks in the cpu_baseline sample")
     ap.add_argument("--ref-entries", type=int, default=16, help="query blocks per reference-arm step")
-    ap.add_argument("--parallel", choices=["replicas", "heads"], default="replicas",
-                    help="N > 1: independent scenes per rank (weak scaling) or one scene split by heads (strong)")
+    ap.add_argument("--parallel", choices=["replicas", "heads"], default="heads",
+                    help="N > 1: one scene split by heads (strong scaling, the default) or independent "
+                         "scenes per rank (weak scaling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "gsa":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -344,9 +385,8 @@ def main() -> None:
     wl = rank_workload(chosen_workload(args), rank, args.parallel)
     wl_scene = wl
     x = generate(wl)
-    parallelism = "replicas (independent scene per rank)"
+    parallelism = parallelism_of(wl, world, mode)
     if mode == "heads":
-        parallelism = f"heads (one scene; {wl.n_heads} heads split over {world} ranks, no exchange in the layer)"
         h0, h1 = head_slice(world, rank, wl.n_heads)
         x.q, x.k, x.v = (t[:, h0:h1].contiguous() for t in (x.q, x.k, x.v))
         x.w = x.w[h0:h1].contiguous()
@@ -360,8 +400,7 @@ def main() -> None:
     q, k, v, w = (t.to(dev) for t in (x.q, x.k, x.v, x.w))
     out = torch.empty_like(q)
     layer = G.GsaLayer(shape, dev)
-    in_bytes = 3 * q.numel() * 2
-    big = in_bytes > 4 * 126 * 2**20
+    big = inputs_exceed_l2(3 * q.numel() * 2)
     flush = None if big else torch.empty(256 * 2**20, dtype=torch.uint8, device=dev)
     n_ev = len(G.FORWARD_STEPS) + 1
 
@@ -409,6 +448,7 @@ def main() -> None:
     # ---- per-stage roofline from the same timed steps ----
     P = peaks()
     work = stage_work(z, H, D, min(shape.top_k, z.NB))
+    gathered = selected_bytes(G.workspace_view(layer.ws, shape, "sel"), z, shape)
     alu_peak = SM_COUNT * FFMA_PER_SM_PER_CLK * 2 * P["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s fp32 FMA
     # the fused compressed stage does QK^T in tf32 (half the bf16 rate) and PV in
     # bf16, equal flops each: its tensor peak is 2/3 of the bf16 peak
@@ -419,7 +459,9 @@ def main() -> None:
         ms = stage_ms[name]
         if ms <= 0:
             continue
-        if bound == "hbm":
+        if name == "selected_gate":
+            amount = gathered
+        if bound in ("hbm", "gather"):
             ach, peak, u = amount / (ms / 1e3) / 1e9, P["hbm_gbs"], "GB/s"
         elif bound == "tensor":
             ach, peak, u = amount / (ms / 1e3) / 1e12, P["bf16_tflops"], "TFLOP/s"
@@ -432,6 +474,10 @@ def main() -> None:
         stages[name] = {"ms": round(ms, 4), "share": round(ms / sum(stage_ms.values()), 4), "bound": bound,
                         "achieved": round(ach, 2), "peak": round(peak, 1), "unit": u,
                         "frac": round(ach / peak, 4)}
+        if name == "selected_gate":
+            stages[name]["note"] = ("achieved = K/V bytes of the valid tokens of the selected blocks "
+                                    f"({amount / 1e9:.1f} GB, counted from this run's selection) per second, "
+                                    "moved L2 -> SM; peak = measured HBM copy bandwidth")
     dom = max(stages, key=lambda n: stages[n]["ms"])
     ds = stages[dom]
     traffic = recorded_traffic(STAGE_SOURCE[dom], wl.name)
@@ -608,8 +654,7 @@ def main() -> None:
                   "sel_exact_where_gap_ge_1e-3": float(res["sel_exact"][wide].mean()) if wide.any() else None,
                   "sel_exact_frac": float(res["sel_exact"].mean())}
 
-    l2 = (f"inputs larger than L2 ({in_bytes / 1e9:.1f} GB of Q/K/V)" if big else
-          "L2 flushed between steps (256 MB write, outside the per-kernel events)")
+    l2 = l2_note(wl_scene, world, mode)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,

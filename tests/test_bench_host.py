@@ -49,6 +49,27 @@ def test_stage_work_at_the_pages_workload():
     work = bench.stage_work(z, 16, 64, 64)
     assert work["compressed_attn"] == ("tensor", 4 * 105_000 ** 2 * 16 * 64, "flop")
     assert work["kept_attn"] == ("tensor", 4 * 1_374_000 * 5000 * 16 * 64, "flop")
-    assert work["selected_gate"][1] == 16 * 105_000 * 64 * 16 * 64 * 2 * 2
+    # 1369 valid tokens in 100 blocks per frame: 13.69 per selected block on average
+    assert work["selected_gate"][0] == "gather"
+    assert work["selected_gate"][1] == 16 * 105_000 * 64 * 1_369_000 // 100_000 * 64 * 2 * 2
     # Q, K, V read once: 3 x 1,374,000 x 16 x 64 x 2 bytes, plus the pooled and kept writes
     assert work["pool"][1] > 3 * 1_374_000 * 16 * 64 * 2
+
+
+def test_selected_bytes_counts_valid_tokens_of_each_selected_block():
+    import torch
+    from sparse_global_attention_view_b200 import Shape
+    # 6 x 7 grid, P = 4: blocks (0,0) 16 tokens, (0,1) 4 x 3 = 12, (1,0) 2 x 4 = 8, (1,1) 2 x 3 = 6
+    shape = Shape(n_frames=2, n_special=1, hp=6, wp=7, n_heads=2, top_k=3)
+    sel = torch.tensor([[[0, 1, -1], [4, 7, 3]], [[2, -1, -1], [5, 6, 0]]], dtype=torch.int32)
+    tokens = (16 + 12) + (16 + 6 + 6) + 8 + (12 + 8 + 16)
+    assert bench.selected_bytes(sel, None, shape) == tokens * 64 * 2 * 2
+
+
+@pytest.mark.parametrize("world,parallel", [(1, "heads"), (1, "replicas"), (2, "heads"), (8, "heads"),
+                                            (4, "replicas")])
+def test_both_arms_describe_the_same_config(world, parallel):
+    wl = WORKLOADS["pages"]
+    cfg = bench.workload_config(wl, bench.l2_note(wl, world, parallel), bench.parallelism_of(wl, world, parallel))
+    assert "l2" in cfg and "L2" in cfg["l2"]
+    assert cfg["parallelism"].startswith("heads" if (world > 1 and parallel == "heads") else "replicas")

@@ -68,10 +68,12 @@ def stage_work(z, H, D, K_eff) -> dict:
                  + (2 * NK * H * D * 2 if NK != NS else 0), "bytes"),
         # QK^T and PV over the Tc x Tc pooled sequence
         "compressed_attn": ("tensor", 4 * Tc * Tc * H * D, "flop"),
-        # one fp32 dot product of length D per (entry, candidate block, head)
-        "block_scores": ("alu", 2 * Tc * (NB - z.B0) * H * D, "flop"),
-        # candidates read once, selection written once
-        "topk_merge": ("hbm", H * Tc * K_eff * 8 + H * Tc * K_eff * 4, "bytes"),
+        # K > 64: the second, ranking-only pass of the fused kernel: QK^T in tf32
+        "block_scores": ("tensor", 2 * Tc * Tc * H * D, "flop"),
+        # the ordering of the selection branch's pairs (each row's best block
+        # read twice, the order written once), and for K > 64 the union of the
+        # two selections (two lists read, one written)
+        "topk_merge": ("hbm", H * Tc * 12 + (H * Tc * K_eff * 12 if K_eff > 64 else 0), "bytes"),
         # QK^T and PV of every token over the NK always-kept tokens
         "kept_attn": ("tensor", 4 * T * NK * H * D, "flop"),
         # the selected blocks' K and V gathered per (entry, head): K_eff blocks
@@ -452,7 +454,7 @@ def main() -> None:
     alu_peak = SM_COUNT * FFMA_PER_SM_PER_CLK * 2 * P["sm_max_mhz"] * 1e6 / 1e12  # TFLOP/s fp32 FMA
     # the fused compressed stage does QK^T in tf32 (half the bf16 rate) and PV in
     # bf16, equal flops each: its tensor peak is 2/3 of the bf16 peak
-    fused_cmp = stage_ms["block_scores"] < 0.01 * stage_ms["compressed_attn"]
+    fused_cmp = True
     stages = {}
     for name in G.FORWARD_STEPS:
         bound, amount, unit = work[name]
@@ -467,6 +469,8 @@ def main() -> None:
             ach, peak, u = amount / (ms / 1e3) / 1e12, P["bf16_tflops"], "TFLOP/s"
             if name == "compressed_attn" and fused_cmp:
                 peak = P["bf16_tflops"] * 2.0 / 3.0
+            if name == "block_scores":  # tf32 only: half the bf16 rate
+                peak = P["bf16_tflops"] / 2.0
         else:
             ach, peak, u = amount / (ms / 1e3) / 1e12, alu_peak, "TFLOP/s"
         if ms < 0.005:

@@ -89,6 +89,12 @@ typedef struct {
   int32_t top_k;     /* K in [1, 128]: selected blocks per (query block, head) */
   float scale;       /* softmax scale; 0 means 1/sqrt(D) */
   int32_t keep;      /* always-kept set of the selection branch: GSA_KEEP_* */
+  int32_t wait_limit_ns; /* >= 0; 0 = default.  Every in-kernel wait of one pipeline role
+                            on another (a TMA copy, a tensor-core product, a softmax tile)
+                            gives up after about this many nanoseconds (default about 2 s)
+                            and records GSA_ERR_TIMEOUT in the error word; the kernel then
+                            drains its own copies and products and returns.  A tiny value
+                            exercises that path (test hook). */
 } gsa_shape;
 
 #define GSA_KEEP_SPECIALS 0  /* every special token of every frame */
@@ -257,15 +263,18 @@ gsa_status gsa_forward(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
  * cudaEvent_t handles created by the caller; events[0] is recorded on `stream`
  * before the first kernel and events[i+1] after step i, the steps being
  *   0 pooling, 1 compressed attention, 2 S_guide block scores with the
- *   streaming top-K, 3 top-K merge, 4 attention of every token over the
- *   always-kept tokens, 5 attention over the selected blocks, merged with
- *   step 4, with the gate.
- * For K <= 64 steps 1-3 are one fused kernel (step 1's interval holds it).
+ *   streaming top-K, 3 top-K merge and the ordering of the selection branch's
+ *   work, 4 attention of every token over the always-kept tokens, 5 attention
+ *   over the selected blocks, merged with step 4, with the gate.
+ * For K <= 64 steps 1-2 are one fused kernel (step 1's interval holds it) and
+ * step 3 sorts the (head, entry) pairs by the grid position of their
+ * best-scoring block, so that pairs whose selections cover the same region of
+ * every frame run together and share K/V blocks in L2.
  * For 64 < K <= 128 step 1 is the fused kernel ranking the top 64 (and
- * recording each row's 64th-best (score, id) key), step 2 a second,
+ * recording each row's 64th-best (score, entry) key), step 2 a second,
  * ranking-only pass of it for the next K - 64 pairs strictly below that key,
- * and step 3 the ascending union of the two selections (Speed3R technical
- * summary 4: a larger Top-K at test time).
+ * and step 3 the ascending union of the two selections and the ordering
+ * (Speed3R technical summary 4: a larger Top-K at test time).
  * A step fused into another one (or absent, such as step 4 when NK == 0)
  * records an empty interval.  If `n_launched` is not NULL it receives
  * the number of kernels enqueued.
@@ -278,12 +287,15 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
 
 /* Byte offsets of gsa_forward's intermediates inside its workspace (host only),
  * for inspecting them after a call: the buffers of gsa_pool_kv (qc32, kc32, vc,
- * qc, kc, ks, vs), oc, the candidates (n_split lists per row), sel, and the
+ * qc, kc, ks, vs), oc, the candidates (n_split lists per row), sel, the
  * always-kept segment's fp32 output [T][H][64] and lse [T][H] (empty when
- * NK == 0). */
+ * NK == 0), and the ordering of the selection branch's work: best [H][Tc]
+ * int32, each row's best-scoring block (-1 when it has none), and order
+ * [H*Tc] int32, the pairs h*Tc + a sorted by (h, best mod Bh*Bw). */
 typedef struct {
   size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cand_score, cand_idx, sel, o_spec, lse_spec, total;
   int32_t n_split;
+  size_t best, order;
 } gsa_ws_offsets;
 gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out);
 
@@ -332,6 +344,12 @@ gsa_status gsa_check_device_error(void* ws, void* stream);
 
 /* Static text for a status code. */
 const char* gsa_status_string(gsa_status status);
+
+/* What a GSA_ERR_CUDA was: the CUDA runtime's last error in the calling host
+ * thread (cudaPeekAtLastError: not cleared; a fault of a kernel stays set for
+ * the context) and the static name of a CUDA error code. */
+int32_t gsa_last_cuda_error(void);
+const char* gsa_cuda_error_name(int32_t code);
 
 #ifdef __cplusplus
 }

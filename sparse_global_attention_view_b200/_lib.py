@@ -39,6 +39,7 @@ class GsaShape(ctypes.Structure):
         ("top_k", c_i32),
         ("scale", c_f32),
         ("keep", c_i32),
+        ("wait_limit_ns", c_i32),
     ]
 
 
@@ -66,7 +67,7 @@ class GsaSizes(ctypes.Structure):
 class GsaWsOffsets(ctypes.Structure):
     _fields_ = [(n, c_size) for n in ("qc32", "kc32", "vc", "qc", "kc", "ks", "vs", "oc",
                                       "cand_score", "cand_idx", "sel", "o_spec", "lse_spec",
-                                      "total")] + [("n_split", c_i32)]
+                                      "total")] + [("n_split", c_i32), ("best", c_size), ("order", c_size)]
 
 
 FORWARD_STEPS = ("pool", "compressed_attn", "block_scores", "topk_merge", "kept_attn", "selected_gate")
@@ -95,6 +96,8 @@ SIGNATURES = {
     "gsa_noalloc_check_device_error": [c_vp],
     "gsa_check_device_error": [c_vp, c_vp],
     "gsa_status_string": [c_i32],
+    "gsa_last_cuda_error": [],
+    "gsa_cuda_error_name": [c_i32],
 }
 
 _lib = None
@@ -111,7 +114,7 @@ def load() -> ctypes.CDLL:
         for name, args in SIGNATURES.items():
             fn = getattr(lib, name)
             fn.argtypes = args
-            fn.restype = ctypes.c_char_p if name == "gsa_status_string" else ctypes.c_int
+            fn.restype = ctypes.c_char_p if name in ("gsa_status_string", "gsa_cuda_error_name") else ctypes.c_int
         _lib = lib
     return _lib
 
@@ -119,7 +122,11 @@ def load() -> ctypes.CDLL:
 class GsaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        text = load().gsa_status_string(status).decode()
+        lib = load()
+        text = lib.gsa_status_string(status).decode()
+        if status == 4:  # GSA_ERR_CUDA: name the CUDA error behind it
+            code = lib.gsa_last_cuda_error()
+            text += f": {lib.gsa_cuda_error_name(code).decode()} ({code})"
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({text})")
 
 

@@ -34,10 +34,12 @@ class Shape:
     top_k: int = 16
     scale: float = 0.0
     keep: int = 0  # 0: every special token always kept; 1: frame 0 + camera tokens
+    wait_limit_ns: int = 0  # 0: default in-kernel wait limit (about 2 s); tiny values test the timeout path
 
     def c(self) -> GsaShape:
         return GsaShape(self.n_frames, self.n_special, self.hp, self.wp, self.n_heads,
-                        self.head_dim, self.pool, self.top_k, float(self.scale), self.keep)
+                        self.head_dim, self.pool, self.top_k, float(self.scale), self.keep,
+                        self.wait_limit_ns)
 
     @staticmethod
     def of(workload) -> "Shape":
@@ -271,6 +273,7 @@ def workspace_view(ws, shape, name: str) -> torch.Tensor:
         "cand_score": (F32, (H, z.Tc, o.n_split, K)), "cand_idx": (I32, (H, z.Tc, o.n_split, K)),
         "sel": (I32, (H, z.Tc, K)),
         "o_spec": (F32, (z.T if z.NK else 0, H, D)), "lse_spec": (F32, (z.T if z.NK else 0, H)),
+        "best": (I32, (H, z.Tc)), "order": (I32, (H * z.Tc,)),
     }[name]
     dtype, shp = spec
     n = 1

@@ -19,6 +19,7 @@ struct Dims {
   long long B0;      // first top-K candidate block (Bf when frame 0 is kept whole)
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
+  long long wait_cycles;  // limit of the in-kernel waits of one role on another
 };
 
 // Bits of the device error word (first word of every workspace).

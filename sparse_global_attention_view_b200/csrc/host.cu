@@ -25,6 +25,7 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
     return GSA_ERR_INVALID_ARG;
   if (s->keep != GSA_KEEP_SPECIALS && s->keep != GSA_KEEP_REFERENCE) return GSA_ERR_INVALID_ARG;
   if (!(s->scale >= 0.f) || isinf(s->scale)) return GSA_ERR_INVALID_ARG;
+  if (s->wait_limit_ns < 0) return GSA_ERR_INVALID_ARG;
   if (s->head_dim != gsa::kHeadDim || s->pool > gsa::kMaxPool || s->top_k > gsa::kMaxTopK ||
       s->n_heads > 128)
     return GSA_ERR_UNSUPPORTED;
@@ -61,6 +62,8 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
   t.NS = NS;
   t.scale = s->scale > 0.f ? s->scale : 1.f / sqrtf((float)s->head_dim);
   t.scale_log2 = t.scale * 1.4426950408889634f;
+  // SM clocks stay below 2 GHz: two cycles per nanosecond is at least the time asked
+  t.wait_cycles = s->wait_limit_ns > 0 ? 2LL * s->wait_limit_ns : 4000000000LL;
   if (d) *d = t;
   if (z) {
     z->T = T;
@@ -84,6 +87,8 @@ constexpr int kMaxCandidates = 2048;  // n_split * K per row in the merge
 // K in (64, 128]: the fused kernel runs twice (top 64, then the next K - 64
 // below the first pass's 64th-best key) and the two selections are merged.
 bool two_pass(const Dims& d) { return d.K > gsa::kFusedTopK && d.K <= 2 * gsa::kFusedTopK; }
+// gsa_forward ranks on the fused tensor-core kernel (one or two passes)
+bool fused_path(const Dims& d) { return gsa::compressed_tc_supported(d) || two_pass(d); }
 
 int forward_splits(const Dims& d) {
   if (gsa::compressed_tc_supported(d) || two_pass(d)) return 1;
@@ -98,7 +103,8 @@ int forward_splits(const Dims& d) {
 }
 
 struct Layout {
-  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cs, ci, sel, ospec, lspec, sel_a, sel_b, root, total;
+  size_t qc32, kc32, vc, qc, kc, ks, vs, oc, cs, ci, sel, ospec, lspec, sel_a, sel_b, root, best, order,
+      counts, total;
   int n_split;
 };
 
@@ -136,6 +142,12 @@ Layout forward_layout(const Dims& d) {
   l.sel_a = take(rows2 * gsa::kFusedTopK * 4);
   l.sel_b = take(rows2 * gsa::kFusedTopK * 4);
   l.root = take(rows2 * 8);
+  // the processing order of the selection branch (fused paths): each row's
+  // best block, the (head, entry) pairs sorted by its position, the buckets
+  const size_t rows_o = fused ? (size_t)d.H * d.Tc : 0;
+  l.best = take(rows_o * 4);
+  l.order = take(rows_o * 4);
+  l.counts = take(fused ? ((size_t)d.H * d.Bf + 1) * 4 : 0);
   l.total = o;
   return l;
 }
@@ -159,6 +171,10 @@ const char* gsa_status_string(gsa_status s) {
   }
   return "unknown status";
 }
+
+int32_t gsa_last_cuda_error(void) { return (int32_t)cudaPeekAtLastError(); }
+
+const char* gsa_cuda_error_name(int32_t code) { return cudaGetErrorName((cudaError_t)code); }
 
 gsa_status gsa_derive(const gsa_shape* shape, gsa_sizes* out) {
   if (out == nullptr) return GSA_ERR_INVALID_ARG;
@@ -254,10 +270,10 @@ gsa_status gsa_selected_attn(const gsa_shape* shape, const gsa_bf16* q, const gs
       !opt_ptr(lse) || !dev_ptr(ws))
     return GSA_ERR_INVALID_ARG;
   if (d.NK > 0 && (!dev_ptr(ks) || !dev_ptr(vs))) return GSA_ERR_INVALID_ARG;
-  return cuda_status(gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v,
-                                          (const bf16*)ks, (const bf16*)vs, sel, nullptr, nullptr,
-                                          nullptr, (bf16*)o_sel, lse, nullptr, nullptr,
-                                          (unsigned*)ws, as_stream(stream)));
+  return cuda_status(gsa::launch_selected_tc(d, (const bf16*)q, (const bf16*)k, (const bf16*)v,
+                                             (const bf16*)ks, (const bf16*)vs, sel, nullptr, nullptr,
+                                             nullptr, nullptr, (bf16*)o_sel, lse, nullptr, nullptr,
+                                             (unsigned*)ws, as_stream(stream)));
 }
 
 gsa_status gsa_gate_combine(const gsa_shape* shape, const float* qc32, const float* w,
@@ -293,6 +309,7 @@ gsa_status dense_global_attn(const gsa_shape* shape, const gsa_bf16* q, const gs
   a.err = (unsigned*)ws;
   a.kv_head_major = 0;
   a.seg_len = 0;
+  a.wait_cycles = d.wait_cycles;
   return cuda_status(gsa::launch_attn_tc(a, (const bf16*)q, (const bf16*)k, (const bf16*)v, d.T,
                                          as_stream(stream)));
 }
@@ -317,6 +334,7 @@ gsa_status frame_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16*
   a.err = (unsigned*)ws;
   a.kv_head_major = 0;
   a.seg_len = d.L;
+  a.wait_cycles = d.wait_cycles;
   return cuda_status(gsa::launch_attn_tc(a, (const bf16*)q, (const bf16*)k, (const bf16*)v, d.T,
                                          as_stream(stream)));
 }
@@ -428,6 +446,8 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
   float* cs = (float*)(base + l.cs);
   int* ci = (int*)(base + l.ci);
   int* sel = (int*)(base + l.sel);
+  int* best = (fused_path(d)) ? (int*)(base + l.best) : nullptr;
+  int* order = (fused_path(d)) ? (int*)(base + l.order) : nullptr;
   cudaStream_t s = as_stream(stream);
   int launched = 0;
   auto mark = [&](int i) -> bool {
@@ -435,6 +455,11 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
   };
   auto step = [&](cudaError_t e, int i) -> bool {
     ++launched;
+    return e == cudaSuccess && mark(i);
+  };
+  // the ordering of the selection branch's work: three kernels
+  auto step3 = [&](cudaError_t e, int i) -> bool {
+    launched += 3;
     return e == cudaSuccess && mark(i);
   };
   if (!mark(0)) return GSA_ERR_CUDA;
@@ -457,6 +482,7 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
     unsigned long long* root = (unsigned long long*)(base + l.root);
     gsa::CmpPass first, second;
     first.root = root;
+    first.best = best;
     second.ub = root;
     second.scores_only = 1;
     if (!step(gsa::launch_compressed_tc(d64, qc32, kc32, vc, oc, nullptr, nullptr, sel_a, (unsigned*)ws, s,
@@ -465,14 +491,19 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
         !step(gsa::launch_compressed_tc(drest, qc32, kc32, vc, oc, nullptr, nullptr, sel_b, (unsigned*)ws, s,
                                         second),
               3) ||
-        !step(gsa::launch_selection_union(d, sel_a, gsa::kFusedTopK, sel_b, drest.K, sel, s), 4))
+        gsa::launch_selection_union(d, sel_a, gsa::kFusedTopK, sel_b, drest.K, sel, s) != cudaSuccess ||
+        !step3(gsa::launch_selection_order(d, best, (int*)(base + l.counts), order, s), 4))
       return GSA_ERR_CUDA;
+    ++launched;  // the union
   } else if (fused) {
-    // steps 1-3 in one kernel (its heaps hold each row's final top-K, written
-    // to sel in ascending order); the intervals of steps 2 and 3 stay empty
-    if (!step(gsa::launch_compressed_tc(d, qc32, kc32, vc, oc, nullptr, nullptr, sel, (unsigned*)ws, s),
+    // steps 1-3 in one kernel (its lists hold each row's final top-K, written
+    // to sel in ascending order); step 3's interval holds the ordering of the
+    // selection branch's work
+    gsa::CmpPass cp;
+    cp.best = best;
+    if (!step(gsa::launch_compressed_tc(d, qc32, kc32, vc, oc, nullptr, nullptr, sel, (unsigned*)ws, s, cp),
               2) ||
-        !mark(3) || !mark(4))
+        !mark(3) || !step3(gsa::launch_selection_order(d, best, (int*)(base + l.counts), order, s), 4))
       return GSA_ERR_CUDA;
   } else {
     gsa::AttnArgs a;
@@ -515,12 +546,13 @@ gsa_status gsa_forward_timed(const gsa_shape* shape, const gsa_bf16* q, const gs
     a.err = (unsigned*)ws;
     a.kv_head_major = 1;
     a.seg_len = 0;
+    a.wait_cycles = d.wait_cycles;
     if (!step(gsa::launch_attn_tc(a, (const bf16*)q, ks, vs, d.NK, s), 5)) return GSA_ERR_CUDA;
   } else if (!mark(5)) {
     return GSA_ERR_CUDA;
   }
-  if (!step(gsa::launch_selected(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, ks, vs, sel, qc32,
-                                 w, oc, (bf16*)out, nullptr, ospec, lspec, (unsigned*)ws, s),
+  if (!step(gsa::launch_selected_tc(d, (const bf16*)q, (const bf16*)k, (const bf16*)v, ks, vs, sel, order,
+                                    qc32, w, oc, (bf16*)out, nullptr, ospec, lspec, (unsigned*)ws, s),
             6))
     return GSA_ERR_CUDA;
   if (n_launched) *n_launched = launched;
@@ -554,6 +586,8 @@ gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out) {
   out->lse_spec = l.lspec;
   out->total = l.total;
   out->n_split = l.n_split;
+  out->best = l.best;
+  out->order = l.order;
   return GSA_OK;
 }
 

@@ -48,6 +48,7 @@ struct AttnTcArgs {
   int kv_head_major;
   long long seg_len;   // > 0: attention within consecutive segments of this many tokens
   long long seg_ctas;  // set by the launcher
+  long long wait_cycles;  // limit of the in-kernel waits of one role on another
 };
 cudaError_t launch_attn_tc(const AttnTcArgs& a, const bf16* q, const bf16* k, const bf16* v,
                            long long kv_rows, cudaStream_t st);
@@ -58,18 +59,25 @@ bool make_tmap_3d(CUtensorMap* m, bool fp32, const void* base, unsigned long lon
                   unsigned long long d1, unsigned long long d2, unsigned long long s1,
                   unsigned long long s2, unsigned b0, unsigned b1, unsigned b2);
 
+// Tiled map of rank <= 5 over bf16 data (128-byte swizzle); dims and box
+// innermost first, rank - 1 strides in bytes.  False if the driver refuses it.
+bool make_tmap(CUtensorMap* m, const void* base, int rank, const unsigned long long* dims,
+               const unsigned long long* strides, const unsigned* box);
+
 // Compressed attention on tcgen05 fused with the S_guide streaming top-K
 // (one candidate list per row, i.e. n_split = 1); needs K <= 64.  Writes the
 // candidate lists when cand_score/cand_idx are non-null and the final
 // selection (ascending ids, -1 padding) when sel is non-null.
-// A second launch ranks the next K pairs: with `ub` set, only (score, id)
-// keys strictly below ub[h*Tc + row] are candidates; `root` (nullable)
-// receives each row's K-th best key (0 when fewer than K candidates exist);
-// `scores_only` skips the attention (no V, P, PV or oc).
+// A second launch ranks the next K pairs: with `ub` set, only pairs whose key
+// (score bits, then the complement of the compressed entry index: a larger
+// key is a better pair) is strictly below ub[h*Tc + row] are candidates;
+// `root` (nullable) receives each row's K-th best key (0 when fewer than K
+// candidates exist); `scores_only` skips the attention (no V, P, PV or oc).
 struct CmpPass {
   const unsigned long long* ub = nullptr;
   unsigned long long* root = nullptr;
   int scores_only = 0;
+  int* best = nullptr;  // nullable [H][Tc]: each row's best-scoring block id (-1 if none)
 };
 bool compressed_tc_supported(const Dims& d);
 constexpr int kFusedTopK = 64;  // heap capacity of one pass of the fused kernel
@@ -96,6 +104,25 @@ cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const b
                             const float* w, const float* oc, bf16* out, float* lse,
                             const float* o_spec, const float* lse_spec, unsigned* err,
                             cudaStream_t st);
+
+// Selection branch on tcgen05 (transposed products per compressed entry).
+// With o_spec/lse_spec the always-kept segment comes from them; otherwise,
+// when NK > 0, the kernel streams the kept keys ks/vs itself.  `order`
+// (nullable, H*Tc entries of h*Tc + a) is the order in which (head, entry)
+// pairs are processed.  With `w` non-null the gate is fused and `out`
+// receives g*oc + (1-g)*o_sel; otherwise o_sel (and lse if non-null).
+cudaError_t launch_selected_tc(const Dims& d, const bf16* q, const bf16* k, const bf16* v,
+                               const bf16* ks, const bf16* vs, const int* sel, const int* order,
+                               const float* qc32, const float* w, const float* oc, bf16* out,
+                               float* lse, const float* o_spec, const float* lse_spec, unsigned* err,
+                               cudaStream_t st);
+
+// Processing order of the (head, entry) pairs for the selection branch:
+// grouped by head and by the grid position (id mod Bh*Bw) of each pair's
+// best-scoring block, so pairs whose selections cover the same region of
+// every frame run at the same time and share their K/V blocks in L2.
+// `counts` holds H * Bf + 1 ints of scratch; order receives H * Tc ints.
+cudaError_t launch_selection_order(const Dims& d, const int* best, int* counts, int* order, cudaStream_t st);
 
 // Subsampled global attention (AVGGT SGA): sizes and the five launches.
 struct SgaSizes {

@@ -1,0 +1,675 @@
+// Step 5 (and, fused, step 6) on the 5th-generation tensor cores: the
+// selection branch (Speed3R technical summary 2.1, selection branch: fine
+// attention over the selected regions only; 2.2, Speed3R-VGGT: the reference
+// frame / camera tokens are always kept).
+//
+// The <= 16 fine queries of one compressed entry (query block) share one key
+// set, so the products run transposed, with the keys on the 128-row M side and
+// the entry's queries as N = 16:
+//   S^T  = K_sel Q^T               M = 128 keys (8 selected blocks x 16 slots), K = 64
+//   O^T += [V_sel | 1]^T P^T       M = 128: the 64 value dims, then 64 rows of
+//                                  ones whose results are the sums of P per query
+// so P never leaves the softmax thread's lane except as the B operand, and the
+// row sums come out of the tensor core with exactly the bf16 weights of the
+// numerator.  A selected P x P block (P <= 4) is one TMA box of 4 x 4 patches
+// over a per-frame view of the token grid (dims: 64 values, head, column, row,
+// frame): 16 rows of 128 bytes, patches outside the grid read as zero.
+//
+// One CTA works through (head, entry) pairs; 12 warps:
+//   warp 0      TMA producer: per entry its queries (one box) and selection,
+//               then per 128-key tile the 8 blocks' K and V (two boxes each),
+//               into a 2-stage ring; when the always-kept tokens are not
+//               supplied as a finished softmax state, their head-major copies
+//               are streamed first as plain 128-key tiles;
+//   warp 1      MMA issuer (one thread): S^T(t+1) is issued before O^T(t), so
+//               the tensor core works while the softmax handles a tile;
+//   warp 2      TMEM allocation (S^T at columns 0/16, O^T at 32/48);
+//   warps 4-7   softmax, one thread per key lane (16 queries per thread);
+//   warps 8-11  epilogue of the previous entry (normalise, merge with the
+//               always-kept segment, gate, store) while the softmax works on
+//               the next one.
+// The softmax shifts every query by a fixed reference: the always-kept
+// segment's log-sum-exp when it is supplied (so that segment's normalised
+// output enters with weight 1), else the first tile's maximum.  A tile whose
+// scores exceed the reference by 2^8 raises it for its queries and rescales
+// their partial sums (rare; one barrier with an OR reduction per tile decides
+// it for all 128 key lanes).  Every mbarrier wait is bounded as in the other
+// tensor-core kernels.
+#include <math_constants.h>
+#include <stddef.h>
+
+#include "internal.h"
+#include "tc_common.cuh"
+
+namespace gsa {
+namespace {
+
+using namespace tc;
+
+constexpr int NQ = 16;           // query slots per entry (P * P <= 16)
+constexpr int TKEYS = 128;       // keys per tile
+constexpr int BPT = 8;           // selected blocks per tile
+constexpr int ST = 2;            // K/V ring stages
+constexpr int NE = 2;            // entry slots (queries, selection, O^T buffer)
+constexpr int kThreads = 384;
+constexpr uint32_t kKV = 16384;  // one [128][64] bf16 tile
+constexpr uint32_t kQ = 2048;    // one [16][64] bf16 query tile
+constexpr uint32_t kPT = 4096;   // one [16][128] bf16 P^T tile (two 64-key atoms)
+
+struct Entry {
+  int h, a;
+  int n_tiles, n_kept;  // tiles in all; the first n_kept stream the always-kept keys
+  int nsel;             // valid ids in sel
+  uint32_t qmask;       // query slots that hold a token
+  int tok[NQ];          // token of each query slot
+  float m0[NQ];         // initial reference (log2 units of the scaled logit)
+  float mf[NQ], wf[NQ]; // final reference and weight of the always-kept segment
+  int sel[kMaxTopK];
+};
+
+constexpr uint32_t OFF_K = 0;
+constexpr uint32_t OFF_V = OFF_K + ST * kKV;
+constexpr uint32_t OFF_ONES = OFF_V + ST * kKV;
+constexpr uint32_t OFF_Q = OFF_ONES + kKV;
+constexpr uint32_t OFF_PT = OFF_Q + NE * kQ;
+constexpr uint32_t OFF_ENT = OFF_PT + 2 * kPT;
+constexpr uint32_t kEntBytes = (sizeof(Entry) + 127) / 128 * 128;
+constexpr uint32_t OFF_RED = OFF_ENT + NE * kEntBytes;   // [4 warps][16] per-query partial maxima
+constexpr uint32_t OFF_LS = OFF_RED + 4 * NQ * 4;        // [16] sums of P (epilogue)
+constexpr uint32_t OFF_GATE = OFF_LS + NQ * 4;           // [2] gate partial dot products
+constexpr uint32_t OFF_BAR = (OFF_GATE + 16 + 255) / 256 * 256;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;
+constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
+static_assert(OFF_Q % 1024 == 0 && OFF_PT % 1024 == 0 && OFF_ONES % 1024 == 0, "operand alignment");
+static_assert(2 * kSmemBytes <= 232448, "two CTAs per SM");
+
+// barriers
+constexpr int B_EF = 0, B_EE = B_EF + NE, B_EM = B_EE + NE, B_KF = B_EM + NE, B_VF = B_KF + ST,
+              B_KE = B_VF + ST, B_VE = B_KE + ST, B_SF = B_VE + ST, B_PF = B_SF + 2, B_PE = B_PF + 2,
+              B_OF = B_PE + 2, B_OD = B_OF + NE, B_DRAIN = B_OD + 1, B_COUNT = B_DRAIN + 1;
+static_assert(B_COUNT * 8 <= 256, "barrier area");
+
+constexpr uint32_t kCols = 64;  // TMEM: S^T at 0 / 16, O^T at 32 / 48
+constexpr uint32_t TM_S = 0, TM_O = 32;
+// Register split: launched with kLaunchRegs per thread (two CTAs per SM); the
+// producer / MMA warpgroup and the epilogue give registers to the softmax.
+// The shares must not exceed the launch allocation, or the increase would wait
+// forever: the host refuses to launch unless the compiled kernel uses exactly
+// kLaunchRegs registers per thread.
+constexpr int kLaunchRegs = 80, kRegsLow = 48, kRegsSoft = 120, kRegsEpi = 72;
+static_assert(128 * (kRegsLow + kRegsSoft + kRegsEpi) <= kThreads * kLaunchRegs, "register split");
+
+__device__ __forceinline__ uint32_t pt_addr(uint32_t base, int q, int k) {
+  // [16 queries][128 keys] bf16, K-major, 128-byte swizzle: keys 0-63 and
+  // 64-127 in two 2 KB atoms of 16 rows
+  const int kk = k & 63;
+  return base + (uint32_t)((k >> 6) * 2048 + (q >> 3) * 1024 + (q & 7) * 128 +
+                           ((((kk >> 3) ^ (q & 7))) << 4) + (kk & 7) * 2);
+}
+__device__ __forceinline__ void sts_u16(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared.u16 [%0], %1;\n" ::"r"(addr), "h"((unsigned short)v) : "memory");
+}
+// Barrier over the 128 threads of one warpgroup (named barrier `id`) that also
+// returns whether `pred` held for any of them.
+__device__ __forceinline__ bool bar_or(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, 128, p;\n"
+      " selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void bar_sync128(int id) {
+  asm volatile("bar.sync %0, 128;\n" ::"r"(id) : "memory");
+}
+
+// Top-left patch (column, row within the frame grid) and frame of block beta,
+// and how many of its P x P patches exist in each direction.
+struct Blk {
+  int f, c0, r0, nr, nc;
+};
+__device__ __forceinline__ Blk block_of(const Dims& d, int beta) {
+  Blk b;
+  b.f = beta / d.Bf;
+  const int j = beta - b.f * d.Bf;
+  const int br = j / d.Bw, bc = j - br * d.Bw;
+  b.r0 = br * d.P;
+  b.c0 = bc * d.P;
+  b.nr = min(d.P, d.Hp - b.r0);
+  b.nc = min(d.P, d.Wp - b.c0);
+  return b;
+}
+
+struct Maps {
+  CUtensorMap q5, k5, v5;  // per-frame grid views, box 4 x 4 patches of one head
+  CUtensorMap q3;          // [T][H][64], box one token of one head (special entries)
+  CUtensorMap ks, vs;      // [H][NK][64] kept copies, box 128 keys (kept keys streamed inline)
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+    selected_tc_kernel(const __grid_constant__ Maps mp, const Dims d, const int* __restrict__ sel,
+                       const int* __restrict__ order, const float* __restrict__ qc32,
+                       const float* __restrict__ w, const float* __restrict__ oc, bf16* __restrict__ out,
+                       float* __restrict__ lse, const float* __restrict__ o_spec,
+                       const float* __restrict__ lse_spec, unsigned* err, int kept_inline) {
+  extern __shared__ __align__(1024) uint8_t st_smem_raw[];
+  const uint32_t raw = smem_u32(st_smem_raw);
+  const uint32_t sb = (raw + 1023u) & ~1023u;
+  uint8_t* sp = st_smem_raw + (sb - raw);
+  auto bar = [&](int i) -> uint32_t { return sb + OFF_BAR + 8u * i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sp + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sp + OFF_MISC + 4);
+  auto ent = [&](int s) -> Entry& { return *reinterpret_cast<Entry*>(sp + OFF_ENT + s * kEntBytes); };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long n_items = (long long)d.H * d.Tc;
+  const int n_kept_tiles = kept_inline ? (int)((d.NK + TKEYS - 1) / TKEYS) : 0;
+
+  if (tid == 0) {
+    for (int s = 0; s < NE; ++s) {
+      mbar_init(bar(B_EF + s), 1);
+      mbar_init(bar(B_EE + s), 128);
+      mbar_init(bar(B_EM + s), 1);
+      mbar_init(bar(B_OF + s), 1);
+    }
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(bar(B_KF + s), 1);
+      mbar_init(bar(B_VF + s), 1);
+      mbar_init(bar(B_KE + s), 1);
+      mbar_init(bar(B_VE + s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_SF + b), 1);
+      mbar_init(bar(B_PF + b), 128);
+      mbar_init(bar(B_PE + b), 1);
+    }
+    mbar_init(bar(B_OD), 1);
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  {
+    // the ones rows of the value operand, and zeroed query tiles (slots a
+    // special entry leaves unused must hold finite values)
+    uint4* ones = reinterpret_cast<uint4*>(sp + OFF_ONES);
+    for (int i = tid; i < (int)(kKV / 16); i += kThreads)
+      ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+    uint4* qz = reinterpret_cast<uint4*>(sp + OFF_Q);
+    for (int i = tid; i < (int)(NE * kQ / 16); i += kThreads) qz[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), kCols);
+    tmem_relinquish();
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tbase = *tmem_slot;
+
+  if (warp < 4) regs_dec<kRegsLow>();
+  if (warp == 0) {
+    // ---------------- TMA producer (the whole warp) ----------------
+    if (lane == 0) {
+      prefetch_tmap(&mp.q5);
+      prefetch_tmap(&mp.k5);
+      prefetch_tmap(&mp.v5);
+      prefetch_tmap(&mp.q3);
+    }
+    int gt = 0;  // tiles loaded
+    int ne = 0;  // entries loaded
+    bool ok = true;
+    for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
+      const int es = ne % NE;
+      if (ne >= NE && !__all_sync(0xffffffffu, mbar_wait(bar(B_EE + es), ((ne / NE) - 1) & 1, abort_flag, err, d.wait_cycles))) {
+        ok = false;
+        break;
+      }
+      const long long pair = order != nullptr ? (long long)order[it] : it;
+      const int h = (int)(pair / d.Tc);
+      const int a = (int)(pair - (long long)h * d.Tc);
+      Entry& E = ent(es);
+      // the selection: ascending ids, -1 padded; an id outside [0, NB) ends the
+      // list and raises the device-check bit instead of being dereferenced
+      const int* sl = sel + ((long long)h * d.Tc + a) * d.K;
+      int nsel = d.K;
+      for (int k0 = 0; k0 < d.K; k0 += 32) {
+        const int k = k0 + lane;
+        const int id = k < d.K ? sl[k] : -1;
+        if (k < d.K) E.sel[k] = id;
+        const unsigned bad = __ballot_sync(0xffffffffu, k < d.K && (id < 0 || id >= d.NB));
+        const unsigned oob = __ballot_sync(0xffffffffu, k < d.K && id >= d.NB);
+        if (oob != 0 && lane == 0) atomicOr(err, kErrDeviceCheck);
+        if (bad != 0 && nsel == d.K) nsel = k0 + __ffs(bad) - 1;
+      }
+      // the entry's queries
+      const int f = a / d.E, j = a - (a / d.E) * d.E;
+      const bool special = j < d.S;
+      Blk qb;
+      if (!special) qb = block_of(d, f * d.Bf + (j - d.S));
+      if (lane < NQ) {
+        const int pr = lane >> 2, pc = lane & 3;
+        bool valid;
+        long long t;
+        if (special) {
+          valid = lane == 0;
+          t = (long long)f * d.L + j;
+        } else {
+          valid = pr < qb.nr && pc < qb.nc;
+          t = (long long)f * d.L + d.S + (long long)(qb.r0 + pr) * d.Wp + qb.c0 + pc;
+        }
+        E.tok[lane] = valid ? (int)t : -1;
+        float m0 = -CUDART_INF_F;
+        if (valid && lse_spec != nullptr) m0 = lse_spec[t * d.H + h] * 1.4426950408889634f;
+        E.m0[lane] = m0;
+      }
+      const unsigned qm = __ballot_sync(0xffffffffu, lane < NQ && (special ? lane == 0 : ((lane >> 2) < qb.nr && (lane & 3) < qb.nc)));
+      if (lane == 0) {
+        E.h = h;
+        E.a = a;
+        E.nsel = nsel;
+        E.n_kept = n_kept_tiles;
+        E.n_tiles = n_kept_tiles + (nsel + BPT - 1) / BPT;
+        E.qmask = qm & 0xffffu;
+      }
+      const int n_tiles = n_kept_tiles + (nsel + BPT - 1) / BPT;
+      __syncwarp();
+      if (lane == 0) {
+        // the one arrival on the entry's barrier (arrive.expect_tx, release: it
+        // also publishes the info the warp wrote above); the phase completes
+        // once the query box has landed
+        const uint32_t dq = sb + OFF_Q + es * kQ;
+        if (special) {
+          mbar_expect_tx(bar(B_EF + es), 128);
+          tma_load_3d(dq, &mp.q3, bar(B_EF + es), 0, h, f * d.L + j);
+        } else {
+          mbar_expect_tx(bar(B_EF + es), kQ);
+          tma_load_5d(dq, &mp.q5, bar(B_EF + es), 0, h, qb.c0, qb.r0, f);
+        }
+      }
+      // the key tiles
+      for (int i = 0; ok && i < n_tiles; ++i, ++gt) {
+        const int s = gt % ST;
+        if (gt >= ST) {
+          const uint32_t ph = ((gt / ST) - 1) & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(bar(B_KE + s), ph, abort_flag, err, d.wait_cycles) &&
+                                          mbar_wait(bar(B_VE + s), ph, abort_flag, err, d.wait_cycles))) {
+            ok = false;
+            break;
+          }
+        }
+        if (lane == 0) {
+          mbar_expect_tx(bar(B_KF + s), kKV);
+          mbar_expect_tx(bar(B_VF + s), kKV);
+        }
+        __syncwarp();
+        const uint32_t dk = sb + OFF_K + s * kKV, dv = sb + OFF_V + s * kKV;
+        if (i < n_kept_tiles) {
+          if (lane == 0) {
+            tma_load_3d(dk, &mp.ks, bar(B_KF + s), 0, i * TKEYS, h);
+            tma_load_3d(dv, &mp.vs, bar(B_VF + s), 0, i * TKEYS, h);
+          }
+        } else if (lane < BPT) {
+          const int idx = (i - n_kept_tiles) * BPT + lane;
+          // past the list: any block, fully masked by the softmax
+          const Blk kb = block_of(d, idx < nsel ? E.sel[idx] : 0);
+          tma_load_5d(dk + lane * 2048, &mp.k5, bar(B_KF + s), 0, h, kb.c0, kb.r0, kb.f);
+          tma_load_5d(dv + lane * 2048, &mp.v5, bar(B_VF + s), 0, h, kb.c0, kb.r0, kb.f);
+        }
+      }
+    }
+    if (*abort_flag && lane == 0) {
+      // let this CTA's own copies land before its shared memory goes away
+      volatile int never = 0;
+      for (int e = ne - 1; e >= 0 && e >= ne - NE; --e) mbar_wait(bar(B_EF + e % NE), (e / NE) & 1, &never, err);
+      for (int g = gt - 1; g >= 0 && g >= gt - ST; --g) {
+        mbar_wait(bar(B_KF + g % ST), (g / ST) & 1, &never, err);
+        mbar_wait(bar(B_VF + g % ST), (g / ST) & 1, &never, err);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t id_s = idesc(128, 16, kFmtBF16, 0, 0);
+      const uint32_t id_o = idesc(128, 16, kFmtBF16, 1, 0);
+      int gt = 0, ne = 0;
+      bool ok = true;
+      // the tile whose O^T product is still to be issued
+      bool pend = false;
+      int p_s = 0, p_b = 0, p_es = 0;
+      bool p_first = false, p_last = false;
+      auto finish = [&]() -> bool {
+        const int g = gt - 1;  // the pending tile's global index
+        if (!mbar_wait(bar(B_VF + p_s), (g / ST) & 1, abort_flag, err, d.wait_cycles) ||
+            !mbar_wait(bar(B_PF + p_b), (g >> 1) & 1, abort_flag, err, d.wait_cycles))
+          return false;
+        fence_after_sync();
+        const uint32_t sv = sb + OFF_V + p_s * kKV;
+        const uint32_t lbo = (sb + OFF_ONES) - sv;  // value dims, then the ones rows
+        const uint32_t spt = sb + OFF_PT + p_b * kPT;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ss(tbase + TM_O + p_es * 16, sdesc(sv + kk * 2048, lbo, 1024),
+                      sdesc_k(spt + (kk >> 2) * 2048 + (kk & 3) * 32), id_o, (!p_first || kk > 0) ? 1u : 0u);
+        mma_commit(bar(B_VE + p_s));
+        mma_commit(bar(B_PE + p_b));
+        mma_commit(bar(B_OD));
+        if (p_last) mma_commit(bar(B_OF + p_es));
+        pend = false;
+        return true;
+      };
+      for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
+        const int es = ne % NE;
+        if (!mbar_wait(bar(B_EF + es), (ne / NE) & 1, abort_flag, err, d.wait_cycles)) {
+          ok = false;
+          break;
+        }
+        const int n = ent(es).n_tiles;
+        if (n == 0) {
+          if (pend && !(ok = finish())) break;
+          mma_commit(bar(B_OF + es));  // nothing to add: the epilogue may start
+          continue;
+        }
+        const uint32_t sq = sb + OFF_Q + es * kQ;
+        for (int i = 0; i < n; ++i) {
+          const int s = gt % ST, b = gt & 1;
+          if (!mbar_wait(bar(B_KF + s), (gt / ST) & 1, abort_flag, err, d.wait_cycles)) {
+            ok = false;
+            break;
+          }
+          fence_after_sync();
+          const uint32_t sk = sb + OFF_K + s * kKV;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_bf16_ss(tbase + TM_S + b * 16, sdesc_k(sk + kk * 32), sdesc_k(sq + kk * 32), id_s, kk > 0);
+          mma_commit(bar(B_SF + b));
+          mma_commit(bar(B_KE + s));
+          ++gt;
+          if (pend && !(ok = finish())) break;
+          pend = true;
+          p_s = s;
+          p_b = b;
+          p_es = es;
+          p_first = i == 0;
+          p_last = i == n - 1;
+        }
+      }
+      if (ok && pend) ok = finish();
+      if (!ok) {
+        volatile int never = 0;
+        mma_commit(bar(B_DRAIN));
+        mbar_wait(bar(B_DRAIN), 0, &never, err);
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    regs_inc<kRegsSoft>();
+    // ---------------- softmax, one thread per key lane ----------------
+    const int q4 = warp & 3;
+    const int k = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float c2 = d.scale_log2;
+    float* red = reinterpret_cast<float*>(sp + OFF_RED);
+    int gt = 0, ne = 0;
+    bool ok = true;
+    for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
+      const int es = ne % NE;
+      // every wait's outcome is agreed on by the whole warpgroup (bar.red), so
+      // the 128 threads always reach the same named barriers
+      if (bar_or(1, !mbar_wait(bar(B_EF + es), (ne / NE) & 1, abort_flag, err, d.wait_cycles))) {
+        ok = false;
+        break;
+      }
+      const Entry& E = ent(es);
+      const int n = E.n_tiles, nk = E.n_kept, nsel = E.nsel;
+      const uint32_t qmask = E.qmask;
+      // reference per query; the weight of the always-kept segment (1 when
+      // its normalised state is supplied, scaled down with every raise of the
+      // reference) is kept in the entry by one thread
+      float m[NQ];
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) m[q] = E.m0[q];
+      Entry& Ew = ent(es);
+      if (tid == 128) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) Ew.wf[q] = (lse_spec != nullptr && ((qmask >> q) & 1u)) ? 1.f : 0.f;
+      }
+      for (int i = 0; i < n; ++i, ++gt) {
+        const int b = gt & 1;
+        // is this lane's key a real key of the tile?
+        bool kvalid;
+        if (i < nk) {
+          kvalid = (long long)i * TKEYS + k < d.NK;
+        } else {
+          const int idx = (i - nk) * BPT + (k >> 4);
+          kvalid = false;
+          if (idx < nsel) {
+            const Blk kb = block_of(d, E.sel[idx]);
+            const int slot = k & 15;
+            kvalid = (slot >> 2) < kb.nr && (slot & 3) < kb.nc;
+          }
+        }
+        if (bar_or(1, !mbar_wait(bar(B_SF + b), (gt >> 1) & 1, abort_flag, err, d.wait_cycles))) {
+          ok = false;
+          break;
+        }
+        fence_after_sync();
+        uint32_t sv[NQ];
+        tmem_ld16(tbase + lane_off + TM_S + b * 16, sv);
+        tmem_wait_ld();
+        float x[NQ];
+        float xmax = -CUDART_INF_F;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const bool use = kvalid && ((qmask >> q) & 1u);
+          x[q] = use ? fmaf(__uint_as_float(sv[q]), c2, -m[q]) : -CUDART_INF_F;
+          xmax = fmaxf(xmax, x[q]);
+        }
+        // a score above its query's reference by 2^8 (or a query without one
+        // yet): raise the references of this tile's queries to their maxima
+        if (bar_or(1, xmax > 8.f)) {
+          float tm[NQ];
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            float v = (kvalid && ((qmask >> q) & 1u)) ? __uint_as_float(sv[q]) * c2 : -CUDART_INF_F;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+            tm[q] = v;
+          }
+          if (lane < NQ) {
+            float v = tm[0];
+#pragma unroll
+            for (int q = 1; q < NQ; ++q)
+              if (lane == q) v = tm[q];
+            red[q4 * NQ + lane] = v;
+          }
+          bar_sync128(1);
+          float corr[NQ];
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const float t = fmaxf(fmaxf(red[q], red[NQ + q]), fmaxf(red[2 * NQ + q], red[3 * NQ + q]));
+            const float mn = fmaxf(m[q], t);
+            corr[q] = mn == -CUDART_INF_F ? 1.f : exp2f(m[q] - mn);
+            m[q] = mn;
+            if (tid == 128) Ew.wf[q] *= corr[q];
+          }
+          bar_sync128(1);  // red is reused by the next tile
+          if (i > 0) {
+            // this entry's partial O^T (and sums) must be complete, then rescaled
+            if (bar_or(1, !mbar_wait(bar(B_OD), (gt - 1) & 1, abort_flag, err, d.wait_cycles))) {
+              ok = false;
+              break;
+            }
+            fence_after_sync();
+            uint32_t ov[NQ];
+            tmem_ld16(tbase + lane_off + TM_O + es * 16, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) ov[q] = __float_as_uint(__uint_as_float(ov[q]) * corr[q]);
+            tmem_st16(tbase + lane_off + TM_O + es * 16, ov);
+            tmem_wait_st();
+          }
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const bool use = kvalid && ((qmask >> q) & 1u);
+            x[q] = use ? fmaf(__uint_as_float(sv[q]), c2, -m[q]) : -CUDART_INF_F;
+          }
+        }
+        uint32_t pk[NQ / 2];
+#pragma unroll
+        for (int u = 0; u < NQ / 2; ++u) pk[u] = exp2_bf16x2(x[2 * u], x[2 * u + 1]);
+        // P^T buffer b is free once the O^T product of tile gt - 2 is complete
+        if (bar_or(1, gt >= 2 && !mbar_wait(bar(B_PE + b), ((gt >> 1) - 1) & 1, abort_flag, err, d.wait_cycles))) {
+          ok = false;
+          break;
+        }
+        const uint32_t spt = sb + OFF_PT + b * kPT;
+#pragma unroll
+        for (int u = 0; u < NQ / 2; ++u) {
+          sts_u16(pt_addr(spt, 2 * u, k), pk[u] & 0xffffu);
+          sts_u16(pt_addr(spt, 2 * u + 1, k), pk[u] >> 16);
+        }
+        fence_proxy_async_smem();
+        fence_before_sync();
+        mbar_arrive(bar(B_PF + b));
+      }
+      if (!ok) break;
+      if (tid == 128) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) Ew.mf[q] = m[q];
+        mbar_arrive(bar(B_EM + es));
+      }
+    }
+  } else if (warp >= 8) {
+    regs_dec<kRegsEpi>();
+    // ---------------- epilogue, one thread per TMEM lane ----------------
+    const int q4 = warp & 3;
+    const int dlane = q4 * 32 + lane;  // lanes 0-63: value dims; 64-127: sums of P
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float* ls = reinterpret_cast<float*>(sp + OFF_LS);
+    float* gz = reinterpret_cast<float*>(sp + OFF_GATE);
+    const long long row = (long long)d.H * kHeadDim;
+    int ne = 0;
+    bool ok = true;
+    for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
+      const int es = ne % NE;
+      const uint32_t ph = (ne / NE) & 1;
+      const bool got = mbar_wait(bar(B_EF + es), ph, abort_flag, err, d.wait_cycles) &&
+                       mbar_wait(bar(B_EM + es), ph, abort_flag, err, d.wait_cycles) &&
+                       mbar_wait(bar(B_OF + es), ph, abort_flag, err, d.wait_cycles);
+      if (bar_or(2, !got)) {  // agreed on by all four epilogue warps
+        ok = false;
+        break;
+      }
+      fence_after_sync();
+      const Entry& E = ent(es);
+      const int h = E.h, a = E.a;
+      const uint32_t qmask = E.qmask;
+      uint32_t ov[NQ];
+      if (E.n_tiles > 0) {
+        tmem_ld16(tbase + lane_off + TM_O + es * 16, ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) ov[q] = 0u;
+      }
+      if (dlane == 64) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) ls[q] = __uint_as_float(ov[q]);
+      }
+      float g = 0.f;
+      if (w != nullptr && dlane < 64) {
+        float z = qc32[((long long)a * d.H + h) * kHeadDim + dlane] * w[(long long)h * kHeadDim + dlane];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+        if (lane == 0) gz[q4] = z;
+      }
+      bar_sync128(2);
+      if (dlane < 64) {
+        if (w != nullptr) g = 1.f / (1.f + expf(-(gz[0] + gz[1])));
+        const float* oca = oc != nullptr ? oc + ((long long)a * d.H + h) * kHeadDim : nullptr;
+        const float cmp = (w != nullptr) ? oca[dlane] : 0.f;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          if (!((qmask >> q) & 1u)) continue;
+          const long long t = E.tok[q];
+          const float wq = E.wf[q];
+          const float den = wq + ls[q];
+          float num = __uint_as_float(ov[q]);
+          if (o_spec != nullptr) num = fmaf(wq, o_spec[(t * d.H + h) * kHeadDim + dlane], num);
+          const float o = num / den;
+          const long long ob = t * row + (long long)h * kHeadDim + dlane;
+          if (w != nullptr) {
+            out[ob] = __float2bfloat16_rn(g * cmp + (1.f - g) * o);
+          } else {
+            out[ob] = __float2bfloat16_rn(o);
+            if (lse != nullptr && dlane == 0) lse[t * d.H + h] = (E.mf[q] + log2f(den)) * 0.6931471805599453f;
+          }
+        }
+      }
+      bar_sync128(2);  // ls / gz are reused by the next entry
+      fence_before_sync();
+      mbar_arrive(bar(B_EE + es));
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 2) {
+    fence_after_sync();
+    tmem_dealloc(tbase, kCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_selected_tc(const Dims& d, const bf16* q, const bf16* k, const bf16* v,
+                               const bf16* ks, const bf16* vs, const int* sel, const int* order,
+                               const float* qc32, const float* w, const float* oc, bf16* out,
+                               float* lse, const float* o_spec, const float* lse_spec, unsigned* err,
+                               cudaStream_t st) {
+  const unsigned long long H = (unsigned long long)d.H;
+  const unsigned long long rowb = H * 128;  // bytes per token row
+  Maps mp;
+  // per-frame grid view of [T][H][64] starting at the first patch of frame 0:
+  // (value, head, column, row, frame) with strides (2, 128, rowb, Wp rowb, L rowb)
+  const unsigned long long dims5[5] = {64, H, (unsigned long long)d.Wp, (unsigned long long)d.Hp,
+                                       (unsigned long long)d.N};
+  const unsigned long long str5[4] = {128, rowb, (unsigned long long)d.Wp * rowb, (unsigned long long)d.L * rowb};
+  const unsigned box5[5] = {64, 1, 4, 4, 1};
+  const long long off = (long long)d.S * d.H * kHeadDim;
+  bool ok = make_tmap(&mp.q5, q + off, 5, dims5, str5, box5) && make_tmap(&mp.k5, k + off, 5, dims5, str5, box5) &&
+            make_tmap(&mp.v5, v + off, 5, dims5, str5, box5);
+  const unsigned long long dims3[3] = {64, H, (unsigned long long)d.T};
+  const unsigned long long str3[2] = {128, rowb};
+  const unsigned box3[3] = {64, 1, 1};
+  ok = ok && make_tmap(&mp.q3, q, 3, dims3, str3, box3);
+  const int kept_inline = (o_spec == nullptr && d.NK > 0) ? 1 : 0;
+  if (kept_inline) {
+    const unsigned long long dk[3] = {64, (unsigned long long)d.NK, H};
+    const unsigned long long sk[2] = {128, (unsigned long long)d.NK * 128};
+    const unsigned bk[3] = {64, 128, 1};
+    ok = ok && make_tmap(&mp.ks, ks, 3, dk, sk, bk) && make_tmap(&mp.vs, vs, 3, dk, sk, bk);
+  } else {
+    mp.ks = mp.q3;
+    mp.vs = mp.q3;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(selected_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, selected_tc_kernel);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long items = (long long)d.H * d.Tc;
+  const long long grid = items < 2LL * sms ? items : 2LL * sms;
+  if (grid <= 0) return cudaSuccess;
+  selected_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mp, d, sel, order, qc32, w, oc, out, lse,
+                                                                  o_spec, lse_spec, err, kept_inline);
+  return cudaGetLastError();
+}
+
+}  // namespace gsa

@@ -217,6 +217,7 @@ cudaError_t launch_sga(const Dims& d, int sub_h, int sub_w, const bf16* q, const
   a.err = err;
   a.kv_head_major = 1;
   a.seg_len = 0;
+  a.wait_cycles = d.wait_cycles;
   e = launch_attn_tc(a, q, ks, vs, z.NK, st);
   if (e != cudaSuccess) return e;
   ++*launched;

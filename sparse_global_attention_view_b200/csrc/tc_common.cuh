@@ -11,8 +11,11 @@
 namespace gsa {
 namespace tc {
 
-// A wait gives up after this many SM clock cycles (about 2 s at 1.9 GHz),
-// sets kErrTimeout in the error word and raises the CTA's abort flag.
+// A wait gives up after this many SM clock cycles by default (about 2 s at
+// 1.9 GHz), sets kErrTimeout in the error word and raises the CTA's abort
+// flag.  gsa_shape.wait_limit_ns shortens the waits of the pipeline roles on
+// one another; the drain waits of an aborting CTA (its own copies and
+// products in flight) always keep this default.
 constexpr long long kWaitCycles = 4000000000LL;
 
 // ---------------------------------------------------------------------------
@@ -24,6 +27,8 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 __device__ __forceinline__ void fence_mbar_init() {
   asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
 }
+// Arrive on `bar` (one of its arrivals) and add `bytes` to the transaction
+// count its current phase waits for.
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
                : "memory");
@@ -46,13 +51,13 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
 // (without completing) when the CTA's abort flag is raised or the wait runs
 // out of time; a timeout also records kErrTimeout and raises the flag.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned* err) {
+                                          unsigned* err, long long limit = kWaitCycles) {
   if (mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_test(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(err, kErrTimeout);
       *abort_flag = 1;
       return false;
@@ -69,6 +74,15 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
       "%4, %5}], [%2];\n" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0,
+                                            int c1, int c2, int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5, %6, %7}], [%2];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
       : "memory");
 }
 
@@ -201,6 +215,54 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
                    bar)
                : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// softmax arithmetic
+
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
+}
+__device__ __forceinline__ unsigned long long pack_f32x2(float lo, float hi) {
+  unsigned long long x;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(lo), "f"(hi));
+  return x;
+}
+// exp2 of two fp32 values, rounded to bf16 and exponentiated two at a time
+// (one special-function instruction for the pair): the packed pair of
+// attention weights (lo in the low half), bf16 like the PV operand they feed.
+__device__ __forceinline__ uint32_t exp2_bf16x2(float lo, float hi) {
+  uint32_t b, e;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(b) : "f"(hi), "f"(lo));
+  asm("ex2.approx.ftz.bf16x2 %0, %1;\n" : "=r"(e) : "r"(b));
+  return e;
+}
+// The same for two raw fp32 scores (bit patterns) scaled and shifted first,
+// x * c + n, as one packed f32x2 FMA.
+__device__ __forceinline__ uint32_t exp2_bf16x2_fma(uint32_t lo, uint32_t hi, unsigned long long c2,
+                                                    unsigned long long n2) {
+  unsigned long long x, y;
+  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "r"(lo), "r"(hi));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(y) : "l"(x), "l"(c2), "l"(n2));
+  uint32_t ylo, yhi, b, e;
+  asm("mov.b64 {%0, %1}, %2;\n" : "=r"(ylo), "=r"(yhi) : "l"(y));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(b) : "r"(yhi), "r"(ylo));
+  asm("ex2.approx.ftz.bf16x2 %0, %1;\n" : "=r"(e) : "r"(b));
+  return e;
+}
+// Generic-proxy writes to shared memory that the tensor core reads next.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+// 16 x 128 bf16 ones: the B operand of a P 1 product (the row sums of P).
+constexpr uint32_t kOnesBytes = 4096;
+__device__ __forceinline__ void fill_ones(uint8_t* p, uint32_t bytes, int tid, int nthreads) {
+  uint4* o = reinterpret_cast<uint4*>(p);
+  for (int i = tid; i < (int)(bytes / 16); i += nthreads)
+    o[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
 }
 
 }  // namespace tc

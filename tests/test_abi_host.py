@@ -195,6 +195,13 @@ def test_noalloc_limit_falls_between_four_and_five_vggt_frames(lib):
     assert workspace_size(shape(n_frames=5, top_k=16)) > NOALLOC_SCRATCH_BYTES
 
 
+def test_negative_wait_limit_is_rejected(lib):
+    import dataclasses
+    s = dataclasses.replace(shape(), wait_limit_ns=-1)
+    n = ctypes.c_size_t()
+    assert lib.gsa_workspace_size(ctypes.byref(s.c()), ctypes.byref(n)) == 1
+
+
 def test_status_strings(lib):
     for code in range(8):
         assert lib.gsa_status_string(code)

@@ -152,8 +152,11 @@ gsa_status gsa_pool_kv(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16
  * n_split in [1, 64], n_split * K <= 2048.  With n_split == 1 and K <= 64 this
  * runs the fused tcgen05 kernel (scores from tf32 products of qc32 / kc32,
  * the list of each row being its exact top-K); otherwise warp-level bf16
- * attention from qc / kc and an fp32 scorer over the slices.  Blocks below
- * B0 are never candidates.
+ * attention from qc / kc and an fp32 scorer over the slices -- an inspection
+ * path for per-slice candidate lists, many times slower at large N.  For
+ * 64 < K <= 128 gsa_forward ranks on the tensor cores in two passes (see
+ * gsa_forward_timed) and is the path to use.  Blocks below B0 are never
+ * candidates.
  */
 gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const gsa_bf16* kc,
                                const gsa_bf16* vc, const float* qc32, const float* kc32,
@@ -179,6 +182,11 @@ gsa_status gsa_topk_blocks(const gsa_shape* shape, const float* cand_score,
  * NULL when NK == 0):
  *   o_sel [T][H][64] bf16, and lse [T][H] fp32 = log sum exp of the scaled
  *   logits (may be NULL).
+ * Runs on tcgen05, one (entry, head) pair at a time with the entry's queries
+ * as the N = 16 side; this stage call streams the NK always-kept keys for
+ * every pair as well, whereas gsa_forward computes that segment once for all
+ * tokens on the M = 128 attention kernel and passes its softmax state on.
+ * An id outside [0, NB) ends the pair's list and sets the device-check bit.
  */
 gsa_status gsa_selected_attn(const gsa_shape* shape, const gsa_bf16* q, const gsa_bf16* k,
                              const gsa_bf16* v, const gsa_bf16* ks, const gsa_bf16* vs,

@@ -45,6 +45,9 @@ Where the pages are silent, the readings used here are:
   * one softmax scale 1/sqrt(D) for every attention;
   * the gate is g = sigmoid(q_mean . w_h) per (query block, head); g weights
     the compression branch and (1 - g) the selection branch.
+The other readings of two of these points are available as variants of
+``gsa_layer``: fine queries against the pooled keys in the compression
+branch (``queries="fine"``) and a gate per fine token (``gate_per="token"``).
 
 Inputs are torch tensors (bf16 or fp32, CPU) or NumPy arrays of shape
 [T, H, D]; they are read in slices and converted exactly to float64, so the
@@ -526,8 +529,24 @@ def combine(g_rows: np.ndarray, o_cmp_up: np.ndarray, o_sel: np.ndarray) -> np.n
 # the whole layer
 
 
+def compressed_attention_fine(geo: Geometry, Q, Kc: np.ndarray, Vc: np.ndarray, rows) -> np.ndarray:
+    """Reading A1 of the compression branch, as a variant: each fine query
+    attends to the pooled keys and values (no pooling of the queries, so no
+    up-sampling of the output).  [len(rows), H, D]."""
+    q = f64(Q, np.asarray(rows, dtype=np.int64))
+    return weighted_values(softmax(qk_logits(q, Kc, geo.sm_scale), axis=-1), Vc)
+
+
+def gate_token(geo: Geometry, Q, rows, w) -> np.ndarray:
+    """Reading A10 of the gate, as a variant: g = sigmoid(q_t . w_h) for every
+    fine token t (the it page's per-token wording taken literally) instead of
+    one gate per query block from the pooled query.  [len(rows), H]."""
+    return gate(geo, f64(Q, np.asarray(rows, dtype=np.int64)), w)
+
+
 def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
-              tie_window: float = 1e-3, chunk_elems: int | None = None, pooled=None) -> dict:
+              tie_window: float = 1e-3, chunk_elems: int | None = None, pooled=None,
+              queries: str = "pooled", gate_per: str = "block") -> dict:
     """The GSA layer for fine query tokens ``rows`` (all tokens when None).
 
     Returns a dict of float64 arrays:
@@ -544,7 +563,11 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     (no unchosen block beats a chosen one by ``tie_window`` or more).
 
     ``pooled`` = (pool(Q), pool(K), pool(V)) from an earlier call on the same
-    inputs skips recomputing step 1.  Steps 2-4 run over the entries in
+    inputs skips recomputing step 1.  ``queries="fine"`` and ``gate_per="token"``
+    evaluate the variant readings A1 (fine queries against the pooled keys in
+    the compression branch; the selection still ranks by the pooled scores)
+    and A10 (a gate per fine token); the defaults are the readings the CUDA
+    path implements.  Steps 2-4 run over the entries in
     chunks whose logits hold about ``chunk_elems`` values
     (``CHUNKS.layer_chunk_elems``).
     """
@@ -589,9 +612,11 @@ def gsa_layer(geo: Geometry, Q, K, V, w, rows=None, sel_override=None,
     g = gate(geo, Qc[entries], w)
     pos = {int(a): i for i, a in enumerate(entries)}
     own = np.array([pos[geo.entry_of_token(int(t))] for t in rows], dtype=np.int64)
-    out = combine(g[own], o_cmp[own], o_sel)
+    o_cmp_up = o_cmp[own] if queries == "pooled" else compressed_attention_fine(geo, Q, Kc_keys, Vc_keys, rows)
+    g_rows = g[own] if gate_per == "block" else gate_token(geo, Q, rows, w)
+    out = combine(g_rows, o_cmp_up, o_sel)
     res = dict(rows=rows, entries=entries, own=own, o_cmp=o_cmp, sel=sel, gap=gap,
-               o_sel=o_sel, g=g, out=out, o_cmp_up=o_cmp[own])
+               o_sel=o_sel, g=g, out=out, o_cmp_up=o_cmp_up, g_rows=g_rows)
     if other is not None:
         res.update(sel_exact=sel_exact, sel_valid=sel_valid)
     if keep_guide:

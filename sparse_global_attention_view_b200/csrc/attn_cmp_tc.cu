@@ -49,6 +49,12 @@ namespace {
 
 using namespace tc;
 
+// Of every 8 pairs of attention weights, this many are computed on the FMA
+// pipe (exp2_bf16x2_poly) and the rest on the special-function unit.
+#ifndef GSA_CMP_POLY_OF_8
+#define GSA_CMP_POLY_OF_8 0
+#endif
+
 constexpr int TQ = 128;
 constexpr int TK = 128;
 constexpr int ST = 2;
@@ -385,7 +391,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = exp2_bf16x2_fma(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2);
+        for (int i = 0; i < 16; ++i)
+          pk[i] = (i & 7) < GSA_CMP_POLY_OF_8 ? exp2_bf16x2_poly(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2)
+                                              : exp2_bf16x2_fma(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2);
         tmem_st16(p_addr + 16 * c, pk);
       }
       tmem_wait_st();

@@ -35,6 +35,13 @@ namespace {
 
 using namespace tc;
 
+// Of every 8 pairs of attention weights, this many are computed on the FMA
+// pipe (exp2_bf16x2_poly) and the rest on the special-function unit: at
+// head dim 64 the exponentials, not the tensor core, bound the softmax.
+#ifndef GSA_ATTN_POLY_OF_8
+#define GSA_ATTN_POLY_OF_8 0
+#endif
+
 constexpr int TQ = 128;            // rows per query tile
 constexpr int NQT = 2;             // query tiles per CTA
 constexpr int TK = 128;            // keys per key tile
@@ -281,7 +288,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = exp2_bf16x2_fma(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2);
+        for (int i = 0; i < 16; ++i)
+          pk[i] = (i & 7) < GSA_ATTN_POLY_OF_8 ? exp2_bf16x2_poly(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2)
+                                               : exp2_bf16x2_fma(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2);
         tmem_st16(s_addr + 16 * c, pk);
       }
       tmem_wait_st();

@@ -450,25 +450,34 @@ __global__ void __launch_bounds__(kThreads, 2)
             kvalid = (slot >> 2) < kb.nr && (slot & 3) < kb.nc;
           }
         }
-        if (bar_or(1, !mbar_wait(bar(B_SF + b), (gt >> 1) & 1, abort_flag, err, d.wait_cycles))) {
-          ok = false;
-          break;
-        }
+        // P^T buffer b is free once the O^T product of tile gt - 2 is complete;
+        // S^T(gt) is in TMEM once its product is.  Both waits and the test for
+        // a raise of the references are decided together by one OR barrier in
+        // the common case.
+        bool waited = gt < 2 || mbar_wait(bar(B_PE + b), ((gt >> 1) - 1) & 1, abort_flag, err, d.wait_cycles);
+        waited = waited && mbar_wait(bar(B_SF + b), (gt >> 1) & 1, abort_flag, err, d.wait_cycles);
+        waited = __all_sync(0xffffffffu, waited);  // tcgen05.ld below is warp-collective
         fence_after_sync();
         uint32_t sv[NQ];
-        tmem_ld16(tbase + lane_off + TM_S + b * 16, sv);
-        tmem_wait_ld();
         float x[NQ];
         float xmax = -CUDART_INF_F;
+        if (waited) {
+          tmem_ld16(tbase + lane_off + TM_S + b * 16, sv);
+          tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const bool use = kvalid && ((qmask >> q) & 1u);
-          x[q] = use ? fmaf(__uint_as_float(sv[q]), c2, -m[q]) : -CUDART_INF_F;
-          xmax = fmaxf(xmax, x[q]);
+          for (int q = 0; q < NQ; ++q) {
+            const bool use = kvalid && ((qmask >> q) & 1u);
+            x[q] = use ? fmaf(__uint_as_float(sv[q]), c2, -m[q]) : -CUDART_INF_F;
+            xmax = fmaxf(xmax, x[q]);
+          }
         }
         // a score above its query's reference by 2^8 (or a query without one
         // yet): raise the references of this tile's queries to their maxima
-        if (bar_or(1, xmax > 8.f)) {
+        if (bar_or(1, !waited || xmax > 8.f)) {
+          if (bar_or(1, !waited)) {
+            ok = false;
+            break;
+          }
           float tm[NQ];
 #pragma unroll
           for (int q = 0; q < NQ; ++q) {
@@ -519,11 +528,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         uint32_t pk[NQ / 2];
 #pragma unroll
         for (int u = 0; u < NQ / 2; ++u) pk[u] = exp2_bf16x2(x[2 * u], x[2 * u + 1]);
-        // P^T buffer b is free once the O^T product of tile gt - 2 is complete
-        if (bar_or(1, gt >= 2 && !mbar_wait(bar(B_PE + b), ((gt >> 1) - 1) & 1, abort_flag, err, d.wait_cycles))) {
-          ok = false;
-          break;
-        }
         const uint32_t spt = sb + OFF_PT + b * kPT;
 #pragma unroll
         for (int u = 0; u < NQ / 2; ++u) {

@@ -408,6 +408,33 @@ def pin_split_sga():
               what=f"split sga {sh}x{sw} brute force")
 
 
+def pin_variant_readings():
+    """The variant readings A1 (fine queries in the compression branch) and A10
+    (a gate per fine token): at P = 1 both equal the default layer; the fine
+    compression branch is torch's SDPA of the fine queries over the pooled keys
+    and values; a per-token gate is 1/2 for w = 0 and saturates with the sign
+    of q_t . w."""
+    geo1, x1 = micro(N=2, S=1, Hp=3, Wp=5, H=2, D=8, P=1, K=4)
+    base = O.gsa_layer(geo1, x1.q, x1.k, x1.v, x1.w)
+    var = O.gsa_layer(geo1, x1.q, x1.k, x1.v, x1.w, queries="fine", gate_per="token")
+    close(var["out"], base["out"], what="variants at P = 1")
+    geo, x = micro(N=2, S=2, Hp=6, Wp=7, H=2, D=8, P=4, K=3)
+    res = O.gsa_layer(geo, x.q, x.k, x.v, x.w, queries="fine")
+    Kc, Vc = O.pool(geo, x.k), O.pool(geo, x.v)
+    t = lambda z: torch.as_tensor(z, dtype=torch.float64).permute(1, 0, 2).unsqueeze(0)  # noqa: E731
+    want = torch.nn.functional.scaled_dot_product_attention(t(x.q.double().numpy()), t(Kc), t(Vc))
+    close(res["o_cmp_up"], want.squeeze(0).permute(1, 0, 2).numpy(), what="fine queries vs sdpa over pooled keys")
+    zero = O.gsa_layer(geo, x.q, x.k, x.v, torch.zeros_like(x.w), gate_per="token")
+    close(zero["g_rows"], np.full(zero["g_rows"].shape, 0.5), what="token gate, w = 0")
+    big = torch.zeros_like(x.w)
+    big[:, 0] = 1000.0
+    q = x.q.clone()
+    q[..., 0] = torch.where(q[..., 0] >= 0, q[..., 0].abs() + 1, -(q[..., 0].abs() + 1))  # |q_t . w| >= 1000
+    sat = O.gsa_layer(geo, q, x.k, x.v, big, gate_per="token")
+    sign = (q[:, :, 0].double().numpy() > 0).astype(np.float64)
+    close(sat["g_rows"], sign, tol=1e-9, what="token gate saturates with sign(q_t . w)")
+
+
 def all_pins(fixture_path):
     return {
         "block_structure": lambda: pin_block_structure(fixture_path),
@@ -433,4 +460,5 @@ def all_pins(fixture_path):
         "split_layer": pin_split_layer,
         "split_dense": pin_split_dense,
         "split_sga": pin_split_sga,
+        "variant_readings": pin_variant_readings,
     }

@@ -162,6 +162,21 @@ def _gate_wrong_sign(geo, Qc_rows, w):
     return 1.0 - _orig["gate"](geo, Qc_rows, w)
 
 
+def _fine_queries_against_fine_keys(geo, Q, Kc, Vc, rows):
+    # the A1 variant attending to the unpooled keys and values instead
+    r = np.asarray(rows, dtype=np.int64)
+    q = O.f64(Q, r)
+    return O.weighted_values(O.softmax(O.qk_logits(q, O.f64(Q, np.arange(geo.T)), geo.sm_scale)),
+                             O.f64(Q, np.arange(geo.T)))
+
+
+def _token_gate_from_pooled_query(geo, Q, rows, w):
+    # the A10 variant falling back to the pooled query of the token's block
+    r = np.asarray(rows, dtype=np.int64)
+    qc = O.pool(geo, Q)
+    return O.gate(geo, qc[[geo.entry_of_token(int(t)) for t in r]], w)
+
+
 def _softmax_torch_wrong_axis(z, axis=-1):
     # the threaded (large-array) form normalises over the first axis
     z = np.asarray(z, dtype=np.float64)
@@ -213,6 +228,8 @@ MUTATIONS = {
     "reference keep keeps every register token": ("Geometry.kept_tokens", _kept_all_specials_of_later_frames),
     "reference keep takes the camera from the last slot": ("Geometry.kept_tokens", _kept_camera_from_last_slot),
     "threaded softmax over the wrong axis": ("softmax", _softmax_torch_wrong_axis),
+    "fine-query variant attends to fine keys": ("compressed_attention_fine", _fine_queries_against_fine_keys),
+    "per-token gate variant uses the pooled query": ("gate_token", _token_gate_from_pooled_query),
 }
 # every split loop of the oracle, with each boundary mistake
 for _fn in ("pool", "gsa_layer", "dense_attention", "sga_attention"):

@@ -347,7 +347,10 @@ gsa_status gsa_forward_noalloc(const gsa_shape* shape, const gsa_bf16* q, const 
 gsa_status gsa_noalloc_check_device_error(void* stream);
 
 /* Synchronise `stream`, read the device error word in `ws`, clear it, and
- * return GSA_OK, GSA_ERR_TIMEOUT or GSA_ERR_DEVICE_CHECK. */
+ * return GSA_OK, GSA_ERR_TIMEOUT or GSA_ERR_DEVICE_CHECK.  For diagnosis, the
+ * header's words 1 and 2 record the first in-kernel wait that ran out (its
+ * barrier's shared-memory address | 1, and threadIdx.x << 8 | phase parity);
+ * they are cleared with the error word. */
 gsa_status gsa_check_device_error(void* ws, void* stream);
 
 /* Static text for a status code. */

@@ -285,7 +285,17 @@ def workspace_view(ws, shape, name: str) -> torch.Tensor:
 
 
 def check_device_error(ws, stream=None) -> None:
-    check(load().gsa_check_device_error(_ws(ws), _stream(stream)), "gsa_check_device_error")
+    """Raise GsaError if a kernel set the workspace's error word (then cleared).
+    A timeout's message carries where the first wait ran out (header words 1-2:
+    the barrier's shared-memory address | 1, threadIdx.x << 8 | parity)."""
+    p = _ws(ws)
+    where = ""
+    st = torch.cuda.current_stream() if stream is None else stream
+    st.synchronize()
+    hdr = ws[:12].view(torch.int32).cpu().tolist() if ws.numel() >= 12 else []
+    if hdr and hdr[1] != 0:
+        where = f" (first wait out: barrier smem 0x{hdr[1] & ~1:x}, thread {hdr[2] >> 8}, parity {hdr[2] & 255})"
+    check(load().gsa_check_device_error(p, _stream(stream)), "gsa_check_device_error" + where)
 
 
 class GsaLayer:

@@ -557,18 +557,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) cm |= (__uint_as_float(g[i]) > tau ? 1u : 0u) << i;
         }
         cm &= (cv[q >> 1] >> ((q & 1) * 16)) & 0xffffu;
-        if (!__any_sync(FULL, cm != 0)) continue;
+        // the columns where any row of the warp has a candidate: usually one
+        // or two, so the append below skips the others with a uniform branch
+        const uint32_t cu = __reduce_or_sync(FULL, cm);
+        if (cu == 0) continue;
         const unsigned over = __ballot_sync(FULL, nb + __popc(cm) > kBuf);
         if (over != 0) merge_rows(over);
         const uint32_t lo0 = 0x7fffffffu - (uint32_t)(e0 + 16 * q);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          if (cm & (1u << i)) {
-            const unsigned long long key =
-                ((unsigned long long)order_bits(__uint_as_float(g[i])) << 32) | (lo0 - (uint32_t)i);
-            if (key < ub) {
-              sts_u64(buf_s + (uint32_t)(nb * TQ + (r ^ nb)) * 8u, key);
-              ++nb;
+          if (cu & (1u << i)) {
+            if (cm & (1u << i)) {
+              const unsigned long long key =
+                  ((unsigned long long)order_bits(__uint_as_float(g[i])) << 32) | (lo0 - (uint32_t)i);
+              if (key < ub) {
+                sts_u64(buf_s + (uint32_t)(nb * TQ + (r ^ nb)) * 8u, key);
+                ++nb;
+              }
             }
           }
         }

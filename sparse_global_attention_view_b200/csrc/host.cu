@@ -598,7 +598,7 @@ gsa_status gsa_check_device_error(void* ws, void* stream) {
   if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return GSA_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return GSA_ERR_CUDA;
-  if (word != 0 && cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return GSA_ERR_CUDA;
+  if (word != 0 && cudaMemsetAsync(ws, 0, 3 * sizeof(word), s) != cudaSuccess) return GSA_ERR_CUDA;
   if (word & gsa::kErrTimeout) return GSA_ERR_TIMEOUT;
   if (word & gsa::kErrDeviceCheck) return GSA_ERR_DEVICE_CHECK;
   return GSA_OK;

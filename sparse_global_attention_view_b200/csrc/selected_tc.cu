@@ -338,10 +338,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       bool ok = true;
       // the tile whose O^T product is still to be issued
       bool pend = false;
-      int p_s = 0, p_b = 0, p_es = 0;
+      int p_g = 0, p_s = 0, p_b = 0, p_es = 0;  // the pending tile: global index, stage, buffer, entry slot
       bool p_first = false, p_last = false;
       auto finish = [&]() -> bool {
-        const int g = gt - 1;  // the pending tile's global index
+        const int g = p_g;
         if (!mbar_wait(bar(B_VF + p_s), (g / ST) & 1, abort_flag, err, d.wait_cycles) ||
             !mbar_wait(bar(B_PF + p_b), (g >> 1) & 1, abort_flag, err, d.wait_cycles))
           return false;
@@ -386,9 +386,9 @@ __global__ void __launch_bounds__(kThreads, 2)
             mma_bf16_ss(tbase + TM_S + b * 16, sdesc_k(sk + kk * 32), sdesc_k(sq + kk * 32), id_s, kk > 0);
           mma_commit(bar(B_SF + b));
           mma_commit(bar(B_KE + s));
-          ++gt;
           if (pend && !(ok = finish())) break;
           pend = true;
+          p_g = gt++;
           p_s = s;
           p_b = b;
           p_es = es;

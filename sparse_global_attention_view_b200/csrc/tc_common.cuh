@@ -59,6 +59,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (*abort_flag) return false;
     if (clock64() - t0 > limit) {
       atomicOr(err, kErrTimeout);
+      // the first wait to run out records where it was: the barrier's shared
+      // memory address (| 1, never 0) and the thread and phase parity
+      if (atomicCAS(err + 1, 0u, bar | 1u) == 0u) err[2] = (threadIdx.x << 8) | parity;
       *abort_flag = 1;
       return false;
     }

@@ -10,35 +10,30 @@
 //               stage refilled once its PV product is complete;
 //   warp 1      MMA issuer: S = Qc Kc^T with kind::tf32 from the fp32 means
 //               (the top-K ranking needs better than bf16 scores), into one of
-//               two TMEM score buffers, then O += P Vc and l += P 1 (bf16, P
-//               from TMEM; the row sums of P come from the tensor core as the
-//               product with a block of ones, so they sum exactly the bf16
-//               weights the numerator uses);
-//   warp 2      TMEM allocation (S at columns 0/128, O at 256, P at 320/384,
-//               l at 448);
+//               two TMEM score buffers, then O += P Vc (bf16, P from TMEM);
+//   warp 2      TMEM allocation (S at columns 0/128, O at 256, P at 320/384);
 //   warps 4-7   softmax, one thread per query row;
 //   warps 8-11  streaming top-K, one thread per query row.
 // S(j+1) is computed while both warpgroups work on S(j): the softmax writes
 // P(j) to its own TMEM columns, so the raw scores stay readable until the
-// top-K warpgroup is done with them.  The softmax forms exp2 two at a time
-// (packed f32x2 scaling, bf16x2 exp2: P is bf16 for the PV product anyway).
-// It also forms the maxima of the tile's eight 16-column groups, compares them
-// with each row's current K-th best score (published in shared memory by the
-// top-K thread) and hands the top-K warp an 8-bit mask of the groups that may
-// hold a candidate.  The top-K warp reads from TMEM only the groups flagged
-// for any of its 32 rows and releases the score buffer after its last read.
-// Candidates (columns that beat the row's K-th best, special entries and
-// blocks below B0 excluded) are appended to a per-row buffer in shared
-// memory.  When a row's buffer cannot take the next group, the whole warp
-// merges it into the row's list of best pairs: the buffer is sorted across the
-// 32 lanes by a bitonic network, combined with the sorted list (two entries
-// per lane) by the max of opposite ends, and the result put in order by a
-// bitonic merge -- a few hundred instructions for up to 28 candidates,
-// instead of a heap insertion per candidate.  Pairs are packed 64-bit keys
-// (score bits, then the complement of the entry index), so a larger key is a
-// better pair and equal scores keep the lower entry, i.e. the lower block id.
-// Columns arrive in ascending entry order, so a column whose score equals
-// the K-th best comes after it and is rightly not a candidate.
+// top-K warpgroup is done with them.  The softmax already forms the maxima of
+// the tile's eight 16-column groups; it compares them with each row's current
+// K-th best score (published in shared memory by the top-K thread) and hands
+// the top-K warp an 8-bit mask of the groups that may hold a candidate.  The
+// top-K warp reads from TMEM only the groups flagged for any of its 32 rows
+// and releases the score buffer after its last read, so once the heaps are
+// full most tiles cost it one mask load.  Candidates (columns that beat the
+// row's K-th best) go to a per-row buffer in shared memory; when any row's
+// buffer is half full the warp inserts all buffered candidates in lockstep
+// (one round of insertions serves every row) into the rows' heaps of K best
+// (score, block id) pairs; special entries are never ranked.  Once every heap
+// of the warp is full, a round is one predicated three-level replacement of
+// the root per lane (lanes without a candidate walk it without moving), with
+// the next round's candidate loaded during the current one: no lane diverges.  Columns arrive
+// in ascending block order and only a strictly larger score displaces the
+// root, so equal scores keep the lower id.  The softmax keeps eight
+// independent max and sum chains: one warp per sub-partition runs it, so
+// dependency latency, not throughput, is what it must avoid.
 #include <math_constants.h>
 
 #include "internal.h"
@@ -49,36 +44,26 @@ namespace {
 
 using namespace tc;
 
-// Of every 8 pairs of attention weights, this many are computed on the FMA
-// pipe (exp2_bf16x2_poly) and the rest on the special-function unit.
-#ifndef GSA_CMP_POLY_OF_8
-#define GSA_CMP_POLY_OF_8 0
-#endif
-
 constexpr int TQ = 128;
 constexpr int TK = 128;
 constexpr int ST = 2;
 constexpr int kThreads = 384;
-constexpr int kMaxK = kFusedTopK;  // list capacity per row (two entries per lane)
-constexpr int kBuf = 28;           // candidate buffer slots per row
+constexpr int kMaxK = kFusedTopK;  // heap capacity per row
+constexpr int kBuf = 32;         // candidate buffer entries per row
 constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16) tile: 16 KB
 
-constexpr uint32_t OFF_Q = 0;                          // 2 sub-tiles (d 0-31, 32-63)
-constexpr uint32_t OFF_K = OFF_Q + 2 * kSub;           // ST x 2 sub-tiles
-constexpr uint32_t OFF_V = OFF_K + ST * 2 * kSub;      // ST x bf16 tile
-constexpr uint32_t OFF_ONES = OFF_V + ST * kSub;       // [16][128] bf16 ones: B of the row-sum product
-constexpr uint32_t OFF_LST = OFF_ONES + 4096;          // [128 rows][64] keys, sorted descending
-constexpr uint32_t OFF_BUF = OFF_LST + TQ * kMaxK * 8; // [kBuf slots][128 rows] keys (row ^ slot)
-constexpr uint32_t OFF_BAR = OFF_BUF + kBuf * TQ * 8;
-constexpr uint32_t OFF_TAU = OFF_BAR + 256;            // each row's K-th best score [128]
-constexpr uint32_t OFF_MASK = OFF_TAU + TQ * 4;        // candidate-group masks [2][128] bytes
+constexpr uint32_t OFF_Q = 0;                        // 2 sub-tiles (d 0-31, 32-63)
+constexpr uint32_t OFF_K = OFF_Q + 2 * kSub;         // ST x 2 sub-tiles
+constexpr uint32_t OFF_V = OFF_K + ST * 2 * kSub;    // ST x bf16 tile
+constexpr uint32_t OFF_HS = OFF_V + ST * kSub;       // heap keys [kMaxK][128] (8 bytes)
+constexpr uint32_t OFF_CS = OFF_HS + kMaxK * TQ * 8; // candidate scores [kBuf][128]
+constexpr uint32_t OFF_CC = OFF_CS + kBuf * TQ * 4;  // candidate entry indices
+constexpr uint32_t OFF_BAR = OFF_CC + kBuf * TQ * 4;
+constexpr uint32_t OFF_TAU = OFF_BAR + 256;          // each row's K-th best score [128]
+constexpr uint32_t OFF_MASK = OFF_TAU + TQ * 4;      // candidate-group masks [2][128] bytes
 constexpr uint32_t OFF_MISC = OFF_MASK + 2 * TQ;
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
-static_assert(OFF_ONES % 1024 == 0, "ones tile alignment");
-
-// TMEM columns: S at 0 / 128, O at 256, P at 320 / 384 (bf16 pairs), l at 448
-constexpr uint32_t TM_S = 0, TM_O = 256, TM_P = 320, TM_L = 448;
 
 // KE / VE: a K / V stage is free again (the QK^T resp. PV product that read it
 // is complete); MR: the softmax has published the candidate-group masks of
@@ -96,10 +81,12 @@ constexpr uint32_t kCols = 512;
 constexpr int kLaunchRegs = 168, kRegsLow = 56, kRegsHigh = 224;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= kThreads * kLaunchRegs, "register split");
 
-// A pair's key: the order-preserving bits of the score, then the complement
-// of the compressed entry index (the map entry -> block id is increasing, so
-// ordering by entry is ordering by block id).  0 is below every real key and
-// marks an empty list slot.
+// The K best (score, block id) pairs of one row: a 4-ary min-heap in shared
+// memory of packed 64-bit keys, [slot][row] layout so the 128 rows hit
+// distinct banks.  key = (order-preserving bits of the score) << 32 |
+// (0x7fffffff - id): a larger key is a better pair (higher score, or equal
+// score and lower id), so the root holds the worst pair.  Four children per
+// node keep a sift to 3 levels of 4 independent loads.
 __device__ __forceinline__ uint32_t order_bits(float s) {
   const uint32_t u = __float_as_uint(s);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -107,23 +94,89 @@ __device__ __forceinline__ uint32_t order_bits(float s) {
 __device__ __forceinline__ float order_value(uint32_t o) {
   return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
 }
-__device__ __forceinline__ unsigned long long u64max(unsigned long long a, unsigned long long b) {
-  return a > b ? a : b;
+__device__ __forceinline__ unsigned long long pair_key(float s, int id) {
+  return ((unsigned long long)order_bits(s) << 32) | (uint32_t)(0x7fffffff - id);
 }
-// Compare-exchange with the lane `delta` away (xor): keep the larger key when
-// `keep_max`, else the smaller.
-__device__ __forceinline__ unsigned long long cmpx(unsigned long long x, int delta, bool keep_max) {
-  const unsigned long long o = __shfl_xor_sync(0xffffffffu, x, delta);
-  return (keep_max == (x > o)) ? x : o;
+struct Heap {
+  unsigned long long* hk;
+  int r, K, cnt;
+  float tau;  // score a candidate must beat (-inf until the heap is full)
+
+  __device__ __forceinline__ unsigned long long at(int i) const { return hk[i * TQ + r]; }
+  __device__ __forceinline__ void put(int i, unsigned long long k) { hk[i * TQ + r] = k; }
+  __device__ __forceinline__ void sift(int p, unsigned long long key) {
+    while (true) {
+      const int c0 = 4 * p + 1;
+      if (c0 >= K) break;
+      unsigned long long m = at(c0);
+      int mc = c0;
+#pragma unroll
+      for (int t = 1; t < 4; ++t) {
+        if (c0 + t < K) {
+          const unsigned long long x = at(c0 + t);
+          if (x < m) m = x, mc = c0 + t;
+        }
+      }
+      if (m >= key) break;
+      put(p, m);
+      p = mc;
+    }
+    put(p, key);
+  }
+  // Replace the root (the worst pair) of a full heap by `key` and restore the
+  // heap order: a fixed three levels (K <= 64 pairs fit in 1 + 4 + 16 + 64
+  // slots), the four children of a level loaded together and the descent
+  // predicated rather than branched, so every lane of the warp takes the same
+  // path; the new root is tracked in a register.
+  __device__ __forceinline__ void replace_root(unsigned long long key, bool take = true) {
+    if (!take) key = 0ull;  // a lane without a candidate walks the levels without moving
+    int p = 0;
+    bool go = take;
+    unsigned long long root = key;
+#pragma unroll
+    for (int lvl = 0; lvl < 3; ++lvl) {
+      const int c0 = 4 * p + 1;
+      unsigned long long x[4];
+#pragma unroll
+      for (int t = 0; t < 4; ++t) x[t] = (go && c0 + t < K) ? at(c0 + t) : ~0ull;
+      unsigned long long m = x[0];
+      int mc = c0;
+#pragma unroll
+      for (int t = 1; t < 4; ++t)
+        if (x[t] < m) m = x[t], mc = c0 + t;
+      const bool move = go && m < key;
+      if (move) put(p, m);
+      if (lvl == 0 && move) root = m;
+      p = move ? mc : p;
+      go = move;
+    }
+    if (take) {
+      put(p, key);
+      tau = order_value((uint32_t)(root >> 32));
+    }
+  }
+  __device__ __forceinline__ void push(unsigned long long key) {
+    if (cnt < K) {
+      put(cnt, key);
+      if (++cnt == K) {
+        for (int p = (K - 2) / 4; p >= 0; --p) sift(p, at(p));
+        tau = order_value((uint32_t)(at(0) >> 32));
+      }
+      return;
+    }
+    replace_root(key);
+  }
+  __device__ __forceinline__ int id_of(int i) const { return 0x7fffffff - (int)(uint32_t)at(i); }
+  __device__ __forceinline__ float score_of(int i) const { return order_value((uint32_t)(at(i) >> 32)); }
+};
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
-__device__ __forceinline__ void sts_u64(uint32_t addr, unsigned long long v) {
-  asm volatile("st.shared.u64 [%0], %1;\n" ::"r"(addr), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long lds_u64(uint32_t addr) {
-  unsigned long long v;
-  asm volatile("ld.shared.u64 %0, [%1];\n" : "=l"(v) : "r"(addr) : "memory");
-  return v;
-}
+// Wait for this thread's TMEM loads; the registers are passed through so that
+// no use of them can be scheduled before the wait.
 __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;\n"
                : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
@@ -176,14 +229,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile float* tau_s = reinterpret_cast<volatile float*>(sp + OFF_TAU);
   volatile uint8_t* mask_s = sp + OFF_MASK;
   if (tid < TQ) tau_s[tid] = -CUDART_INF_F;
-  {
-    // the B operand of the row-sum product: 16 x 128 bf16 ones (layout-free)
-    fill_ones(sp + OFF_ONES, kOnesBytes, tid, kThreads);
-    // empty lists: key 0 is below every real pair
-    uint4* lst = reinterpret_cast<uint4*>(sp + OFF_LST);
-    for (int i = tid; i < TQ * kMaxK * 8 / 16; i += kThreads) lst[i] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
-  }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), kCols);
     tmem_relinquish();
@@ -243,13 +288,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_qk = idesc(128, 128, kFmtTF32, 0, 0);
       const uint32_t id_pv = idesc(128, 64, kFmtBF16, 0, 1);
-      const uint32_t id_l = idesc(128, 16, kFmtBF16, 0, 0);
-      const uint32_t sOnes = sb + OFF_ONES;
       auto issue_s = [&](int s, int b) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-          mma_tf32_ss(tbase + TM_S + b * 128, sdesc_k(sQ + off), sdesc_k(sK + 2 * s * kSub + off), id_qk, kk > 0);
+          mma_tf32_ss(tbase + b * 128, sdesc_k(sQ + off), sdesc_k(sK + 2 * s * kSub + off), id_qk, kk > 0);
         }
         mma_commit(bar(B_SF + b));
         mma_commit(bar(B_KE + s));
@@ -278,13 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (cp.scores_only) continue;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tbase + TM_O, tbase + TM_P + b * 64 + kk * 8, sdesc_mn(sV + s * kSub + kk * 2048), id_pv,
+          mma_bf16_ts(tbase + 256, tbase + 320 + b * 64 + kk * 8, sdesc_mn(sV + s * kSub + kk * 2048), id_pv,
                       (j > 0 || kk > 0) ? 1u : 0u);
-        // l += P 1: every column of the 16-wide result holds the row sum
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tbase + TM_L, tbase + TM_P + b * 64 + kk * 8,
-                      sdesc_k(sOnes + (kk >> 2) * 2048 + (kk & 3) * 32), id_l, (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(B_OD));
         mma_commit(bar(B_VE + s));
       }
@@ -302,11 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t o_addr = tbase + lane_off + TM_O;
-    const uint32_t l_addr = tbase + lane_off + TM_L;
+    const uint32_t o_addr = tbase + lane_off + 256;
     const float c2 = d.scale_log2;
-    const unsigned long long c2x2 = pack_f32x2(c2, c2);
-    float m_used = -CUDART_INF_F;
+    float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
@@ -315,8 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       fence_after_sync();
-      const uint32_t s_addr = tbase + lane_off + TM_S + b * 128;
-      const uint32_t p_addr = tbase + lane_off + TM_P + b * 64;
+      const uint32_t s_addr = tbase + lane_off + b * 128;
+      const uint32_t p_addr = tbase + lane_off + 320 + b * 64;
       const long long rem = n_k - (long long)j * TK;
       // all 128 scores in one round of TMEM loads: the softmax is bound by
       // TMEM load latency, so a second round would cost as much as the first
@@ -331,17 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      // the maxima of the eight 16-column groups, three values per max
-      // instruction and eight independent chains
+      // the maxima of the eight 16-column groups: eight independent chains keep
+      // the single softmax warp of each sub-partition from stalling on one
+      // 128-long dependency chain
       float mq[8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t* g = &sv[q >> 1][(q & 1) * 16];
-        float m = fmax3(__uint_as_float(g[0]), __uint_as_float(g[1]), __uint_as_float(g[2]));
+      for (int q = 0; q < 8; ++q) mq[q] = __uint_as_float(sv[q >> 1][(q & 1) * 16]);
 #pragma unroll
-        for (int i = 3; i < 15; i += 2) m = fmax3(m, __uint_as_float(g[i]), __uint_as_float(g[i + 1]));
-        mq[q] = fmaxf(m, __uint_as_float(g[15]));
-      }
+      for (int i = 1; i < 16; ++i)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mq[q] = fmaxf(mq[q], __uint_as_float(sv[q >> 1][(q & 1) * 16 + i]));
       {
         // tell the top-K warp which groups may hold a candidate for this row:
         // those whose maximum beats the row's K-th best so far (a stale, lower
@@ -359,44 +394,50 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(B_PF + b));
         continue;
       }
-      const float mx = fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
+      const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                             fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
       const bool need = mxs > m_used + 8.f;
       if (__any_sync(0xffffffffu, need)) {
         const float corr = need ? exp2f(m_used - mxs) : 1.f;
         if (j > 0) {
-          // the previous P V and P 1 products must be complete before O and l
-          // are rescaled
+          // the previous P V product must be complete before O is rescaled
           if (!__all_sync(0xffffffffu, mbar_wait(bar(B_OD), (j - 1) & 1, abort_flag, err, d.wait_cycles))) {
             ok = false;
             break;
           }
           fence_after_sync();
 #pragma unroll
-          for (int c = 0; c < 5; ++c) {
-            const uint32_t addr = c < 4 ? o_addr + 16 * c : l_addr;
+          for (int c = 0; c < 4; ++c) {
             uint32_t ov[16];
-            tmem_ld16(addr, ov);
+            tmem_ld16(o_addr + 16 * c, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-            tmem_st16(addr, ov);
+            tmem_st16(o_addr + 16 * c, ov);
           }
           tmem_wait_st();
         }
-        if (need) m_used = mxs;
+        if (need) {
+          l *= corr;
+          m_used = mxs;
+        }
       }
-      const unsigned long long n2 = pack_f32x2(-m_used, -m_used);
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = (i & 7) < GSA_CMP_POLY_OF_8 ? exp2_bf16x2_poly(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2)
-                                              : exp2_bf16x2_fma(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2);
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used));
+          ps[i & 7] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
         tmem_st16(p_addr + 16 * c, pk);
       }
       tmem_wait_st();
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       fence_before_sync();
       mbar_arrive(bar(B_PF + b));
     }
@@ -405,10 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after_sync();
       const long long row = m0 + r;
       const bool store = row < d.Tc;
-      uint32_t lv[16];
-      tmem_ld16(l_addr, lv);
-      tmem_wait_ld();
-      const float inv = 1.f / __uint_as_float(lv[0]);
+      const float inv = 1.f / l;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t ov[16];
@@ -425,114 +463,105 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 8) {
     regs_inc<kRegsHigh>();
     // ---------------- streaming top-K over S_guide ----------------
-    constexpr unsigned FULL = 0xffffffffu;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    ulonglong2* lst2 = reinterpret_cast<ulonglong2*>(sp + OFF_LST);  // [row][32]: entries 2i, 2i+1
-    const uint32_t buf_s = sb + OFF_BUF;
-    const int K = d.K;
-    const int E = d.E, S = d.S;
-    const int e_min = d.B0 > 0 ? E : 0;  // frame 0's entries are not candidates when it is kept whole
-    const bool all_cols = S == 0 && e_min == 0;
+    float* cb_s = reinterpret_cast<float*>(sp + OFF_CS);
+    int* cb_e = reinterpret_cast<int*>(sp + OFF_CC);
+    Heap top{reinterpret_cast<unsigned long long*>(sp + OFF_HS), r, d.K, 0, -CUDART_INF_F};
+    const int E = d.E, S = d.S, Bf = d.Bf, B0 = (int)d.B0;
     const int ntok = (int)n_k;
     const long long my_row = m0 + r;
-    const float inv_e = 1.f / (float)E;
     // a second ranking pass keeps only pairs strictly below the first pass's
-    // K-th best key of the row
+    // K-th best (score, id) key of the row
     const unsigned long long ub =
         (cp.ub != nullptr && my_row < d.Tc) ? cp.ub[(long long)h * d.Tc + my_row] : ~0ull;
-    const bool has_ub = cp.ub != nullptr;
-    const float ub_score = ub == ~0ull ? CUDART_INF_F : order_value((uint32_t)(ub >> 32));
-    float tau = -CUDART_INF_F;  // score a candidate must beat (-inf until the list holds K pairs)
-    int nb = 0;                 // candidates in this row's buffer
-    int cnt = 0;                // pairs in this row's list (at most kMaxK)
-
-    // Merge the buffers of the rows whose lanes are set in `rows` into their
-    // lists, the whole warp working on one row at a time.
-    auto merge_rows = [&](unsigned rows) {
-      __syncwarp();
-      while (rows != 0) {
-        const int rl = __ffs(rows) - 1;
-        rows &= rows - 1;
-        const int rr = q4 * 32 + rl;
-        const int nbr = __shfl_sync(FULL, nb, rl);
-        const int cntr = __shfl_sync(FULL, cnt, rl);
-        unsigned long long bk = lane < nbr ? lds_u64(buf_s + (uint32_t)(lane * TQ + (rr ^ lane)) * 8u) : 0ull;
-        // sort the buffer descending across the lanes (bitonic)
-#pragma unroll
-        for (int k = 2; k <= 32; k <<= 1)
-#pragma unroll
-          for (int jj = k >> 1; jj > 0; jj >>= 1) bk = cmpx(bk, jj, ((lane & jj) == 0) == ((lane & k) == 0));
-        // the 64 largest of list (descending) and buffer (descending, padded
-        // with zeros to 64): max of entry i and buffer entry 63 - i, a bitonic
-        // sequence
-        ulonglong2 a2 = lst2[rr * 32 + lane];
-        const unsigned long long x0 = __shfl_sync(FULL, bk, (63 - 2 * lane) & 31);
-        const unsigned long long x1 = __shfl_sync(FULL, bk, (62 - 2 * lane) & 31);
-        if (lane >= 16) {
-          a2.x = u64max(a2.x, x0);
-          a2.y = u64max(a2.y, x1);
+    int nb = 0;  // candidates waiting in this row's buffer
+    // Insert the buffered candidates.  All lanes run this together, so one
+    // round of insertions serves every row of the warp at once.
+    const float inv_e = 1.f / (float)E;
+    auto flush = [&]() {
+      if (__all_sync(0xffffffffu, top.cnt == d.K)) {
+        // every heap of the warp is full: one predicated replacement per round
+        const int rounds = (int)__reduce_max_sync(0xffffffffu, (unsigned)nb);
+        float v_next = nb > 0 ? cb_s[r] : -CUDART_INF_F;
+        int e_next = nb > 0 ? cb_e[r] : 0;
+        for (int n = 0; n < rounds; ++n) {
+          const bool have = n < nb;
+          const float v = v_next;
+          const int e = e_next;
+          // the next round's candidate is read while this one is inserted
+          v_next = n + 1 < nb ? cb_s[(n + 1) * TQ + r] : -CUDART_INF_F;
+          e_next = n + 1 < nb ? cb_e[(n + 1) * TQ + r] : 0;
+          int f = (int)((float)e * inv_e);
+          int i = e - f * E;
+          if (i < 0) i += E, --f;
+          if (i >= E) i -= E, ++f;
+          const int id = f * Bf + (i - S);
+          const unsigned long long key = pair_key(v, id);
+          const bool take = have && v > top.tau && i >= S && id >= B0 && key < ub;
+          top.replace_root(key, take);
         }
-        // bitonic merge into descending order (element distance 2 jj, then 1)
-#pragma unroll
-        for (int jj = 16; jj > 0; jj >>= 1) {
-          const bool lower = (lane & jj) == 0;
-          a2.x = cmpx(a2.x, jj, lower);
-          a2.y = cmpx(a2.y, jj, lower);
-        }
-        if (a2.y > a2.x) {
-          const unsigned long long t = a2.x;
-          a2.x = a2.y;
-          a2.y = t;
-        }
-        lst2[rr * 32 + lane] = a2;
-        const int nc = min(cntr + nbr, kMaxK);
-        const unsigned long long kth = __shfl_sync(FULL, ((K - 1) & 1) ? a2.y : a2.x, (K - 1) >> 1);
-        if (lane == rl) {
-          cnt = nc;
-          nb = 0;
-          tau = nc >= K ? order_value((uint32_t)(kth >> 32)) : -CUDART_INF_F;
-          tau_s[r] = tau;
+        nb = 0;
+        tau_s[r] = top.tau;
+        return;
+      }
+      for (int n = 0; n < nb; ++n) {
+        const float v = cb_s[n * TQ + r];
+        if (!(v > top.tau)) continue;
+        // entry e -> frame f, position i; the float quotient is off by at most one
+        const int e = cb_e[n * TQ + r];
+        int f = (int)((float)e * inv_e);
+        int i = e - f * E;
+        if (i < 0) i += E, --f;
+        if (i >= E) i -= E, ++f;
+        // special entries are never ranked, nor blocks below B0 (frame 0 when
+        // it is kept whole)
+        if (i >= S && f * Bf + (i - S) >= B0) {
+          const unsigned long long key = pair_key(v, f * Bf + (i - S));
+          if (key < ub) top.push(key);
         }
       }
-      __syncwarp();
+      nb = 0;
+      tau_s[r] = top.tau;
     };
-
+    // One 16-column group of the score tile: candidates are the columns that
+    // beat the row's K-th best; the warp only scans groups where some of its
+    // rows has one.
+    auto group = [&](const uint32_t (&g)[16], int q, int e0, int lim) {
+      float v[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        v[i] = (16 * q + i < lim) ? __uint_as_float(g[i]) : -CUDART_INF_F;
+      float m[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) m[u] = fmaxf(fmaxf(v[u], v[u + 4]), fmaxf(v[u + 8], v[u + 12]));
+      const float m16 = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+      if (__any_sync(0xffffffffu, m16 > top.tau)) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (v[i] > top.tau) {
+            cb_s[nb * TQ + r] = v[i];
+            cb_e[nb * TQ + r] = e0 + 16 * q + i;
+            ++nb;
+          }
+        }
+        if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush();
+      }
+    };
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       const int b = j & 1;
-      if (!__all_sync(FULL, mbar_wait(bar(B_MR + b), (j >> 1) & 1, abort_flag, err, d.wait_cycles))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MR + b), (j >> 1) & 1, abort_flag, err, d.wait_cycles))) {
         ok = false;
         break;
       }
       fence_after_sync();
-      const uint32_t s_addr = tbase + lane_off + TM_S + b * 128;
+      const uint32_t s_addr = tbase + lane_off + b * 128;
       const int e0 = j * TK;
       const int lim = ntok - e0;
       // the groups flagged by the softmax for any of the warp's 32 rows
-      uint32_t G = __reduce_or_sync(FULL, (uint32_t)mask_s[b * TQ + r]);
-      // which of the tile's 128 columns may be ranked at all (the same for
-      // every row): inside the sequence, not a special entry, not below B0
-      uint32_t cv[4];
-      if (G != 0) {
-        if (all_cols && lim >= TK) {
-          cv[0] = cv[1] = cv[2] = cv[3] = FULL;
-        } else {
-          const int i0 = (e0 + lane) % E;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int c = 32 * w + lane;
-            // (i0 + 32 w) mod E; the float quotient of a small number is off by at most one
-            const int x = i0 + 32 * w;
-            int f = (int)((float)x * inv_e);
-            int i = x - f * E;
-            if (i < 0) i += E;
-            if (i >= E) i -= E;
-            cv[w] = __ballot_sync(FULL, c < lim && e0 + c >= e_min && i >= S);
-          }
-        }
-      }
+      uint32_t G = __reduce_or_sync(0xffffffffu, (uint32_t)mask_s[b * TQ + r]);
       bool released = false;
       while (G != 0) {
         const int q = __ffs(G) - 1;
@@ -545,96 +574,44 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(bar(B_SR + b));  // the tensor core may overwrite this buffer now
           released = true;
         }
-        uint32_t cm = 0;
-        if (has_ub) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float v = __uint_as_float(g[i]);
-            cm |= (v > tau && v <= ub_score ? 1u : 0u) << i;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) cm |= (__uint_as_float(g[i]) > tau ? 1u : 0u) << i;
-        }
-        cm &= (cv[q >> 1] >> ((q & 1) * 16)) & 0xffffu;
-        // the columns where any row of the warp has a candidate: usually one
-        // or two, so the append below skips the others with a uniform branch
-        const uint32_t cu = __reduce_or_sync(FULL, cm);
-        if (cu == 0) continue;
-        const unsigned over = __ballot_sync(FULL, nb + __popc(cm) > kBuf);
-        if (over != 0) merge_rows(over);
-        const uint32_t lo0 = 0x7fffffffu - (uint32_t)(e0 + 16 * q);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (cu & (1u << i)) {
-            if (cm & (1u << i)) {
-              const unsigned long long key =
-                  ((unsigned long long)order_bits(__uint_as_float(g[i])) << 32) | (lo0 - (uint32_t)i);
-              if (key < ub) {
-                sts_u64(buf_s + (uint32_t)(nb * TQ + (r ^ nb)) * 8u, key);
-                ++nb;
-              }
-            }
-          }
-        }
+        group(g, q, e0, lim);
       }
       if (!released) {
         fence_before_sync();
         mbar_arrive(bar(B_SR + b));
       }
     }
-    ok = __all_sync(FULL, ok);
-    if (ok) merge_rows(__ballot_sync(FULL, nb > 0));
-    if (ok) {
-      // write each row's result, the warp working on one row at a time: the
-      // list's first min(cnt, K) pairs are the row's top-K
-      for (int rl = 0; rl < 32; ++rl) {
-        const int rr = q4 * 32 + rl;
-        const long long row = m0 + rr;
-        if (row >= d.Tc) break;
-        const int kk = min(__shfl_sync(FULL, cnt, rl), K);
-        const ulonglong2 a2 = lst2[rr * 32 + lane];
-        const long long cb = ((long long)h * d.Tc + row) * d.K;
-        if (cp.root != nullptr && lane == ((K - 1) >> 1))
-          cp.root[(long long)h * d.Tc + row] = kk == K ? (((K - 1) & 1) ? a2.y : a2.x) : 0ull;
-        int id[2];
-        bool have[2];
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const unsigned long long key = t ? a2.y : a2.x;
-          const int e = (int)(0x7fffffffu - (uint32_t)key);
-          const int f = e / E;
-          id[t] = f * d.Bf + (e - f * E - S);
-          have[t] = 2 * lane + t < kk;
+    if (__all_sync(0xffffffffu, ok)) flush();
+    const long long row = m0 + r;
+    if (ok && row < d.Tc && cp.root != nullptr)
+      cp.root[(long long)h * d.Tc + row] = top.cnt == d.K ? top.at(0) : 0ull;
+    if (ok && row < d.Tc && cp.best != nullptr) {
+      // the row's best pair: the largest key of its heap (-1 when it is empty)
+      unsigned long long bk = 0ull;
+      int bi = -1;
+      for (int k = 0; k < top.cnt; ++k)
+        if (top.at(k) > bk) bk = top.at(k), bi = k;
+      cp.best[(long long)h * d.Tc + row] = bi >= 0 ? top.id_of(bi) : -1;
+    }
+    if (ok && row < d.Tc) {
+      const long long cb = ((long long)h * d.Tc + row) * d.K;
+      if (cand_s != nullptr) {
+        for (int k = 0; k < d.K; ++k) {
+          const bool have = k < top.cnt;
+          cand_s[cb + k] = have ? top.score_of(k) * d.scale : -CUDART_INF_F;
+          cand_i[cb + k] = have ? top.id_of(k) : -1;
         }
-        if (cp.best != nullptr && lane == 0) cp.best[(long long)h * d.Tc + row] = kk > 0 ? id[0] : -1;
-        if (cand_s != nullptr) {
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int k = 2 * lane + t;
-            if (k < K) {
-              const unsigned long long key = t ? a2.y : a2.x;
-              cand_s[cb + k] = have[t] ? order_value((uint32_t)(key >> 32)) * d.scale : -CUDART_INF_F;
-              cand_i[cb + k] = have[t] ? id[t] : -1;
-            }
-          }
+      }
+      if (sel != nullptr) {
+        // the heap holds exactly this row's top-K: write its ids in ascending
+        // order (rank of each id among the row's distinct ids), then -1 padding
+        for (int k = 0; k < top.cnt; ++k) {
+          const int me = top.id_of(k);
+          int rank = 0;
+          for (int k2 = 0; k2 < top.cnt; ++k2) rank += top.id_of(k2) < me;
+          sel[cb + rank] = me;
         }
-        if (sel != nullptr) {
-          // ascending ids: each pair's rank among the row's kk distinct ids
-          int rank[2] = {0, 0};
-          for (int m = 0; m < 32; ++m) {
-            const int o0 = __shfl_sync(FULL, id[0], m), o1 = __shfl_sync(FULL, id[1], m);
-            const bool h0 = 2 * m < kk, h1 = 2 * m + 1 < kk;
-#pragma unroll
-            for (int t = 0; t < 2; ++t) rank[t] += (h0 && o0 < id[t]) + (h1 && o1 < id[t]);
-          }
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const int k = 2 * lane + t;
-            if (have[t]) sel[cb + rank[t]] = id[t];
-            else if (k < K) sel[cb + k] = -1;
-          }
-        }
+        for (int k = top.cnt; k < d.K; ++k) sel[cb + k] = -1;
       }
     }
   }

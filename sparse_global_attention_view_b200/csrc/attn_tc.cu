@@ -9,18 +9,14 @@
 //   warp 0      TMA producer: Q tiles once, then a 4-stage ring of 128-key K/V
 //               tiles (128-byte swizzle, out-of-range rows zero-filled);
 //   warp 1      MMA issuer (one thread): S_t = Q_t K^T (bf16, fp32 in TMEM),
-//               then O_t += P_t V and l_t += P_t 1 with P_t read from TMEM;
-//   warp 2      TMEM allocation (512 columns: S_0, S_1, O_0, O_1, l_0, l_1);
+//               then O_t += P_t V with P_t read from TMEM;
+//   warp 2      TMEM allocation (512 columns: S_0, S_1, O_0, O_1);
 //   warps 4-11  softmax, one warpgroup per query tile, one thread per row.
 // The MMA thread interleaves the two tiles so one tile's softmax overlaps the
-// other tile's matrix products.  The softmax forms its maxima three values per
-// instruction in eight independent chains and its weights two per
-// instruction (packed f32x2 scaling, bf16x2 exp2: P is bf16 for the PV product
-// anyway); the row sums come from the tensor core as P times a block of ones,
-// so they add exactly the bf16 weights of the numerator.  The softmax keeps a
-// stale maximum until a tile's maximum exceeds it by 2^8 and only then
-// rescales O and the sums (in TMEM), so the common case never waits for the
-// tensor core.  Every mbarrier wait is
+// other tile's matrix products.  The softmax keeps eight independent max and
+// sum chains and takes a quarter of its exponentials on the FMA pipe.  The softmax keeps a stale maximum until a
+// tile's maximum exceeds it by 2^8 and only then rescales O (in TMEM), so the
+// common case never waits for the tensor core.  Every mbarrier wait is
 // bounded: on timeout the CTA records kErrTimeout, raises its abort flag, drains
 // its own TMA loads and MMAs, frees TMEM and returns.
 #include <math_constants.h>
@@ -35,12 +31,29 @@ namespace {
 
 using namespace tc;
 
-// Of every 8 pairs of attention weights, this many are computed on the FMA
-// pipe (exp2_bf16x2_poly) and the rest on the special-function unit: at
-// head dim 64 the exponentials, not the tensor core, bound the softmax.
-#ifndef GSA_ATTN_POLY_OF_8
-#define GSA_ATTN_POLY_OF_8 0
-#endif
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
+}
+// 2^x on the FMA pipe, for a quarter of the softmax's exponentials so that the
+// special-function unit is not the only bound: Cody-Waite range reduction
+// x = j + f, j = round(x) (added to the exponent bits), f in [-1/2, 1/2], and a
+// cubic fitted to 2^f on that interval by iteratively reweighted least squares
+// on Chebyshev nodes (max relative error 7.5e-5 in fp32, below the bf16
+// rounding of P).  x is clamped at -125 (the result is then ~2^-125, i.e. 0 for
+// the softmax).
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;
+  const int j = __float_as_int(t) - 0x4B400000;
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(0.055171769f, f, 0.24261113f);
+  p = fmaf(p, f, 0.69326097f);
+  p = fmaf(p, f, 0.99992806f);
+  return __int_as_float(__float_as_int(p) + (j << 23));
+}
+
 
 constexpr int TQ = 128;            // rows per query tile
 constexpr int NQT = 2;             // query tiles per CTA
@@ -52,8 +65,7 @@ constexpr uint32_t kTile = 128 * 128;  // bytes of one [128][64] bf16 tile
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_K = OFF_Q + NQT * kTile;
 constexpr uint32_t OFF_V = OFF_K + ST * kTile;
-constexpr uint32_t OFF_ONES = OFF_V + ST * kTile;  // B operand of the row-sum product
-constexpr uint32_t OFF_BAR = OFF_ONES + kOnesBytes;
+constexpr uint32_t OFF_BAR = OFF_V + ST * kTile;
 constexpr uint32_t OFF_MISC = OFF_BAR + 256;
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;  // + alignment slack
 
@@ -62,7 +74,7 @@ constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + ST, B_KVE = B_VF + ST, B_SF = B_K
               B_PF = B_SF + NQT, B_OF = B_PF + NQT, B_DRAIN = B_OF + NQT, B_COUNT = B_DRAIN + 1;
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 
-constexpr uint32_t kCols = 512;  // TMEM columns: S_t at 128 t, O_t at 256 + 64 t, l_t at 384 + 16 t
+constexpr uint32_t kCols = 512;  // TMEM columns: S_t at 128 t, O_t at 256 + 64 t
 // Register split between the producer/MMA warpgroup and the two softmax
 // warpgroups; it must not exceed the launch allocation, or the increase would
 // wait forever (the host checks the compiled register count before launching).
@@ -117,8 +129,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  fill_ones(sp + OFF_ONES, kOnesBytes, tid, kThreads);
-  fence_proxy_async_smem();
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), kCols);
     tmem_relinquish();
@@ -165,8 +175,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       const uint32_t id_qk = idesc(128, 128, kFmtBF16, 0, 0);
       const uint32_t id_pv = idesc(128, 64, kFmtBF16, 0, 1);
-      const uint32_t id_l = idesc(128, 16, kFmtBF16, 0, 0);
-      const uint32_t sOnes = sb + OFF_ONES;
       auto issue_s = [&](int t, int s) {
         const uint32_t d = tbase + t * 128;
 #pragma unroll
@@ -192,10 +200,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int kk = 0; kk < 8; ++kk)
             mma_bf16_ts(d, tbase + t * 128 + kk * 8, sdesc_mn(sV + s * kTile + kk * 2048), id_pv,
                         (j > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16_ts(tbase + 384 + t * 16, tbase + t * 128 + kk * 8,
-                        sdesc_k(sOnes + (kk >> 2) * 2048 + (kk & 3) * 32), id_l, (j > 0 || kk > 0) ? 1u : 0u);
           if (j + 1 < nt) {
             const int s1 = (j + 1) % ST;
             if (t == 0) {
@@ -225,10 +229,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const uint32_t s_addr = tbase + lane_off + t * 128;
     const uint32_t o_addr = tbase + lane_off + 256 + t * 64;
-    const uint32_t l_addr = tbase + lane_off + 384 + t * 16;
     const float c2 = a.c2;
-    const unsigned long long c2x2 = pack_f32x2(c2, c2);
-    float m_used = -CUDART_INF_F;
+    float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
       // the whole warp leaves together: tcgen05.ld/st below are warp-collective
@@ -249,18 +251,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      // eight independent max chains, three values per instruction: each
-      // softmax warp owns whole rows, so one long chain would leave it stalled
+      // eight independent max / sum chains: each softmax warp owns whole rows,
+      // so a single 128-long dependency chain would leave it stalled
       float mq[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const uint32_t* g = &sv[u >> 1][(u & 1) * 16];
-        float m = fmax3(__uint_as_float(g[0]), __uint_as_float(g[1]), __uint_as_float(g[2]));
+      for (int u = 0; u < 8; ++u) mq[u] = __uint_as_float(sv[0][u]);
 #pragma unroll
-        for (int i = 3; i < 15; i += 2) m = fmax3(m, __uint_as_float(g[i]), __uint_as_float(g[i + 1]));
-        mq[u] = fmaxf(m, __uint_as_float(g[15]));
-      }
-      const float mx = fmax3(fmax3(mq[0], mq[1], mq[2]), fmax3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
+      for (int k = 8; k < 128; ++k) mq[k & 7] = fmaxf(mq[k & 7], __uint_as_float(sv[k >> 5][k & 31]));
+      const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
+                             fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
       const bool need = mxs > m_used + 8.f;
       // tcgen05.ld/st are warp-collective: the warp rescales together, with
@@ -268,32 +267,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (__any_sync(0xffffffffu, need)) {
         const float corr = need ? exp2f(m_used - mxs) : 1.f;
         if (j > 0) {
-          // O_t's and l_t's previous products are complete: S_t(j) was issued after them
+          // O_t's previous product is complete: S_t(j) was issued after it
 #pragma unroll
-          for (int c = 0; c < 5; ++c) {
-            const uint32_t addr = c < 4 ? o_addr + 16 * c : l_addr;
+          for (int c = 0; c < 4; ++c) {
             uint32_t ov[16];
-            tmem_ld16(addr, ov);
+            tmem_ld16(o_addr + 16 * c, ov);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * corr);
-            tmem_st16(addr, ov);
+            tmem_st16(o_addr + 16 * c, ov);
           }
           tmem_wait_st();
         }
-        if (need) m_used = mxs;
+        if (need) {
+          l *= corr;
+          m_used = mxs;
+        }
       }
-      const unsigned long long n2 = pack_f32x2(-m_used, -m_used);
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = (i & 7) < GSA_ATTN_POLY_OF_8 ? exp2_bf16x2_poly(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2)
-                                               : exp2_bf16x2_fma(sv[c][2 * i], sv[c][2 * i + 1], c2x2, n2);
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
+          const float x1 = fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used);
+          const float p1 = (i & 1) ? exp2_fma(x1) : fast_exp2(x1);  // one in four on the FMA pipe
+          ps[i & 7] += p0 + p1;
+          pk[i] = pack_bf16x2(p0, p1);
+        }
         tmem_st16(s_addr + 16 * c, pk);
       }
       tmem_wait_st();
+      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       fence_before_sync();
       mbar_arrive(bar(B_PF + t));
     }
@@ -302,10 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after_sync();
       const long long row = m0 + t * TQ + q4 * 32 + lane;
       const bool store = row < q_end;
-      uint32_t lv[16];
-      tmem_ld16(l_addr, lv);
-      tmem_wait_ld();
-      const float l = __uint_as_float(lv[0]);
       const float inv = 1.f / l;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {

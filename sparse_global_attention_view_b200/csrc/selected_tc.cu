@@ -15,15 +15,17 @@
 // over a per-frame view of the token grid (dims: 64 values, head, column, row,
 // frame): 16 rows of 128 bytes, patches outside the grid read as zero.
 //
-// One CTA works through (head, entry) pairs; 12 warps:
+// One CTA per SM works through (head, entry) pairs; 12 warps:
 //   warp 0      TMA producer: per entry its queries (one box) and selection,
 //               then per 128-key tile the 8 blocks' K and V (two boxes each),
-//               into a 2-stage ring; when the always-kept tokens are not
+//               into a 5-stage ring (the gathers are latency-bound: many small
+//               boxes, so as many as possible are kept in flight); when the always-kept tokens are not
 //               supplied as a finished softmax state, their head-major copies
 //               are streamed first as plain 128-key tiles;
 //   warp 1      MMA issuer (one thread): S^T(t+1) is issued before O^T(t), so
 //               the tensor core works while the softmax handles a tile;
-//   warp 2      TMEM allocation (S^T at columns 0/16, O^T at 32/48);
+//   warp 2      TMEM allocation (S^T at columns 0/16, O^T at 32 + 16 e for
+//               the four entry slots e);
 //   warps 4-7   softmax, one thread per key lane (16 queries per thread);
 //   warps 8-11  epilogue of the previous entry (normalise, merge with the
 //               always-kept segment, gate, store) while the softmax works on
@@ -49,8 +51,8 @@ using namespace tc;
 constexpr int NQ = 16;           // query slots per entry (P * P <= 16)
 constexpr int TKEYS = 128;       // keys per tile
 constexpr int BPT = 8;           // selected blocks per tile
-constexpr int ST = 2;            // K/V ring stages
-constexpr int NE = 2;            // entry slots (queries, selection, O^T buffer)
+constexpr int ST = 5;            // K/V ring stages: the gathers of 5 tiles in flight
+constexpr int NE = 4;            // entry slots (queries, selection, O^T buffer)
 constexpr int kThreads = 384;
 constexpr uint32_t kKV = 16384;  // one [128][64] bf16 tile
 constexpr uint32_t kQ = 2048;    // one [16][64] bf16 query tile
@@ -78,26 +80,20 @@ constexpr uint32_t OFF_RED = OFF_ENT + NE * kEntBytes;   // [4 warps][16] per-qu
 constexpr uint32_t OFF_LS = OFF_RED + 4 * NQ * 4;        // [16] sums of P (epilogue)
 constexpr uint32_t OFF_GATE = OFF_LS + NQ * 4;           // [2] gate partial dot products
 constexpr uint32_t OFF_BAR = (OFF_GATE + 16 + 255) / 256 * 256;
-constexpr uint32_t OFF_MISC = OFF_BAR + 256;
+constexpr uint32_t OFF_MISC = OFF_BAR + 512;
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 static_assert(OFF_Q % 1024 == 0 && OFF_PT % 1024 == 0 && OFF_ONES % 1024 == 0, "operand alignment");
-static_assert(2 * kSmemBytes <= 232448, "two CTAs per SM");
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 // barriers
 constexpr int B_EF = 0, B_EE = B_EF + NE, B_EM = B_EE + NE, B_KF = B_EM + NE, B_VF = B_KF + ST,
               B_KE = B_VF + ST, B_VE = B_KE + ST, B_SF = B_VE + ST, B_PF = B_SF + 2, B_PE = B_PF + 2,
               B_OF = B_PE + 2, B_OD = B_OF + NE, B_DRAIN = B_OD + 1, B_COUNT = B_DRAIN + 1;
-static_assert(B_COUNT * 8 <= 256, "barrier area");
+static_assert(B_COUNT * 8 <= 512, "barrier area");
 
-constexpr uint32_t kCols = 64;  // TMEM: S^T at 0 / 16, O^T at 32 / 48
+constexpr uint32_t kCols = 128;  // TMEM: S^T at 0 / 16, O^T at 32 + 16 e (e < NE)
 constexpr uint32_t TM_S = 0, TM_O = 32;
-// Register split: launched with kLaunchRegs per thread (two CTAs per SM); the
-// producer / MMA warpgroup and the epilogue give registers to the softmax.
-// The shares must not exceed the launch allocation, or the increase would wait
-// forever: the host refuses to launch unless the compiled kernel uses exactly
-// kLaunchRegs registers per thread.
-constexpr int kLaunchRegs = 80, kRegsLow = 48, kRegsSoft = 120, kRegsEpi = 72;
-static_assert(128 * (kRegsLow + kRegsSoft + kRegsEpi) <= kThreads * kLaunchRegs, "register split");
+static_assert(TM_O + 16 * NE <= kCols, "TMEM columns");
 
 __device__ __forceinline__ uint32_t pt_addr(uint32_t base, int q, int k) {
   // [16 queries][128 keys] bf16, K-major, 128-byte swizzle: keys 0-63 and
@@ -148,7 +144,7 @@ struct Maps {
   CUtensorMap ks, vs;      // [H][NK][64] kept copies, box 128 keys (kept keys streamed inline)
 };
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     selected_tc_kernel(const __grid_constant__ Maps mp, const Dims d, const int* __restrict__ sel,
                        const int* __restrict__ order, const float* __restrict__ qc32,
                        const float* __restrict__ w, const float* __restrict__ oc, bf16* __restrict__ out,
@@ -209,7 +205,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   fence_after_sync();
   const uint32_t tbase = *tmem_slot;
 
-  if (warp < 4) regs_dec<kRegsLow>();
   if (warp == 0) {
     // ---------------- TMA producer (the whole warp) ----------------
     if (lane == 0) {
@@ -404,7 +399,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   } else if (warp >= 4 && warp < 8) {
-    regs_inc<kRegsSoft>();
     // ---------------- softmax, one thread per key lane ----------------
     const int q4 = warp & 3;
     const int k = q4 * 32 + lane;
@@ -546,7 +540,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   } else if (warp >= 8) {
-    regs_dec<kRegsEpi>();
     // ---------------- epilogue, one thread per TMEM lane ----------------
     const int q4 = warp & 3;
     const int dlane = q4 * 32 + lane;  // lanes 0-63: value dims; 64-127: sums of P
@@ -662,14 +655,10 @@ cudaError_t launch_selected_tc(const Dims& d, const bf16* q, const bf16* k, cons
   cudaError_t e = cudaFuncSetAttribute(selected_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, selected_tc_kernel);
-  if (e != cudaSuccess) return e;
-  if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long items = (long long)d.H * d.Tc;
-  const long long grid = items < 2LL * sms ? items : 2LL * sms;
+  const long long grid = items < (long long)sms ? items : (long long)sms;
   if (grid <= 0) return cudaSuccess;
   selected_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mp, d, sel, order, qc32, w, oc, out, lse,
                                                                   o_spec, lse_spec, err, kept_inline);

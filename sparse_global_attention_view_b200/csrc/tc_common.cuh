@@ -223,17 +223,6 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 // ---------------------------------------------------------------------------
 // softmax arithmetic
 
-// max of three (one instruction on sm_100)
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float m;
-  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(m) : "f"(a), "f"(b), "f"(c));
-  return m;
-}
-__device__ __forceinline__ unsigned long long pack_f32x2(float lo, float hi) {
-  unsigned long long x;
-  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "f"(lo), "f"(hi));
-  return x;
-}
 // exp2 of two fp32 values, rounded to bf16 and exponentiated two at a time
 // (one special-function instruction for the pair): the packed pair of
 // attention weights (lo in the low half), bf16 like the PV operand they feed.
@@ -243,66 +232,9 @@ __device__ __forceinline__ uint32_t exp2_bf16x2(float lo, float hi) {
   asm("ex2.approx.ftz.bf16x2 %0, %1;\n" : "=r"(e) : "r"(b));
   return e;
 }
-// The same for two raw fp32 scores (bit patterns) scaled and shifted first,
-// x * c + n, as one packed f32x2 FMA.
-__device__ __forceinline__ uint32_t exp2_bf16x2_fma(uint32_t lo, uint32_t hi, unsigned long long c2,
-                                                    unsigned long long n2) {
-  unsigned long long x, y;
-  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "r"(lo), "r"(hi));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(y) : "l"(x), "l"(c2), "l"(n2));
-  uint32_t ylo, yhi, b, e;
-  asm("mov.b64 {%0, %1}, %2;\n" : "=r"(ylo), "=r"(yhi) : "l"(y));
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(b) : "r"(yhi), "r"(ylo));
-  asm("ex2.approx.ftz.bf16x2 %0, %1;\n" : "=r"(e) : "r"(b));
-  return e;
-}
-// The same pair of weights computed on the FMA pipe instead of the
-// special-function unit, so a softmax can split its exponentials between the
-// two pipes: x = j + f with j = round(x) (the 1.5 * 2^23 rounding constant)
-// and f in [-1/2, 1/2], 2^f from a cubic fitted here to 2^f on that interval
-// (iteratively reweighted least squares on Chebyshev nodes; largest relative
-// error 7.5e-5, far below the bf16 rounding that follows), 2^j added to the
-// exponent bits.  x is clamped at -125 (the weight is then 0 in bf16).
-__device__ __forceinline__ uint32_t exp2_bf16x2_poly(uint32_t lo, uint32_t hi, unsigned long long c2,
-                                                     unsigned long long n2) {
-  unsigned long long x, y;
-  asm("mov.b64 %0, {%1, %2};\n" : "=l"(x) : "r"(lo), "r"(hi));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(y) : "l"(x), "l"(c2), "l"(n2));
-  float y0, y1;
-  asm("mov.b64 {%0, %1}, %2;\n" : "=f"(y0), "=f"(y1) : "l"(y));
-  y = pack_f32x2(fmaxf(y0, -125.f), fmaxf(y1, -125.f));
-  const unsigned long long kRound = pack_f32x2(12582912.f, 12582912.f);  // 1.5 * 2^23
-  unsigned long long t, r, f, p;
-  asm("add.rn.f32x2 %0, %1, %2;\n" : "=l"(t) : "l"(y), "l"(kRound));
-  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(r) : "l"(t), "l"(kRound));
-  asm("sub.rn.f32x2 %0, %1, %2;\n" : "=l"(f) : "l"(y), "l"(r));
-  const unsigned long long k3 = pack_f32x2(0.055171769f, 0.055171769f);
-  const unsigned long long k2 = pack_f32x2(0.24261113f, 0.24261113f);
-  const unsigned long long k1 = pack_f32x2(0.69326097f, 0.69326097f);
-  const unsigned long long k0 = pack_f32x2(0.99992806f, 0.99992806f);
-  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(p) : "l"(k3), "l"(f), "l"(k2));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(p) : "l"(p), "l"(f), "l"(k1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;\n" : "=l"(p) : "l"(p), "l"(f), "l"(k0));
-  uint32_t p0, p1, t0, t1, b;
-  asm("mov.b64 {%0, %1}, %2;\n" : "=r"(p0), "=r"(p1) : "l"(p));
-  asm("mov.b64 {%0, %1}, %2;\n" : "=r"(t0), "=r"(t1) : "l"(t));
-  p0 += (t0 - 0x4B400000u) << 23;
-  p1 += (t1 - 0x4B400000u) << 23;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;\n" : "=r"(b) : "r"(p1), "r"(p0));
-  return b;
-}
-
 // Generic-proxy writes to shared memory that the tensor core reads next.
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
-// 16 x 128 bf16 ones: the B operand of a P 1 product (the row sums of P).
-constexpr uint32_t kOnesBytes = 4096;
-__device__ __forceinline__ void fill_ones(uint8_t* p, uint32_t bytes, int tid, int nthreads) {
-  uint4* o = reinterpret_cast<uint4*>(p);
-  for (int i = tid; i < (int)(bytes / 16); i += nthreads)
-    o[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-}
-
 }  // namespace tc
 }  // namespace gsa

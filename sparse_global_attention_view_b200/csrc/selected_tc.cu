@@ -6,22 +6,27 @@
 // The <= 16 fine queries of one compressed entry (query block) share one key
 // set, so the products run transposed, with the keys on the 128-row M side and
 // the entry's queries as N = 16:
-//   S^T  = K_sel Q^T               M = 128 keys (8 selected blocks x 16 slots), K = 64
+//   S^T  = K_sel Q^T               M = 128 keys, K = 64
 //   O^T += [V_sel | 1]^T P^T       M = 128: the 64 value dims, then 64 rows of
 //                                  ones whose results are the sums of P per query
 // so P never leaves the softmax thread's lane except as the B operand, and the
 // row sums come out of the tensor core with exactly the bf16 weights of the
-// numerator.  A selected P x P block (P <= 4) is one TMA box of 4 x 4 patches
-// over a per-frame view of the token grid (dims: 64 values, head, column, row,
-// frame): 16 rows of 128 bytes, patches outside the grid read as zero.
+// numerator.  The keys of a pair are the valid tokens of its selected blocks
+// packed into consecutive slots (a block at the right or bottom edge holds 4
+// or 1 of its 16 patches, and those are the blocks S_guide tends to rank
+// first: their means keep more of the tokens' noise, so their scores spread
+// wider), so a pair needs ceil(valid tokens / 128) tiles rather than K / 8.
+// The producer gathers each slot's 128 bytes with cp.async straight into the
+// 128-byte-swizzled operand layout; the entry's queries are one TMA box of
+// 4 x 4 patches over a per-frame view of the token grid.
 //
 // One CTA per SM works through (head, entry) pairs; 12 warps:
-//   warp 0      TMA producer: per entry its queries (one box) and selection,
-//               then per 128-key tile the 8 blocks' K and V (two boxes each),
-//               into a 5-stage ring (the gathers are latency-bound: many small
-//               boxes, so as many as possible are kept in flight); when the always-kept tokens are not
-//               supplied as a finished softmax state, their head-major copies
-//               are streamed first as plain 128-key tiles;
+//   warp 0      producer: per entry its queries (one TMA box) and its packed
+//               token list (from the selection, loaded one entry ahead), then
+//               per 128-key tile the K and V rows by cp.async into a 5-stage
+//               ring; when the always-kept tokens are not supplied as a
+//               finished softmax state, their head-major copies are streamed
+//               first as plain 128-key TMA tiles;
 //   warp 1      MMA issuer (one thread): S^T(t+1) is issued before O^T(t), so
 //               the tensor core works while the softmax handles a tile;
 //   warp 2      TMEM allocation (S^T at columns 0/16, O^T at 32 + 16 e for
@@ -50,7 +55,6 @@ using namespace tc;
 
 constexpr int NQ = 16;           // query slots per entry (P * P <= 16)
 constexpr int TKEYS = 128;       // keys per tile
-constexpr int BPT = 8;           // selected blocks per tile
 constexpr int ST = 5;            // K/V ring stages: the gathers of 5 tiles in flight
 constexpr int NE = 4;            // entry slots (queries, selection, O^T buffer)
 constexpr int kThreads = 384;
@@ -61,12 +65,11 @@ constexpr uint32_t kPT = 4096;   // one [16][128] bf16 P^T tile (two 64-key atom
 struct Entry {
   int h, a;
   int n_tiles, n_kept;  // tiles in all; the first n_kept stream the always-kept keys
-  int nsel;             // valid ids in sel
+  int n_keys;           // valid tokens of the selected blocks (key slots 0 .. n_keys - 1)
   uint32_t qmask;       // query slots that hold a token
   int tok[NQ];          // token of each query slot
   float m0[NQ];         // initial reference (log2 units of the scaled logit)
   float mf[NQ], wf[NQ]; // final reference and weight of the always-kept segment
-  int sel[kMaxTopK];
 };
 
 constexpr uint32_t OFF_K = 0;
@@ -76,7 +79,8 @@ constexpr uint32_t OFF_Q = OFF_ONES + kKV;
 constexpr uint32_t OFF_PT = OFF_Q + NE * kQ;
 constexpr uint32_t OFF_ENT = OFF_PT + 2 * kPT;
 constexpr uint32_t kEntBytes = (sizeof(Entry) + 127) / 128 * 128;
-constexpr uint32_t OFF_RED = OFF_ENT + NE * kEntBytes;   // [4 warps][16] per-query partial maxima
+constexpr uint32_t OFF_TOK = OFF_ENT + NE * kEntBytes;   // the producer's token list of one entry
+constexpr uint32_t OFF_RED = OFF_TOK + kMaxTopK * NQ * 4;  // [4 warps][16] per-query partial maxima
 constexpr uint32_t OFF_LS = OFF_RED + 4 * NQ * 4;        // [16] sums of P (epilogue)
 constexpr uint32_t OFF_GATE = OFF_LS + NQ * 4;           // [2] gate partial dot products
 constexpr uint32_t OFF_BAR = (OFF_GATE + 16 + 255) / 256 * 256;
@@ -139,13 +143,14 @@ __device__ __forceinline__ Blk block_of(const Dims& d, int beta) {
 }
 
 struct Maps {
-  CUtensorMap q5, k5, v5;  // per-frame grid views, box 4 x 4 patches of one head
+  CUtensorMap q5;          // per-frame grid view of Q, box 4 x 4 patches of one head
   CUtensorMap q3;          // [T][H][64], box one token of one head (special entries)
   CUtensorMap ks, vs;      // [H][NK][64] kept copies, box 128 keys (kept keys streamed inline)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    selected_tc_kernel(const __grid_constant__ Maps mp, const Dims d, const int* __restrict__ sel,
+    selected_tc_kernel(const __grid_constant__ Maps mp, const Dims d, const bf16* __restrict__ kg,
+                       const bf16* __restrict__ vg, const int* __restrict__ sel,
                        const int* __restrict__ order, const float* __restrict__ qc32,
                        const float* __restrict__ w, const float* __restrict__ oc, bf16* __restrict__ out,
                        float* __restrict__ lse, const float* __restrict__ o_spec,
@@ -171,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_OF + s), 1);
     }
     for (int s = 0; s < ST; ++s) {
-      mbar_init(bar(B_KF + s), 1);
-      mbar_init(bar(B_VF + s), 1);
+      mbar_init(bar(B_KF + s), 32);  // one arrival per producer lane
+      mbar_init(bar(B_VF + s), 32);
       mbar_init(bar(B_KE + s), 1);
       mbar_init(bar(B_VE + s), 1);
     }
@@ -194,6 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
     uint4* qz = reinterpret_cast<uint4*>(sp + OFF_Q);
     for (int i = tid; i < (int)(NE * kQ / 16); i += kThreads) qz[i] = make_uint4(0u, 0u, 0u, 0u);
+    // the K/V ring: gathered tiles copy only their valid key slots, so the
+    // rest must start finite
+    uint4* kvz = reinterpret_cast<uint4*>(sp + OFF_K);
+    for (int i = tid; i < (int)(2 * ST * kKV / 16); i += kThreads) kvz[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();
   }
   if (warp == 2) {
@@ -209,68 +218,136 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------- TMA producer (the whole warp) ----------------
     if (lane == 0) {
       prefetch_tmap(&mp.q5);
-      prefetch_tmap(&mp.k5);
-      prefetch_tmap(&mp.v5);
       prefetch_tmap(&mp.q3);
     }
+    int* tok_list = reinterpret_cast<int*>(sp + OFF_TOK);
+    const int KU = (d.K + 31) / 32;  // ids per lane
+    // the selection and the pair of an entry are loaded one entry ahead, so
+    // their latency overlaps the gathers of the entry before
+    auto pair_of = [&](long long item) -> long long {
+      return item < n_items ? (order != nullptr ? (long long)order[item] : item) : -1;
+    };
+    // The query slot `lane` (< 16) of a pair: its token (or -1), and the
+    // always-kept segment's log-sum-exp for it, in log2 units (-inf without).
+    struct QSlot {
+      long long t;
+      float m0;
+    };
+    auto query_slot = [&](long long pair) -> QSlot {
+      QSlot r{-1, -CUDART_INF_F};
+      if (pair < 0 || lane >= NQ) return r;
+      const int h = (int)(pair / d.Tc);
+      const int a = (int)(pair - (long long)h * d.Tc);
+      const int f = a / d.E, j = a - (a / d.E) * d.E;
+      if (j < d.S) {
+        if (lane == 0) r.t = (long long)f * d.L + j;
+      } else {
+        const Blk qb = block_of(d, f * d.Bf + (j - d.S));
+        const int pr = lane >> 2, pc = lane & 3;
+        if (pr < qb.nr && pc < qb.nc) r.t = (long long)f * d.L + d.S + (long long)(qb.r0 + pr) * d.Wp + qb.c0 + pc;
+      }
+      if (r.t >= 0 && lse_spec != nullptr) r.m0 = lse_spec[r.t * d.H + h] * 1.4426950408889634f;
+      return r;
+    };
+    long long pair_cur = pair_of(blockIdx.x);
+    long long pair_nxt = pair_of(blockIdx.x + (long long)gridDim.x);
+    int ids_cur[kMaxTopK / 32];
+#pragma unroll
+    for (int u = 0; u < kMaxTopK / 32; ++u) {
+      const int k = lane + 32 * u;
+      ids_cur[u] = (u < KU && k < d.K && pair_cur >= 0) ? sel[pair_cur * d.K + k] : -1;
+    }
+    QSlot qs_cur = query_slot(pair_cur);
     int gt = 0;  // tiles loaded
     int ne = 0;  // entries loaded
     bool ok = true;
     for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
       const int es = ne % NE;
+      // prefetch: the next entry's selection and query slots, the pair after it
+      int ids_nxt[kMaxTopK / 32];
+#pragma unroll
+      for (int u = 0; u < kMaxTopK / 32; ++u) {
+        const int k = lane + 32 * u;
+        ids_nxt[u] = (u < KU && k < d.K && pair_nxt >= 0) ? sel[pair_nxt * d.K + k] : -1;
+      }
+      const QSlot qs_nxt = query_slot(pair_nxt);
+      const long long pair_nn = pair_of(it + 2LL * gridDim.x);
       if (ne >= NE && !__all_sync(0xffffffffu, mbar_wait(bar(B_EE + es), ((ne / NE) - 1) & 1, abort_flag, err, d.wait_cycles))) {
         ok = false;
         break;
       }
-      const long long pair = order != nullptr ? (long long)order[it] : it;
+      const long long pair = pair_cur;
       const int h = (int)(pair / d.Tc);
       const int a = (int)(pair - (long long)h * d.Tc);
       Entry& E = ent(es);
       // the selection: ascending ids, -1 padded; an id outside [0, NB) ends the
       // list and raises the device-check bit instead of being dereferenced
-      const int* sl = sel + ((long long)h * d.Tc + a) * d.K;
       int nsel = d.K;
-      for (int k0 = 0; k0 < d.K; k0 += 32) {
-        const int k = k0 + lane;
-        const int id = k < d.K ? sl[k] : -1;
-        if (k < d.K) E.sel[k] = id;
-        const unsigned bad = __ballot_sync(0xffffffffu, k < d.K && (id < 0 || id >= d.NB));
-        const unsigned oob = __ballot_sync(0xffffffffu, k < d.K && id >= d.NB);
+#pragma unroll
+      for (int u = 0; u < kMaxTopK / 32; ++u) {
+        if (u >= KU) break;
+        const int k = lane + 32 * u;
+        const bool in = k < d.K;
+        const unsigned bad = __ballot_sync(0xffffffffu, in && (ids_cur[u] < 0 || ids_cur[u] >= d.NB));
+        const unsigned oob = __ballot_sync(0xffffffffu, in && ids_cur[u] >= d.NB);
         if (oob != 0 && lane == 0) atomicOr(err, kErrDeviceCheck);
-        if (bad != 0 && nsel == d.K) nsel = k0 + __ffs(bad) - 1;
+        if (bad != 0 && nsel == d.K) nsel = 32 * u + __ffs(bad) - 1;
       }
-      // the entry's queries
+      // the valid tokens of the selected blocks, in selection order, packed
+      // into consecutive key slots: a prefix sum of the blocks' token counts;
+      // a block's valid patches are its first nr rows and nc columns
+      int carry = 0;
+#pragma unroll
+      for (int u = 0; u < kMaxTopK / 32; ++u) {
+        if (u >= KU || 32 * u >= nsel) break;
+        const int k = lane + 32 * u;
+        Blk kb{0, 0, 0, 0, 0};
+        int cnt = 0;
+        if (k < nsel) {
+          kb = block_of(d, ids_cur[u]);
+          cnt = kb.nr * kb.nc;
+        }
+        int incl = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        int pos = carry + incl - cnt;
+        const long long t0 = (long long)kb.f * d.L + d.S + (long long)kb.r0 * d.Wp + kb.c0;
+#pragma unroll
+        for (int pr = 0; pr < kMaxPool; ++pr) {
+#pragma unroll
+          for (int pc = 0; pc < kMaxPool; ++pc) {
+            if (pr < kb.nr && pc < kb.nc) {
+              tok_list[pos] = (int)(t0 + (long long)pr * d.Wp + pc);
+              ++pos;
+            }
+          }
+        }
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      const int n_keys = carry;
+      const int n_tiles = n_kept_tiles + (n_keys + TKEYS - 1) / TKEYS;
+      // the entry's queries (tokens and references prefetched with the selection)
       const int f = a / d.E, j = a - (a / d.E) * d.E;
       const bool special = j < d.S;
-      Blk qb;
+      Blk qb{0, 0, 0, 0, 0};
       if (!special) qb = block_of(d, f * d.Bf + (j - d.S));
       if (lane < NQ) {
-        const int pr = lane >> 2, pc = lane & 3;
-        bool valid;
-        long long t;
-        if (special) {
-          valid = lane == 0;
-          t = (long long)f * d.L + j;
-        } else {
-          valid = pr < qb.nr && pc < qb.nc;
-          t = (long long)f * d.L + d.S + (long long)(qb.r0 + pr) * d.Wp + qb.c0 + pc;
-        }
-        E.tok[lane] = valid ? (int)t : -1;
-        float m0 = -CUDART_INF_F;
-        if (valid && lse_spec != nullptr) m0 = lse_spec[t * d.H + h] * 1.4426950408889634f;
-        E.m0[lane] = m0;
+        E.tok[lane] = (int)qs_cur.t;
+        E.m0[lane] = qs_cur.m0;
       }
-      const unsigned qm = __ballot_sync(0xffffffffu, lane < NQ && (special ? lane == 0 : ((lane >> 2) < qb.nr && (lane & 3) < qb.nc)));
+      const unsigned qm = __ballot_sync(0xffffffffu, lane < NQ && qs_cur.t >= 0);
       if (lane == 0) {
         E.h = h;
         E.a = a;
-        E.nsel = nsel;
+        E.n_keys = n_keys;
         E.n_kept = n_kept_tiles;
-        E.n_tiles = n_kept_tiles + (nsel + BPT - 1) / BPT;
+        E.n_tiles = n_tiles;
         E.qmask = qm & 0xffffu;
       }
-      const int n_tiles = n_kept_tiles + (nsel + BPT - 1) / BPT;
-      __syncwarp();
+      __syncwarp();  // the entry info and the token list are written
       if (lane == 0) {
         // the one arrival on the entry's barrier (arrive.expect_tx, release: it
         // also publishes the info the warp wrote above); the phase completes
@@ -284,7 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_5d(dq, &mp.q5, bar(B_EF + es), 0, h, qb.c0, qb.r0, f);
         }
       }
-      // the key tiles
+      // the key tiles: every lane arrives once on the tile's K and V barriers
+      // (count 32): through the TMA transaction count for the always-kept
+      // tiles, through cp.async completion for the gathered ones
       for (int i = 0; ok && i < n_tiles; ++i, ++gt) {
         const int s = gt % ST;
         if (gt >= ST) {
@@ -295,26 +374,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
         }
-        if (lane == 0) {
-          mbar_expect_tx(bar(B_KF + s), kKV);
-          mbar_expect_tx(bar(B_VF + s), kKV);
-        }
-        __syncwarp();
         const uint32_t dk = sb + OFF_K + s * kKV, dv = sb + OFF_V + s * kKV;
         if (i < n_kept_tiles) {
           if (lane == 0) {
+            mbar_expect_tx(bar(B_KF + s), kKV);
+            mbar_expect_tx(bar(B_VF + s), kKV);
             tma_load_3d(dk, &mp.ks, bar(B_KF + s), 0, i * TKEYS, h);
             tma_load_3d(dv, &mp.vs, bar(B_VF + s), 0, i * TKEYS, h);
+          } else {
+            mbar_arrive(bar(B_KF + s));
+            mbar_arrive(bar(B_VF + s));
           }
-        } else if (lane < BPT) {
-          const int idx = (i - n_kept_tiles) * BPT + lane;
-          // past the list: any block, fully masked by the softmax
-          const Blk kb = block_of(d, idx < nsel ? E.sel[idx] : 0);
-          tma_load_5d(dk + lane * 2048, &mp.k5, bar(B_KF + s), 0, h, kb.c0, kb.r0, kb.f);
-          tma_load_5d(dv + lane * 2048, &mp.v5, bar(B_VF + s), 0, h, kb.c0, kb.r0, kb.f);
+        } else {
+          // key slot c of the tile = packed slot 128 i' + c; row c of the
+          // operand tile is that token's 128 bytes, its 16-byte chunks in the
+          // 128-byte swizzle.  Only the valid slots are copied: the rest keep
+          // finite data (zeroed at start, or an earlier tile's rows) that the
+          // softmax masks to weight 0
+          const int g0 = (i - n_kept_tiles) * TKEYS;
+          const int nv8 = min(TKEYS, n_keys - g0) * 8;
+          const long long hoff = (long long)h * kHeadDim;
+          const long long row = (long long)d.H * kHeadDim;
+#pragma unroll 4
+          for (int u = lane; u < nv8; u += 32) {
+            const int c = u >> 3, ch = u & 7;
+            cp_async16(dk + (uint32_t)(c * 128 + ((ch ^ (c & 7)) << 4)),
+                       kg + (long long)tok_list[g0 + c] * row + hoff + ch * 8, true);
+          }
+          cp_async_mbar_arrive_noinc(bar(B_KF + s));
+#pragma unroll 4
+          for (int u = lane; u < nv8; u += 32) {
+            const int c = u >> 3, ch = u & 7;
+            cp_async16(dv + (uint32_t)(c * 128 + ((ch ^ (c & 7)) << 4)),
+                       vg + (long long)tok_list[g0 + c] * row + hoff + ch * 8, true);
+          }
+          cp_async_mbar_arrive_noinc(bar(B_VF + s));
         }
       }
+      __syncwarp();  // the token list is rebuilt for the next entry
+#pragma unroll
+      for (int u = 0; u < kMaxTopK / 32; ++u) ids_cur[u] = ids_nxt[u];
+      qs_cur = qs_nxt;
+      pair_cur = pair_nxt;
+      pair_nxt = pair_nn;
     }
+    cp_async_wait<0>();  // this lane's gathers have landed
     if (*abort_flag && lane == 0) {
       // let this CTA's own copies land before its shared memory goes away
       volatile int never = 0;
@@ -341,6 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             !mbar_wait(bar(B_PF + p_b), (g >> 1) & 1, abort_flag, err, d.wait_cycles))
           return false;
         fence_after_sync();
+        fence_proxy_async_smem();
         const uint32_t sv = sb + OFF_V + p_s * kKV;
         const uint32_t lbo = (sb + OFF_ONES) - sv;  // value dims, then the ones rows
         const uint32_t spt = sb + OFF_PT + p_b * kPT;
@@ -375,6 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           fence_after_sync();
+          fence_proxy_async_smem();  // the gathered rows were written by cp.async (generic proxy)
           const uint32_t sk = sb + OFF_K + s * kKV;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
@@ -416,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       const Entry& E = ent(es);
-      const int n = E.n_tiles, nk = E.n_kept, nsel = E.nsel;
+      const int n = E.n_tiles, nk = E.n_kept, n_keys = E.n_keys;
       const uint32_t qmask = E.qmask;
       // reference per query; the weight of the always-kept segment (1 when
       // its normalised state is supplied, scaled down with every raise of the
@@ -432,18 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < n; ++i, ++gt) {
         const int b = gt & 1;
         // is this lane's key a real key of the tile?
-        bool kvalid;
-        if (i < nk) {
-          kvalid = (long long)i * TKEYS + k < d.NK;
-        } else {
-          const int idx = (i - nk) * BPT + (k >> 4);
-          kvalid = false;
-          if (idx < nsel) {
-            const Blk kb = block_of(d, E.sel[idx]);
-            const int slot = k & 15;
-            kvalid = (slot >> 2) < kb.nr && (slot & 3) < kb.nc;
-          }
-        }
+        const bool kvalid = i < nk ? (long long)i * TKEYS + k < d.NK : (i - nk) * TKEYS + k < n_keys;
         // P^T buffer b is free once the O^T product of tile gt - 2 is complete;
         // S^T(gt) is in TMEM once its product is.  Both waits and the test for
         // a raise of the references are decided together by one OR barrier in
@@ -552,17 +647,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
       const int es = ne % NE;
       const uint32_t ph = (ne / NE) & 1;
-      const bool got = mbar_wait(bar(B_EF + es), ph, abort_flag, err, d.wait_cycles) &&
-                       mbar_wait(bar(B_EM + es), ph, abort_flag, err, d.wait_cycles) &&
+      // the entry is known once its info has landed: its global loads (the
+      // always-kept segment's outputs, the compressed output, the gate's
+      // inputs) are issued now, all at once, so that their latency overlaps
+      // the entry's products instead of following them one by one
+      if (bar_or(2, !mbar_wait(bar(B_EF + es), ph, abort_flag, err, d.wait_cycles))) {  // agreed on by all four warps
+        ok = false;
+        break;
+      }
+      const Entry& E = ent(es);
+      const int h = E.h, a = E.a;
+      const uint32_t qmask = E.qmask;
+      float osv[NQ];
+      float cmp = 0.f, zpart = 0.f;
+      if (dlane < 64) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+          osv[q] = (o_spec != nullptr && ((qmask >> q) & 1u))
+                       ? o_spec[((long long)E.tok[q] * d.H + h) * kHeadDim + dlane] : 0.f;
+        if (w != nullptr) {
+          cmp = oc[((long long)a * d.H + h) * kHeadDim + dlane];
+          zpart = qc32[((long long)a * d.H + h) * kHeadDim + dlane] * w[(long long)h * kHeadDim + dlane];
+        }
+      }
+      const bool got = mbar_wait(bar(B_EM + es), ph, abort_flag, err, d.wait_cycles) &&
                        mbar_wait(bar(B_OF + es), ph, abort_flag, err, d.wait_cycles);
-      if (bar_or(2, !got)) {  // agreed on by all four epilogue warps
+      if (bar_or(2, !got)) {
         ok = false;
         break;
       }
       fence_after_sync();
-      const Entry& E = ent(es);
-      const int h = E.h, a = E.a;
-      const uint32_t qmask = E.qmask;
       uint32_t ov[NQ];
       if (E.n_tiles > 0) {
         tmem_ld16(tbase + lane_off + TM_O + es * 16, ov);
@@ -575,27 +689,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < NQ; ++q) ls[q] = __uint_as_float(ov[q]);
       }
-      float g = 0.f;
       if (w != nullptr && dlane < 64) {
-        float z = qc32[((long long)a * d.H + h) * kHeadDim + dlane] * w[(long long)h * kHeadDim + dlane];
+        float z = zpart;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
         if (lane == 0) gz[q4] = z;
       }
       bar_sync128(2);
       if (dlane < 64) {
-        if (w != nullptr) g = 1.f / (1.f + expf(-(gz[0] + gz[1])));
-        const float* oca = oc != nullptr ? oc + ((long long)a * d.H + h) * kHeadDim : nullptr;
-        const float cmp = (w != nullptr) ? oca[dlane] : 0.f;
+        const float g = w != nullptr ? 1.f / (1.f + expf(-(gz[0] + gz[1]))) : 0.f;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           if (!((qmask >> q) & 1u)) continue;
           const long long t = E.tok[q];
           const float wq = E.wf[q];
           const float den = wq + ls[q];
-          float num = __uint_as_float(ov[q]);
-          if (o_spec != nullptr) num = fmaf(wq, o_spec[(t * d.H + h) * kHeadDim + dlane], num);
-          const float o = num / den;
+          const float o = fmaf(wq, osv[q], __uint_as_float(ov[q])) / den;
           const long long ob = t * row + (long long)h * kHeadDim + dlane;
           if (w != nullptr) {
             out[ob] = __float2bfloat16_rn(g * cmp + (1.f - g) * o);
@@ -635,8 +744,7 @@ cudaError_t launch_selected_tc(const Dims& d, const bf16* q, const bf16* k, cons
   const unsigned long long str5[4] = {128, rowb, (unsigned long long)d.Wp * rowb, (unsigned long long)d.L * rowb};
   const unsigned box5[5] = {64, 1, 4, 4, 1};
   const long long off = (long long)d.S * d.H * kHeadDim;
-  bool ok = make_tmap(&mp.q5, q + off, 5, dims5, str5, box5) && make_tmap(&mp.k5, k + off, 5, dims5, str5, box5) &&
-            make_tmap(&mp.v5, v + off, 5, dims5, str5, box5);
+  bool ok = make_tmap(&mp.q5, q + off, 5, dims5, str5, box5);
   const unsigned long long dims3[3] = {64, H, (unsigned long long)d.T};
   const unsigned long long str3[2] = {128, rowb};
   const unsigned box3[3] = {64, 1, 1};
@@ -660,7 +768,7 @@ cudaError_t launch_selected_tc(const Dims& d, const bf16* q, const bf16* k, cons
   const long long items = (long long)d.H * d.Tc;
   const long long grid = items < (long long)sms ? items : (long long)sms;
   if (grid <= 0) return cudaSuccess;
-  selected_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mp, d, sel, order, qc32, w, oc, out, lse,
+  selected_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, st>>>(mp, d, k, v, sel, order, qc32, w, oc, out, lse,
                                                                   o_spec, lse_spec, err, kept_inline);
   return cudaGetLastError();
 }

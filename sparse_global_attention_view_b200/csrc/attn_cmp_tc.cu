@@ -10,28 +10,32 @@
 //               stage refilled once its PV product is complete;
 //   warp 1      MMA issuer: S = Qc Kc^T with kind::tf32 from the fp32 means
 //               (the top-K ranking needs better than bf16 scores), into one of
-//               two TMEM score buffers, then O += P Vc (bf16, P from TMEM);
-//   warp 2      TMEM allocation (S at columns 0/128, O at 256, P at 320/384);
+//               three TMEM score buffers, then O += P Vc (bf16, P from TMEM);
+//   warp 2      TMEM allocation (S at columns 0/128/256, O at 384, P at 448);
 //   warps 4-7   softmax, one thread per query row;
 //   warps 8-11  streaming top-K, one thread per query row.
 // S(j+1) is computed while both warpgroups work on S(j): the softmax writes
-// P(j) to its own TMEM columns, so the raw scores stay readable until the
-// top-K warpgroup is done with them.  The softmax already forms the maxima of
-// the tile's eight 16-column groups; it compares them with each row's current
-// K-th best score (published in shared memory by the top-K thread) and hands
-// the top-K warp an 8-bit mask of the groups that may hold a candidate.  The
-// top-K warp reads from TMEM only the groups flagged for any of its 32 rows
-// and releases the score buffer after its last read, so once the heaps are
-// full most tiles cost it one mask load.  Candidates (columns that beat the
-// row's K-th best) go to a per-row buffer in shared memory; when any row's
-// buffer is half full the warp inserts all buffered candidates in lockstep
-// (one round of insertions serves every row) into the rows' heaps of K best
-// (score, block id) pairs; special entries are never ranked.  Once every heap
-// of the warp is full, a round is one predicated three-level replacement of
-// the root per lane (lanes without a candidate walk it without moving), with
-// the next round's candidate loaded during the current one: no lane diverges.  Columns arrive
-// in ascending block order and only a strictly larger score displaces the
-// root, so equal scores keep the lower id.  The softmax keeps eight
+// P(j) to its own TMEM columns (one buffer, rewritten once the P V product of
+// the tile before is complete), so the raw scores stay readable until the
+// top-K warpgroup is done with them; with three score buffers the top-K
+// warpgroup may trail the softmax by a tile without stalling the tensor core.
+// The softmax already forms the maxima of the tile's eight 16-column groups;
+// it compares them with each row's current K-th best score (published in
+// shared memory by the top-K thread) and hands the top-K warp an 8-bit mask
+// of the groups that may hold a candidate.  The top-K warp reads from TMEM
+// only the groups flagged for any of its 32 rows and releases the score
+// buffer after its last read.  Candidates (columns that beat the row's K-th
+// best) go to a per-row buffer in shared memory without branches (every
+// column is written to the next free slot, which is kept only for a
+// candidate); when any row's buffer is half full the warp inserts all
+// buffered candidates in lockstep (one round of insertions serves every row)
+// into the rows' heaps of K best (score, block id) pairs; special entries are
+// never ranked.  Once every heap of the warp is full, a round is one
+// predicated three-level replacement of the root per lane (lanes without a
+// candidate walk it without moving), with the next round's candidate loaded
+// during the current one: no lane diverges.  Columns arrive in ascending
+// block order and only a strictly larger score displaces the root, so equal
+// scores keep the lower id.  The softmax keeps eight
 // independent max and sum chains: one warp per sub-partition runs it, so
 // dependency latency, not throughput, is what it must avoid.
 #include <math_constants.h>
@@ -59,9 +63,11 @@ constexpr uint32_t OFF_HS = OFF_V + ST * kSub;       // heap keys [kMaxK][128] (
 constexpr uint32_t OFF_CS = OFF_HS + kMaxK * TQ * 8; // candidate scores [kBuf][128]
 constexpr uint32_t OFF_CC = OFF_CS + kBuf * TQ * 4;  // candidate entry indices
 constexpr uint32_t OFF_BAR = OFF_CC + kBuf * TQ * 4;
+constexpr int kCandGap = (int)((OFF_CC - OFF_CS) / 4);  // floats from a candidate's score to its index
 constexpr uint32_t OFF_TAU = OFF_BAR + 256;          // each row's K-th best score [128]
-constexpr uint32_t OFF_MASK = OFF_TAU + TQ * 4;      // candidate-group masks [2][128] bytes
-constexpr uint32_t OFF_MISC = OFF_MASK + 2 * TQ;
+constexpr int NS = 3;                                // TMEM score buffers
+constexpr uint32_t OFF_MASK = OFF_TAU + TQ * 4;      // candidate-group masks [NS][128] bytes
+constexpr uint32_t OFF_MISC = OFF_MASK + NS * TQ;
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
@@ -69,7 +75,7 @@ static_assert(kSmemBytes <= 232448, "shared memory per block");
 // is complete); MR: the softmax has published the candidate-group masks of
 // score buffer b.
 constexpr int B_Q = 0, B_KF = 1, B_VF = B_KF + ST, B_KE = B_VF + ST, B_VE = B_KE + ST,
-              B_SF = B_VE + ST, B_PF = B_SF + 2, B_SR = B_PF + 2, B_MR = B_SR + 2, B_OD = B_MR + 2,
+              B_SF = B_VE + ST, B_PF = B_SF + NS, B_SR = B_PF + 1, B_MR = B_SR + NS, B_OD = B_MR + NS,
               B_OF = B_OD + 1, B_DRAIN = B_OF + 1, B_COUNT = B_DRAIN + 1;
 static_assert(B_COUNT * 8 <= 256, "barrier area");
 constexpr uint32_t kCols = 512;
@@ -214,12 +220,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(B_KE + s), 1);
       mbar_init(bar(B_VE + s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NS; ++b) {
       mbar_init(bar(B_SF + b), 1);
-      mbar_init(bar(B_PF + b), TQ);
       mbar_init(bar(B_SR + b), TQ);  // top-K warpgroup is done with S buffer b
       mbar_init(bar(B_MR + b), TQ);
     }
+    mbar_init(bar(B_PF), TQ);
     mbar_init(bar(B_OD), 1);
     mbar_init(bar(B_OF), 1);
     mbar_init(bar(B_DRAIN), 1);
@@ -303,25 +309,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_s(0, 0);
       }
       for (int j = 0; ok && j < nt; ++j) {
-        const int s = j % ST, b = j & 1;
+        const int s = j % ST;
         if (j + 1 < nt) {
-          const int s1 = (j + 1) % ST;
+          const int s1 = (j + 1) % ST, b1 = (j + 1) % NS;
           ok = mbar_wait(bar(B_KF + s1), ((j + 1) / ST) & 1, abort_flag, err, d.wait_cycles);
-          // S(j+1) reuses the buffer of S(j-1): the top-K warpgroup must have read it
-          if (ok && j >= 1) ok = mbar_wait(bar(B_SR + (b ^ 1)), (((j + 1) >> 1) - 1) & 1, abort_flag, err, d.wait_cycles);
+          // S(j+1) reuses the buffer of S(j+1-NS): the top-K warpgroup must
+          // have read it (the softmax has: PV(j-1) waited for its P)
+          if (ok && j + 1 >= NS)
+            ok = mbar_wait(bar(B_SR + b1), (((j + 1) / NS) - 1) & 1, abort_flag, err, d.wait_cycles);
           if (!ok) break;
           fence_after_sync();
-          issue_s(s1, b ^ 1);
+          issue_s(s1, b1);
         }
-        // (the softmax's arrival on PF(b) also says it has read S(j) from buffer b)
-        ok = (cp.scores_only || mbar_wait(bar(B_VF + s), (j / ST) & 1, abort_flag, err, d.wait_cycles)) &&
-             mbar_wait(bar(B_PF + b), (j >> 1) & 1, abort_flag, err, d.wait_cycles);
+        if (cp.scores_only) continue;
+        // P(j) is in TMEM once the softmax has arrived on PF
+        ok = mbar_wait(bar(B_VF + s), (j / ST) & 1, abort_flag, err, d.wait_cycles) &&
+             mbar_wait(bar(B_PF), j & 1, abort_flag, err, d.wait_cycles);
         if (!ok) break;
         fence_after_sync();
-        if (cp.scores_only) continue;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tbase + 256, tbase + 320 + b * 64 + kk * 8, sdesc_mn(sV + s * kSub + kk * 2048), id_pv,
+          mma_bf16_ts(tbase + 384, tbase + 448 + kk * 8, sdesc_mn(sV + s * kSub + kk * 2048), id_pv,
                       (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(bar(B_OD));
         mma_commit(bar(B_VE + s));
@@ -340,19 +348,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t o_addr = tbase + lane_off + 256;
+    const uint32_t o_addr = tbase + lane_off + 384;
     const float c2 = d.scale_log2;
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
-      const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + b), (j >> 1) & 1, abort_flag, err, d.wait_cycles))) {
+      const int b = j % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_SF + b), (j / NS) & 1, abort_flag, err, d.wait_cycles))) {
         ok = false;
         break;
       }
       fence_after_sync();
       const uint32_t s_addr = tbase + lane_off + b * 128;
-      const uint32_t p_addr = tbase + lane_off + 320 + b * 64;
+      const uint32_t p_addr = tbase + lane_off + 448;
       const long long rem = n_k - (long long)j * TK;
       // all 128 scores in one round of TMEM loads: the softmax is bound by
       // TMEM load latency, so a second round would cost as much as the first
@@ -389,9 +397,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(B_MR + b));
       }
       if (cp.scores_only) {
-        // ranking pass: no attention; S(j) has been read
-        fence_before_sync();
-        mbar_arrive(bar(B_PF + b));
+        // ranking pass: no attention (the top-K warpgroup's release of the
+        // buffer also says this warpgroup has read it: it follows MR)
         continue;
       }
       const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
@@ -423,6 +430,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = mxs;
         }
       }
+      // P has one TMEM buffer: the P V product of the previous tile must be
+      // complete before it is overwritten
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(bar(B_OD), (j - 1) & 1, abort_flag, err, d.wait_cycles))) {
+        ok = false;
+        break;
+      }
       float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -439,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       fence_before_sync();
-      mbar_arrive(bar(B_PF + b));
+      mbar_arrive(bar(B_PF));
     }
     if (ok && !cp.scores_only) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OF), 0, abort_flag, err, d.wait_cycles));
     if (ok && !cp.scores_only) {
@@ -479,7 +492,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     int nb = 0;  // candidates waiting in this row's buffer
     // Insert the buffered candidates.  All lanes run this together, so one
     // round of insertions serves every row of the warp at once.
-    const float inv_e = 1.f / (float)E;
+    // entry e -> frame f = e / E, position i = e - f E on the integer pipe
+    // (a float quotient would queue its conversions behind the softmax's
+    // exponentials): with m = floor((2^32 - 1) / E), hi32(e m) is e / E or
+    // one less for every e < 2^31
+    const uint32_t e_magic = 0xffffffffu / (uint32_t)E;
+    auto decode = [&](int e, int& f, int& i) {
+      f = (int)__umulhi((uint32_t)e, e_magic);
+      i = e - f * E;
+      if (i >= E) i -= E, ++f;
+    };
     auto flush = [&]() {
       if (__all_sync(0xffffffffu, top.cnt == d.K)) {
         // every heap of the warp is full: one predicated replacement per round
@@ -493,10 +515,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the next round's candidate is read while this one is inserted
           v_next = n + 1 < nb ? cb_s[(n + 1) * TQ + r] : -CUDART_INF_F;
           e_next = n + 1 < nb ? cb_e[(n + 1) * TQ + r] : 0;
-          int f = (int)((float)e * inv_e);
-          int i = e - f * E;
-          if (i < 0) i += E, --f;
-          if (i >= E) i -= E, ++f;
+          int f, i;
+          decode(e, f, i);
           const int id = f * Bf + (i - S);
           const unsigned long long key = pair_key(v, id);
           const bool take = have && v > top.tau && i >= S && id >= B0 && key < ub;
@@ -509,12 +529,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int n = 0; n < nb; ++n) {
         const float v = cb_s[n * TQ + r];
         if (!(v > top.tau)) continue;
-        // entry e -> frame f, position i; the float quotient is off by at most one
-        const int e = cb_e[n * TQ + r];
-        int f = (int)((float)e * inv_e);
-        int i = e - f * E;
-        if (i < 0) i += E, --f;
-        if (i >= E) i -= E, ++f;
+        int f, i;
+        decode(cb_e[n * TQ + r], f, i);
         // special entries are never ranked, nor blocks below B0 (frame 0 when
         // it is kept whole)
         if (i >= S && f * Bf + (i - S) >= B0) {
@@ -529,30 +545,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // beat the row's K-th best; the warp only scans groups where some of its
     // rows has one.
     auto group = [&](const uint32_t (&g)[16], int q, int e0, int lim) {
-      float v[16];
+      // branch-free appends: every column is written to the row's next free
+      // slot and the slot is kept only when the column is a candidate (the
+      // buffer has room for 16 more, so the writes stay inside it)
+      const float tau = top.tau;
+      const int n_in = lim - 16 * q;  // columns of the group inside the sequence
+      const int cbase = e0 + 16 * q;
+      float* ps = cb_s + nb * TQ + r;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        v[i] = (16 * q + i < lim) ? __uint_as_float(g[i]) : -CUDART_INF_F;
-      float m[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) m[u] = fmaxf(fmaxf(v[u], v[u + 4]), fmaxf(v[u + 8], v[u + 12]));
-      const float m16 = fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-      if (__any_sync(0xffffffffu, m16 > top.tau)) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          if (v[i] > top.tau) {
-            cb_s[nb * TQ + r] = v[i];
-            cb_e[nb * TQ + r] = e0 + 16 * q + i;
-            ++nb;
-          }
-        }
-        if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush();
+      for (int i = 0; i < 16; ++i) {
+        const float v = __uint_as_float(g[i]);
+        const bool c = v > tau && i < n_in;
+        ps[0] = v;
+        ps[kCandGap] = __int_as_float(cbase + i);
+        ps += c ? TQ : 0;
+        nb += c ? 1 : 0;
       }
+        if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush();
     };
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
-      const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MR + b), (j >> 1) & 1, abort_flag, err, d.wait_cycles))) {
+      const int b = j % NS;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_MR + b), (j / NS) & 1, abort_flag, err, d.wait_cycles))) {
         ok = false;
         break;
       }

@@ -54,6 +54,7 @@ constexpr int ST = 2;
 constexpr int kThreads = 384;
 constexpr int kMaxK = kFusedTopK;  // heap capacity per row
 constexpr int kBuf = 32;         // candidate buffer entries per row
+constexpr int kKeep = 12;        // candidates a row may keep buffered after a flush (<= kBuf - 16)
 constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16) tile: 16 KB
 
 constexpr uint32_t OFF_Q = 0;                        // 2 sub-tiles (d 0-31, 32-63)
@@ -502,19 +503,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       i = e - f * E;
       if (i >= E) i -= E, ++f;
     };
-    auto flush = [&]() {
+    auto flush = [&](int keep) {
       if (__all_sync(0xffffffffu, top.cnt == d.K)) {
-        // every heap of the warp is full: one predicated replacement per round
-        const int rounds = (int)__reduce_max_sync(0xffffffffu, (unsigned)nb);
-        float v_next = nb > 0 ? cb_s[r] : -CUDART_INF_F;
-        int e_next = nb > 0 ? cb_e[r] : 0;
+        // every heap of the warp is full: one predicated replacement per
+        // round, each row taking its newest candidate, until no row holds
+        // more than `keep` (the order of insertion does not change the K
+        // largest keys, and a row that keeps a few candidates keeps its lane
+        // busy in the next flush's rounds)
+        const int rounds = max(0, (int)__reduce_max_sync(0xffffffffu, (unsigned)nb) - keep);
+        float v_next = nb > 0 ? cb_s[(nb - 1) * TQ + r] : -CUDART_INF_F;
+        int e_next = nb > 0 ? cb_e[(nb - 1) * TQ + r] : 0;
         for (int n = 0; n < rounds; ++n) {
-          const bool have = n < nb;
+          const bool have = nb > 0;
           const float v = v_next;
           const int e = e_next;
+          nb -= have ? 1 : 0;
           // the next round's candidate is read while this one is inserted
-          v_next = n + 1 < nb ? cb_s[(n + 1) * TQ + r] : -CUDART_INF_F;
-          e_next = n + 1 < nb ? cb_e[(n + 1) * TQ + r] : 0;
+          v_next = nb > 0 ? cb_s[(nb - 1) * TQ + r] : -CUDART_INF_F;
+          e_next = nb > 0 ? cb_e[(nb - 1) * TQ + r] : 0;
           int f, i;
           decode(e, f, i);
           const int id = f * Bf + (i - S);
@@ -522,7 +528,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool take = have && v > top.tau && i >= S && id >= B0 && key < ub;
           top.replace_root(key, take);
         }
-        nb = 0;
         tau_s[r] = top.tau;
         return;
       }
@@ -561,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ps += c ? TQ : 0;
         nb += c ? 1 : 0;
       }
-        if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush();
+      if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush(kKeep);
     };
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -595,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(bar(B_SR + b));
       }
     }
-    if (__all_sync(0xffffffffu, ok)) flush();
+    if (__all_sync(0xffffffffu, ok)) flush(0);
     const long long row = m0 + r;
     if (ok && row < d.Tc && cp.root != nullptr)
       cp.root[(long long)h * d.Tc + row] = top.cnt == d.K ? top.at(0) : 0ull;

@@ -54,7 +54,7 @@ constexpr int ST = 2;
 constexpr int kThreads = 384;
 constexpr int kMaxK = kFusedTopK;  // heap capacity per row
 constexpr int kBuf = 32;         // candidate buffer entries per row
-constexpr int kKeep = 12;        // candidates a row may keep buffered after a flush (<= kBuf - 16)
+constexpr int kKeep = 20;        // candidates a row may keep buffered after a flush (<= kBuf - 8)        // candidates a row may keep buffered after a flush (<= kBuf - 16)
 constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16) tile: 16 KB
 
 constexpr uint32_t OFF_Q = 0;                        // 2 sub-tiles (d 0-31, 32-63)
@@ -68,7 +68,7 @@ constexpr int kCandGap = (int)((OFF_CC - OFF_CS) / 4);  // floats from a candida
 constexpr uint32_t OFF_TAU = OFF_BAR + 256;          // each row's K-th best score [128]
 constexpr int NS = 3;                                // TMEM score buffers
 constexpr uint32_t OFF_MASK = OFF_TAU + TQ * 4;      // candidate-group masks [NS][128] bytes
-constexpr uint32_t OFF_MISC = OFF_MASK + NS * TQ;
+constexpr uint32_t OFF_MISC = OFF_MASK + NS * TQ * 2;
 constexpr uint32_t kSmemBytes = OFF_MISC + 64 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory per block");
 
@@ -193,6 +193,18 @@ __device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
                : "memory");
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld8(uint32_t (&r)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+               :
+               : "memory");
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_cmp_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const Dims d, float* __restrict__ oc,
@@ -234,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   volatile float* tau_s = reinterpret_cast<volatile float*>(sp + OFF_TAU);
-  volatile uint8_t* mask_s = sp + OFF_MASK;
+  volatile uint16_t* mask_s = reinterpret_cast<volatile uint16_t*>(sp + OFF_MASK);
   if (tid < TQ) tau_s[tid] = -CUDART_INF_F;
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), kCols);
@@ -379,13 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the maxima of the eight 16-column groups: eight independent chains keep
       // the single softmax warp of each sub-partition from stalling on one
       // 128-long dependency chain
-      float mq[8];
+      float mq[16];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) mq[q] = __uint_as_float(sv[q >> 1][(q & 1) * 16]);
+      for (int q = 0; q < 16; ++q) mq[q] = __uint_as_float(sv[q >> 2][(q & 3) * 8]);
 #pragma unroll
-      for (int i = 1; i < 16; ++i)
+      for (int i = 1; i < 8; ++i)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) mq[q] = fmaxf(mq[q], __uint_as_float(sv[q >> 1][(q & 1) * 16 + i]));
+        for (int q = 0; q < 16; ++q) mq[q] = fmaxf(mq[q], __uint_as_float(sv[q >> 2][(q & 3) * 8 + i]));
       {
         // tell the top-K warp which groups may hold a candidate for this row:
         // those whose maximum beats the row's K-th best so far (a stale, lower
@@ -393,8 +405,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float tau = tau_s[r];
         uint32_t msk = 0;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) msk |= (mq[q] > tau ? 1u : 0u) << q;
-        mask_s[b * TQ + r] = (uint8_t)msk;
+        for (int q = 0; q < 16; ++q) msk |= (mq[q] > tau ? 1u : 0u) << q;
+        mask_s[b * TQ + r] = (uint16_t)msk;
         mbar_arrive(bar(B_MR + b));
       }
       if (cp.scores_only) {
@@ -402,6 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // buffer also says this warpgroup has read it: it follows MR)
         continue;
       }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mq[q] = fmaxf(mq[q], mq[q + 8]);
       const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
                              fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
@@ -549,16 +563,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // One 16-column group of the score tile: candidates are the columns that
     // beat the row's K-th best; the warp only scans groups where some of its
     // rows has one.
-    auto group = [&](const uint32_t (&g)[16], int q, int e0, int lim) {
+    auto group = [&](const uint32_t (&g)[8], int q, int e0, int lim) {
       // branch-free appends: every column is written to the row's next free
       // slot and the slot is kept only when the column is a candidate (the
       // buffer has room for 16 more, so the writes stay inside it)
       const float tau = top.tau;
-      const int n_in = lim - 16 * q;  // columns of the group inside the sequence
-      const int cbase = e0 + 16 * q;
+      const int n_in = lim - 8 * q;  // columns of the group inside the sequence
+      const int cbase = e0 + 8 * q;
       float* ps = cb_s + nb * TQ + r;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < 8; ++i) {
         const float v = __uint_as_float(g[i]);
         const bool c = v > tau && i < n_in;
         ps[0] = v;
@@ -566,7 +580,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ps += c ? TQ : 0;
         nb += c ? 1 : 0;
       }
-      if (__any_sync(0xffffffffu, nb > kBuf - 16)) flush(kKeep);
+      if (__any_sync(0xffffffffu, nb > kBuf - 8)) flush(kKeep);
     };
     bool ok = true;
     for (int j = 0; j < nt; ++j) {
@@ -585,9 +599,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (G != 0) {
         const int q = __ffs(G) - 1;
         G &= G - 1;
-        uint32_t g[16];
-        tmem_ld16(s_addr + 16 * q, g);
-        tmem_wait_ld16(g);
+        uint32_t g[8];
+        tmem_ld8(s_addr + 8 * q, g);
+        tmem_wait_ld8(g);
         if (G == 0) {
           fence_before_sync();
           mbar_arrive(bar(B_SR + b));  // the tensor core may overwrite this buffer now

@@ -353,6 +353,16 @@ gsa_status gsa_noalloc_check_device_error(void* stream);
  * they are cleared with the error word. */
 gsa_status gsa_check_device_error(void* ws, void* stream);
 
+/* Self-test of the exponential the attention kernels' softmax takes on the
+ * FMA pipe for a quarter of its terms (2^x by range reduction and a cubic, a
+ * relative error below 7.5e-5 on [-125, 0], the clamp at -125 included):
+ *   y[i] = that 2^x[i] for i < n, computed on the device as the softmax does
+ *   (two lanes per instruction).
+ * x, y: device float arrays of n elements (y written, x read), launched on
+ * `stream`; GSA_ERR_INVALID_ARG for n < 0 or a NULL array with n > 0.  Not part of the
+ * attention path: for tests that compare it with the exact 2^x. */
+gsa_status gsa_selftest_exp2(const float* x, float* y, int64_t n, void* stream);
+
 /* Static text for a status code. */
 const char* gsa_status_string(gsa_status status);
 

@@ -9,6 +9,7 @@ from .api import (  # noqa: F401
     GsaLayer,
     Shape,
     check_device_error,
+    selftest_exp2,
     compressed_attn,
     dense_global_attn,
     dense_global_attn_mma,

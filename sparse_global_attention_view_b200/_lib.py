@@ -95,6 +95,7 @@ SIGNATURES = {
     "gsa_forward_noalloc": [P_SHAPE] + [c_vp] * 6,
     "gsa_noalloc_check_device_error": [c_vp],
     "gsa_check_device_error": [c_vp, c_vp],
+    "gsa_selftest_exp2": [c_vp, c_vp, ctypes.c_int64, c_vp],
     "gsa_status_string": [c_i32],
     "gsa_last_cuda_error": [],
     "gsa_cuda_error_name": [c_i32],

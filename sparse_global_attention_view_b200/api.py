@@ -284,6 +284,13 @@ def workspace_view(ws, shape, name: str) -> torch.Tensor:
     return ws[off:off + nbytes].view(dtype).view(shp)
 
 
+def selftest_exp2(x, y, stream=None) -> None:
+    """y[i] = the softmax's FMA-pipe 2^x[i] on the device (gsa_selftest_exp2); x, y cuda float32."""
+    n = x.numel()
+    check(load().gsa_selftest_exp2(_ptr(x, torch.float32, n, "x"), _ptr(y, torch.float32, n, "y"), n, _stream(stream)),
+          "gsa_selftest_exp2")
+
+
 def check_device_error(ws, stream=None) -> None:
     """Raise GsaError if a kernel set the workspace's error word (then cleared).
     A timeout's message carries where the first wait ran out (header words 1-2:

@@ -42,19 +42,28 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // cubic fitted to 2^f on that interval by iteratively reweighted least squares
 // on Chebyshev nodes (max relative error 7.5e-5 in fp32, below the bf16
 // rounding of P).  x is clamped at -125 (the result is then ~2^-125, i.e. 0 for
-// the softmax).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const int j = __float_as_int(t) - 0x4B400000;
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.055171769f, f, 0.24261113f);
-  p = fmaf(p, f, 0.69326097f);
-  p = fmaf(p, f, 0.99992806f);
-  return __int_as_float(__float_as_int(p) + (j << 23));
+// the softmax).  Both halves of a pair are computed with the paired forms of
+// the additions and multiply-adds.
+__device__ __forceinline__ uint64_t exp2_fma2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t big = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(x, big);
+  float t0, t1;
+  f2_unpack(t, t0, t1);
+  const uint64_t f = f2_sub(x, f2_sub(t, big));
+  uint64_t p = f2_fma(f2_pack(0.055171769f, 0.055171769f), f, f2_pack(0.24261113f, 0.24261113f));
+  p = f2_fma(p, f, f2_pack(0.69326097f, 0.69326097f));
+  p = f2_fma(p, f, f2_pack(0.99992806f, 0.99992806f));
+  float p0, p1;
+  f2_unpack(p, p0, p1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + ((__float_as_int(t0) - 0x4B400000) << 23)),
+                 __int_as_float(__float_as_int(p1) + ((__float_as_int(t1) - 0x4B400000) << 23)));
 }
 
 
+constexpr int kPolyOf8 = 2;        // exponential pairs of every eight taken on the FMA pipe
 constexpr int TQ = 128;            // rows per query tile
 constexpr int NQT = 2;             // query tiles per CTA
 constexpr int TK = 128;            // keys per key tile
@@ -252,12 +261,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
       // eight independent max / sum chains: each softmax warp owns whole rows,
-      // so a single 128-long dependency chain would leave it stalled
+      // so a single 128-long dependency chain would leave it stalled; a
+      // three-input maximum takes two columns per instruction
+      auto sval = [&](int k) -> float { return __uint_as_float(sv[k >> 5][k & 31]); };
       float mq[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mq[u] = __uint_as_float(sv[0][u]);
+      for (int u = 0; u < 8; ++u) mq[u] = fmaxf(sval(u), sval(u + 8));
 #pragma unroll
-      for (int k = 8; k < 128; ++k) mq[k & 7] = fmaxf(mq[k & 7], __uint_as_float(sv[k >> 5][k & 31]));
+      for (int k = 16; k < 128; k += 16)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mq[u] = fmax3(mq[u], sval(k + u), sval(k + 8 + u));
       const float mx = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])),
                              fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
       const float mxs = mx * c2;
@@ -284,22 +297,38 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_used = mxs;
         }
       }
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // the scaled, shifted scores two at a time; one pair in four takes its
+      // exponentials on the FMA pipe; four paired sum chains
+      const uint64_t c2p = f2_pack(c2, c2), nmp = f2_pack(-m_used, -m_used);
+      uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
-          const float x1 = fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used);
-          const float p1 = (i & 1) ? exp2_fma(x1) : fast_exp2(x1);  // one in four on the FMA pipe
-          ps[i & 7] += p0 + p1;
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[c][2 * i]), __uint_as_float(sv[c][2 * i + 1])), c2p, nmp);
+          uint64_t p2;
+          if ((i & 7) >= 8 - kPolyOf8) {
+            p2 = exp2_fma2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(fast_exp2(x0), fast_exp2(x1));
+          }
+          ps2[i & 3] = f2_add(ps2[i & 3], p2);
+          float p0, p1;
+          f2_unpack(p2, p0, p1);
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(s_addr + 16 * c, pk);
       }
       tmem_wait_st();
-      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      {
+        const uint64_t s01 = f2_add(f2_add(ps2[0], ps2[1]), f2_add(ps2[2], ps2[3]));
+        float lo, hi;
+        f2_unpack(s01, lo, hi);
+        l += lo + hi;
+      }
       fence_before_sync();
       mbar_arrive(bar(B_PF + t));
     }
@@ -373,6 +402,25 @@ EncodeTiledFn encode_fn() {
 }
 
 }  // namespace
+
+namespace {
+__global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restrict__ y, long long n) {
+  const long long i = 2 * ((long long)blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const bool two = i + 1 < n;
+  float r0, r1;
+  f2_unpack(exp2_fma2(f2_pack(x[i], two ? x[i + 1] : 0.f)), r0, r1);
+  y[i] = r0;
+  if (two) y[i + 1] = r1;
+}
+}  // namespace
+
+cudaError_t launch_exp2_selftest(const float* x, float* y, long long n, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  const long long pairs = (n + 1) / 2;
+  exp2_selftest_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, st>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 // 3-D tiled map over bf16 or fp32 data; dims/strides innermost first, strides in bytes.
 bool make_tmap_3d(CUtensorMap* m, bool fp32, const void* base, unsigned long long d0,

@@ -591,6 +591,11 @@ gsa_status gsa_workspace_offsets(const gsa_shape* shape, gsa_ws_offsets* out) {
   return GSA_OK;
 }
 
+gsa_status gsa_selftest_exp2(const float* x, float* y, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (x == nullptr || y == nullptr))) return GSA_ERR_INVALID_ARG;
+  return cuda_status(gsa::launch_exp2_selftest(x, y, (long long)n, as_stream(stream)));
+}
+
 gsa_status gsa_check_device_error(void* ws, void* stream) {
   if (!dev_ptr(ws)) return GSA_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);

@@ -52,6 +52,8 @@ struct AttnTcArgs {
 };
 cudaError_t launch_attn_tc(const AttnTcArgs& a, const bf16* q, const bf16* k, const bf16* v,
                            long long kv_rows, cudaStream_t st);
+// y[i] = the attention softmax's FMA-pipe 2^x of x[i] (self-test of that path).
+cudaError_t launch_exp2_selftest(const float* x, float* y, long long n, cudaStream_t st);
 
 // 3-D tiled TMA map (128-byte swizzle) over bf16 or fp32 data; dims and
 // strides innermost first, strides in bytes.  False if the driver refuses it.

@@ -331,7 +331,7 @@ def job_value(world: int, tokens_per_rank: int, step_ms_max: float, parallel: st
 
 
 STAGE_SOURCE = {"pool": "pool.cu", "compressed_attn": "attn_cmp_tc.cu", "block_scores": "topk.cu",
-                "topk_merge": "topk.cu", "kept_attn": "attn_tc.cu", "selected_gate": "selected.cu"}
+                "topk_merge": "topk.cu", "kept_attn": "attn_tc.cu", "selected_gate": "selected_tc.cu"}
 
 
 def main() -> None:
@@ -478,6 +478,12 @@ def main() -> None:
         stages[name] = {"ms": round(ms, 4), "share": round(ms / sum(stage_ms.values()), 4), "bound": bound,
                         "achieved": round(ach, 2), "peak": round(peak, 1), "unit": u,
                         "frac": round(ach / peak, 4)}
+        dram = recorded_traffic(STAGE_SOURCE[name], wl.name)
+        if dram:
+            # DRAM bytes of one launch (committed ncu counters of this source)
+            # against the measured HBM copy bandwidth
+            stages[name]["dram_bytes"] = dram
+            stages[name]["dram_frac"] = round(dram / (ms / 1e3) / 1e9 / P["hbm_gbs"], 4)
         if name == "selected_gate":
             stages[name]["note"] = ("achieved = K/V bytes of the valid tokens of the selected blocks "
                                     f"({amount / 1e9:.1f} GB, counted from this run's selection) per second, "

@@ -20,7 +20,20 @@ struct Dims {
   float scale;       // softmax scale
   float scale_log2;  // scale * log2(e)
   long long wait_cycles;  // limit of the in-kernel waits of one role on another
+  // floor((2^32 - 1) / x) for x = E, Bf, Bw, Tc: quotients by these on the
+  // integer pipe (udiv31)
+  uint32_t mE, mBf, mBw, mTc;
 };
+
+// floor(n / x) for 0 <= n < 2^31 and 1 <= x < 2^31, from m = floor((2^32 - 1) / x):
+// hi32(n m) is the quotient or one less (n m / 2^32 > n / x - 2n / 2^32 > n / x - 1),
+// so one correction step is exact.  Avoids the float reciprocal of a general
+// integer division, whose conversions share a pipe with the exponentials.
+__device__ __forceinline__ int udiv31(int n, int x, uint32_t m) {
+  int q = (int)__umulhi((uint32_t)n, m);
+  if (n - q * x >= x) ++q;
+  return q;
+}
 
 // Bits of the device error word (first word of every workspace).
 enum : unsigned { kErrTimeout = 1u, kErrDeviceCheck = 2u };

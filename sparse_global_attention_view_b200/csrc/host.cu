@@ -64,6 +64,10 @@ gsa_status make_dims(const gsa_shape* s, Dims* d, gsa_sizes* z) {
   t.scale_log2 = t.scale * 1.4426950408889634f;
   // SM clocks stay below 2 GHz: two cycles per nanosecond is at least the time asked
   t.wait_cycles = s->wait_limit_ns > 0 ? 2LL * s->wait_limit_ns : 4000000000LL;
+  t.mE = 0xffffffffu / (uint32_t)(E > 0 ? E : 1);
+  t.mBf = 0xffffffffu / (uint32_t)(Bf > 0 ? Bf : 1);
+  t.mBw = 0xffffffffu / (uint32_t)(Bw > 0 ? Bw : 1);
+  t.mTc = 0xffffffffu / (uint32_t)(Tc > 0 ? Tc : 1);
   if (d) *d = t;
   if (z) {
     z->T = T;

@@ -21,9 +21,11 @@
 // 4 x 4 patches over a per-frame view of the token grid.
 //
 // One CTA per SM works through (head, entry) pairs; 12 warps:
-//   warp 0      producer: per entry its queries (one TMA box) and its packed
-//               token list (from the selection, loaded one entry ahead), then
-//               per 128-key tile the K and V rows by cp.async into a 5-stage
+//   warp 0      builder: per entry its queries (one TMA box) and its packed
+//               token list (from the selection, loaded one entry ahead) into
+//               one of two list buffers;
+//   warp 3      gather warp: per entry, once its list is handed over, the K
+//               and V rows of every 128-key tile by cp.async into a 5-stage
 //               ring; when the always-kept tokens are not supplied as a
 //               finished softmax state, their head-major copies are streamed
 //               first as plain 128-key TMA tiles;
@@ -79,8 +81,9 @@ constexpr uint32_t OFF_Q = OFF_ONES + kKV;
 constexpr uint32_t OFF_PT = OFF_Q + NE * kQ;
 constexpr uint32_t OFF_ENT = OFF_PT + 2 * kPT;
 constexpr uint32_t kEntBytes = (sizeof(Entry) + 127) / 128 * 128;
-constexpr uint32_t OFF_TOK = OFF_ENT + NE * kEntBytes;   // the producer's token list of one entry
-constexpr uint32_t OFF_RED = OFF_TOK + kMaxTopK * NQ * 4;  // [4 warps][16] per-query partial maxima
+constexpr int kTokList = kMaxTopK * NQ;                  // key slots of one entry at most
+constexpr uint32_t OFF_TOK = OFF_ENT + NE * kEntBytes;   // two token lists (builder -> gather warp)
+constexpr uint32_t OFF_RED = OFF_TOK + 2 * kTokList * 4;  // [4 warps][16] per-query partial maxima
 constexpr uint32_t OFF_LS = OFF_RED + 4 * NQ * 4;        // [16] sums of P (epilogue)
 constexpr uint32_t OFF_GATE = OFF_LS + NQ * 4;           // [2] gate partial dot products
 constexpr uint32_t OFF_BAR = (OFF_GATE + 16 + 255) / 256 * 256;
@@ -92,7 +95,8 @@ static_assert(kSmemBytes <= 232448, "shared memory per block");
 // barriers
 constexpr int B_EF = 0, B_EE = B_EF + NE, B_EM = B_EE + NE, B_KF = B_EM + NE, B_VF = B_KF + ST,
               B_KE = B_VF + ST, B_VE = B_KE + ST, B_SF = B_VE + ST, B_PF = B_SF + 2, B_PE = B_PF + 2,
-              B_OF = B_PE + 2, B_OD = B_OF + NE, B_DRAIN = B_OD + 1, B_COUNT = B_DRAIN + 1;
+              B_OF = B_PE + 2, B_OD = B_OF + NE, B_DRAIN = B_OD + 1, B_TF = B_DRAIN + 1, B_TE = B_TF + 2,
+              B_COUNT = B_TE + 2;
 static_assert(B_COUNT * 8 <= 512, "barrier area");
 
 constexpr uint32_t kCols = 128;  // TMEM: S^T at 0 / 16, O^T at 32 + 16 e (e < NE)
@@ -132,9 +136,9 @@ struct Blk {
 };
 __device__ __forceinline__ Blk block_of(const Dims& d, int beta) {
   Blk b;
-  b.f = beta / d.Bf;
+  b.f = udiv31(beta, d.Bf, d.mBf);
   const int j = beta - b.f * d.Bf;
-  const int br = j / d.Bw, bc = j - br * d.Bw;
+  const int br = udiv31(j, d.Bw, d.mBw), bc = j - br * d.Bw;
   b.r0 = br * d.P;
   b.c0 = bc * d.P;
   b.nr = min(d.P, d.Hp - b.r0);
@@ -188,6 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(bar(B_OD), 1);
     mbar_init(bar(B_DRAIN), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(B_TF + b), 32);  // token list b written (every builder lane)
+      mbar_init(bar(B_TE + b), 32);  // token list b read (every gather lane)
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -220,7 +228,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&mp.q5);
       prefetch_tmap(&mp.q3);
     }
-    int* tok_list = reinterpret_cast<int*>(sp + OFF_TOK);
     const int KU = (d.K + 31) / 32;  // ids per lane
     // the selection and the pair of an entry are loaded one entry ahead, so
     // their latency overlaps the gathers of the entry before
@@ -236,9 +243,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto query_slot = [&](long long pair) -> QSlot {
       QSlot r{-1, -CUDART_INF_F};
       if (pair < 0 || lane >= NQ) return r;
-      const int h = (int)(pair / d.Tc);
+      const int h = pair < 0x7fffffffLL ? udiv31((int)pair, (int)d.Tc, d.mTc) : (int)(pair / d.Tc);
       const int a = (int)(pair - (long long)h * d.Tc);
-      const int f = a / d.E, j = a - (a / d.E) * d.E;
+      const int f = udiv31(a, d.E, d.mE), j = a - f * d.E;
       if (j < d.S) {
         if (lane == 0) r.t = (long long)f * d.L + j;
       } else {
@@ -258,8 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ids_cur[u] = (u < KU && k < d.K && pair_cur >= 0) ? sel[pair_cur * d.K + k] : -1;
     }
     QSlot qs_cur = query_slot(pair_cur);
-    int gt = 0;  // tiles loaded
-    int ne = 0;  // entries loaded
+    int ne = 0;  // entries built
     bool ok = true;
     for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
       const int es = ne % NE;
@@ -272,12 +278,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const QSlot qs_nxt = query_slot(pair_nxt);
       const long long pair_nn = pair_of(it + 2LL * gridDim.x);
-      if (ne >= NE && !__all_sync(0xffffffffu, mbar_wait(bar(B_EE + es), ((ne / NE) - 1) & 1, abort_flag, err, d.wait_cycles))) {
+      // the entry slot is free once the epilogue is done with it; the token
+      // list buffer once the gather warp has read it
+      const int lb = ne & 1;
+      if ((ne >= NE && !__all_sync(0xffffffffu, mbar_wait(bar(B_EE + es), ((ne / NE) - 1) & 1, abort_flag, err, d.wait_cycles))) ||
+          (ne >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(B_TE + lb), ((ne >> 1) - 1) & 1, abort_flag, err, d.wait_cycles)))) {
         ok = false;
         break;
       }
+      int* tok_list = reinterpret_cast<int*>(sp + OFF_TOK) + lb * kTokList;
       const long long pair = pair_cur;
-      const int h = (int)(pair / d.Tc);
+      const int h = pair < 0x7fffffffLL ? udiv31((int)pair, (int)d.Tc, d.mTc) : (int)(pair / d.Tc);
       const int a = (int)(pair - (long long)h * d.Tc);
       Entry& E = ent(es);
       // the selection: ascending ids, -1 padded; an id outside [0, NB) ends the
@@ -330,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int n_keys = carry;
       const int n_tiles = n_kept_tiles + (n_keys + TKEYS - 1) / TKEYS;
       // the entry's queries (tokens and references prefetched with the selection)
-      const int f = a / d.E, j = a - (a / d.E) * d.E;
+      const int f = udiv31(a, d.E, d.mE), j = a - f * d.E;
       const bool special = j < d.S;
       Blk qb{0, 0, 0, 0, 0};
       if (!special) qb = block_of(d, f * d.Bf + (j - d.S));
@@ -361,9 +372,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_5d(dq, &mp.q5, bar(B_EF + es), 0, h, qb.c0, qb.r0, f);
         }
       }
-      // the key tiles: every lane arrives once on the tile's K and V barriers
-      // (count 32): through the TMA transaction count for the always-kept
-      // tiles, through cp.async completion for the gathered ones
+      // hand the token list to the gather warp (every lane arrives: release
+      // of its own writes)
+      mbar_arrive(bar(B_TF + lb));
+#pragma unroll
+      for (int u = 0; u < kMaxTopK / 32; ++u) ids_cur[u] = ids_nxt[u];
+      qs_cur = qs_nxt;
+      pair_cur = pair_nxt;
+      pair_nxt = pair_nn;
+    }
+    if (*abort_flag && lane == 0) {
+      // let this CTA's query boxes land before its shared memory goes away
+      volatile int never = 0;
+      for (int e = ne - 1; e >= 0 && e >= ne - NE; --e) mbar_wait(bar(B_EF + e % NE), (e / NE) & 1, &never, err);
+    }
+  } else if (warp == 3) {
+    // ---------------- gather warp ----------------
+    // per entry, once its token list is handed over: the key tiles into the
+    // K/V ring; every lane arrives once on the tile's K and V barriers (count
+    // 32): through the TMA transaction count for the always-kept tiles,
+    // through cp.async completion for the gathered ones
+    int gt = 0;  // tiles loaded
+    int ne = 0;  // entries taken
+    bool ok = true;
+    const long long row = (long long)d.H * kHeadDim;
+    for (long long it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++ne) {
+      const int es = ne % NE, lb = ne & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar(B_TF + lb), (ne >> 1) & 1, abort_flag, err, d.wait_cycles))) {
+        ok = false;
+        break;
+      }
+      const int* tl = reinterpret_cast<const int*>(sp + OFF_TOK) + lb * kTokList;
+      const Entry& E = ent(es);
+      const int n_tiles = E.n_tiles, n_kept = E.n_kept, n_keys = E.n_keys, h = E.h;
+      const long long hoff = (long long)h * kHeadDim;
       for (int i = 0; ok && i < n_tiles; ++i, ++gt) {
         const int s = gt % ST;
         if (gt >= ST) {
@@ -375,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         const uint32_t dk = sb + OFF_K + s * kKV, dv = sb + OFF_V + s * kKV;
-        if (i < n_kept_tiles) {
+        if (i < n_kept) {
           if (lane == 0) {
             mbar_expect_tx(bar(B_KF + s), kKV);
             mbar_expect_tx(bar(B_VF + s), kKV);
@@ -390,39 +432,30 @@ __global__ void __launch_bounds__(kThreads, 1)
           // operand tile is that token's 128 bytes, its 16-byte chunks in the
           // 128-byte swizzle.  Only the valid slots are copied: the rest keep
           // finite data (zeroed at start, or an earlier tile's rows) that the
-          // softmax masks to weight 0
-          const int g0 = (i - n_kept_tiles) * TKEYS;
-          const int nv8 = min(TKEYS, n_keys - g0) * 8;
-          const long long hoff = (long long)h * kHeadDim;
-          const long long row = (long long)d.H * kHeadDim;
+          // softmax masks to weight 0.  A lane copies chunk lane % 8 of keys
+          // lane / 8 + 4 m.
+          const int g0 = (i - n_kept) * TKEYS;
+          const int nv = min(TKEYS, n_keys - g0);
+          const int ch = lane & 7;
+          const bf16* kh = kg + hoff + ch * 8;
+          const bf16* vh = vg + hoff + ch * 8;
 #pragma unroll 4
-          for (int u = lane; u < nv8; u += 32) {
-            const int c = u >> 3, ch = u & 7;
-            cp_async16(dk + (uint32_t)(c * 128 + ((ch ^ (c & 7)) << 4)),
-                       kg + (long long)tok_list[g0 + c] * row + hoff + ch * 8, true);
-          }
+          for (int c = lane >> 3; c < nv; c += 4)
+            cp_async16(dk + (uint32_t)(c * 128 + ((ch ^ (c & 7)) << 4)), kh + (long long)tl[g0 + c] * row, true);
           cp_async_mbar_arrive_noinc(bar(B_KF + s));
 #pragma unroll 4
-          for (int u = lane; u < nv8; u += 32) {
-            const int c = u >> 3, ch = u & 7;
-            cp_async16(dv + (uint32_t)(c * 128 + ((ch ^ (c & 7)) << 4)),
-                       vg + (long long)tok_list[g0 + c] * row + hoff + ch * 8, true);
-          }
+          for (int c = lane >> 3; c < nv; c += 4)
+            cp_async16(dv + (uint32_t)(c * 128 + ((ch ^ (c & 7)) << 4)), vh + (long long)tl[g0 + c] * row, true);
           cp_async_mbar_arrive_noinc(bar(B_VF + s));
         }
       }
-      __syncwarp();  // the token list is rebuilt for the next entry
-#pragma unroll
-      for (int u = 0; u < kMaxTopK / 32; ++u) ids_cur[u] = ids_nxt[u];
-      qs_cur = qs_nxt;
-      pair_cur = pair_nxt;
-      pair_nxt = pair_nn;
+      // the token list may be rebuilt (its reads are done)
+      mbar_arrive(bar(B_TE + lb));
     }
     cp_async_wait<0>();  // this lane's gathers have landed
     if (*abort_flag && lane == 0) {
       // let this CTA's own copies land before its shared memory goes away
       volatile int never = 0;
-      for (int e = ne - 1; e >= 0 && e >= ne - NE; --e) mbar_wait(bar(B_EF + e % NE), (e / NE) & 1, &never, err);
       for (int g = gt - 1; g >= 0 && g >= gt - ST; --g) {
         mbar_wait(bar(B_KF + g % ST), (g / ST) & 1, &never, err);
         mbar_wait(bar(B_VF + g % ST), (g / ST) & 1, &never, err);

@@ -84,7 +84,7 @@ constexpr uint32_t kEntBytes = (sizeof(Entry) + 127) / 128 * 128;
 constexpr int kTokList = kMaxTopK * NQ;                  // key slots of one entry at most
 constexpr uint32_t OFF_TOK = OFF_ENT + NE * kEntBytes;   // two token lists (builder -> gather warp)
 constexpr uint32_t OFF_RED = OFF_TOK + 2 * kTokList * 4;  // [4 warps][16] per-query partial maxima
-constexpr uint32_t OFF_LS = OFF_RED + 4 * NQ * 4;        // [16] sums of P (epilogue)
+constexpr uint32_t OFF_LS = OFF_RED + 4 * NQ * 4;        // [16] reciprocal denominators (epilogue)
 constexpr uint32_t OFF_GATE = OFF_LS + NQ * 4;           // [2] gate partial dot products
 constexpr uint32_t OFF_BAR = (OFF_GATE + 16 + 255) / 256 * 256;
 constexpr uint32_t OFF_MISC = OFF_BAR + 512;
@@ -508,6 +508,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sq = sb + OFF_Q + es * kQ;
         for (int i = 0; i < n; ++i) {
           const int s = gt % ST, b = gt & 1;
+          // S^T(t+1) goes first when its keys have landed (the tensor core
+          // then works while the softmax finishes tile t); otherwise O^T(t)
+          // is issued at once, so that its entry's epilogue is not held up by
+          // the next tile's gathers
+          if (pend && !mbar_peek(bar(B_KF + s), (gt / ST) & 1) && !(ok = finish())) break;
           if (!mbar_wait(bar(B_KF + s), (gt / ST) & 1, abort_flag, err, d.wait_cycles)) {
             ok = false;
             break;
@@ -672,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q4 = warp & 3;
     const int dlane = q4 * 32 + lane;  // lanes 0-63: value dims; 64-127: sums of P
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    float* ls = reinterpret_cast<float*>(sp + OFF_LS);
+    float* ls = reinterpret_cast<float*>(sp + OFF_LS);  // [16] reciprocal denominators
     float* gz = reinterpret_cast<float*>(sp + OFF_GATE);
     const long long row = (long long)d.H * kHeadDim;
     int ne = 0;
@@ -718,9 +723,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < NQ; ++q) ov[q] = 0u;
       }
-      if (dlane == 64) {
+      if (dlane >= 64 && dlane < 64 + NQ) {
+        // rows 64-127 of O^T all hold the sums of P: thread 64 + q forms
+        // query q's denominator (the always-kept segment's weight plus the
+        // sum), its reciprocal for the value threads, and the log-sum-exp
+        const int q = dlane - 64;
+        float sq = 0.f;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) ls[q] = __uint_as_float(ov[q]);
+        for (int u = 0; u < NQ; ++u)
+          if (u == q) sq = __uint_as_float(ov[u]);
+        const float den = E.wf[q] + sq;
+        ls[q] = 1.f / den;
+        if (w == nullptr && lse != nullptr && ((qmask >> q) & 1u))
+          lse[(long long)E.tok[q] * d.H + h] = (E.mf[q] + log2f(den)) * 0.6931471805599453f;
       }
       if (w != nullptr && dlane < 64) {
         float z = zpart;
@@ -735,16 +750,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < NQ; ++q) {
           if (!((qmask >> q) & 1u)) continue;
           const long long t = E.tok[q];
-          const float wq = E.wf[q];
-          const float den = wq + ls[q];
-          const float o = fmaf(wq, osv[q], __uint_as_float(ov[q])) / den;
+          const float o = fmaf(E.wf[q], osv[q], __uint_as_float(ov[q])) * ls[q];
           const long long ob = t * row + (long long)h * kHeadDim + dlane;
-          if (w != nullptr) {
-            out[ob] = __float2bfloat16_rn(g * cmp + (1.f - g) * o);
-          } else {
-            out[ob] = __float2bfloat16_rn(o);
-            if (lse != nullptr && dlane == 0) lse[t * d.H + h] = (E.mf[q] + log2f(den)) * 0.6931471805599453f;
-          }
+          out[ob] = __float2bfloat16_rn(w != nullptr ? g * cmp + (1.f - g) * o : o);
         }
       }
       bar_sync128(2);  // ls / gz are reused by the next entry

@@ -97,16 +97,6 @@ cudaError_t launch_block_scores_topk(const Dims& d, const float* qc32, const flo
 cudaError_t launch_topk_merge(const Dims& d, const float* cand_score, const int* cand_idx,
                               int n_split, int* sel, cudaStream_t st);
 
-// Selection branch; when `w` is non-null the gate is fused and `out` receives
-// g*oc + (1-g)*o_sel, otherwise `out` receives o_sel (and lse if non-null).
-// With o_spec/lse_spec non-null the special-token segment is taken from them
-// (normalised fp32 [T][H][64] and natural-log lse [T][H]) instead of ks/vs.
-cudaError_t launch_selected(const Dims& d, const bf16* q, const bf16* k, const bf16* v,
-                            const bf16* ks, const bf16* vs, const int* sel, const float* qc32,
-                            const float* w, const float* oc, bf16* out, float* lse,
-                            const float* o_spec, const float* lse_spec, unsigned* err,
-                            cudaStream_t st);
-
 // Selection branch on tcgen05 (transposed products per compressed entry).
 // With o_spec/lse_spec the always-kept segment comes from them; otherwise,
 // when NK > 0, the kernel streams the kept keys ks/vs itself.  `order`

@@ -54,7 +54,7 @@ constexpr int ST = 2;
 constexpr int kThreads = 384;
 constexpr int kMaxK = kFusedTopK;  // heap capacity per row
 constexpr int kBuf = 32;         // candidate buffer entries per row
-constexpr int kKeep = 20;        // candidates a row may keep buffered after a flush (<= kBuf - 8)        // candidates a row may keep buffered after a flush (<= kBuf - 16)
+constexpr int kKeep = 20;        // candidates a row may keep buffered after a flush (<= kBuf - 8)
 constexpr uint32_t kSub = 128 * 128;    // one [128][32] fp32 (or [128][64] bf16) tile: 16 KB
 
 constexpr uint32_t OFF_Q = 0;                        // 2 sub-tiles (d 0-31, 32-63)

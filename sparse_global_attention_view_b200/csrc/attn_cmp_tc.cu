@@ -392,12 +392,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the single softmax warp of each sub-partition from stalling on one
       // 128-long dependency chain
       float mq[16];
+      {
+        // three-input maxima: four instructions per group of eight
+        auto e = [&](int q, int i) -> float { return __uint_as_float(sv[q >> 2][(q & 3) * 8 + i]); };
 #pragma unroll
-      for (int q = 0; q < 16; ++q) mq[q] = __uint_as_float(sv[q >> 2][(q & 3) * 8]);
-#pragma unroll
-      for (int i = 1; i < 8; ++i)
-#pragma unroll
-        for (int q = 0; q < 16; ++q) mq[q] = fmaxf(mq[q], __uint_as_float(sv[q >> 2][(q & 3) * 8 + i]));
+        for (int q = 0; q < 16; ++q)
+          mq[q] = fmaxf(fmax3(fmax3(e(q, 0), e(q, 1), e(q, 2)), fmax3(e(q, 3), e(q, 4), e(q, 5)), e(q, 6)), e(q, 7));
+      }
       {
         // tell the top-K warp which groups may hold a candidate for this row:
         // those whose maximum beats the row's K-th best so far (a stale, lower
@@ -451,21 +452,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // scaled, shifted scores two at a time (paired fp32 instructions, each
+      // half rounded as the scalar form); four paired sum chains
+      const uint64_t c2p = f2_pack(c2, c2), nmp = f2_pack(-m_used, -m_used);
+      uint64_t ps2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i]), c2, -m_used));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][2 * i + 1]), c2, -m_used));
-          ps[i & 7] += p0 + p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c][2 * i]), __uint_as_float(sv[c][2 * i + 1])), c2p, nmp), x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          ps2[i & 3] = f2_add(ps2[i & 3], f2_pack(p0, p1));
           pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(p_addr + 16 * c, pk);
       }
       tmem_wait_st();
-      l += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      {
+        float lo, hi;
+        f2_unpack(f2_add(f2_add(ps2[0], ps2[1]), f2_add(ps2[2], ps2[3])), lo, hi);
+        l += lo + hi;
+      }
       fence_before_sync();
       mbar_arrive(bar(B_PF));
     }

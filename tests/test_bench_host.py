@@ -73,3 +73,34 @@ def test_both_arms_describe_the_same_config(world, parallel):
     cfg = bench.workload_config(wl, bench.l2_note(wl, world, parallel), bench.parallelism_of(wl, world, parallel))
     assert "l2" in cfg and "L2" in cfg["l2"]
     assert cfg["parallelism"].startswith("heads" if (world > 1 and parallel == "heads") else "replicas")
+
+
+def test_recorded_traffic_follows_the_kernel_source(tmp_path, monkeypatch):
+    # DRAM bytes from the committed ncu summary count only while the kernel's
+    # source is the one they were captured from
+    import json
+    csrc = tmp_path / "sparse_global_attention_view_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = csrc / "k.cu"
+    src.write_text("__global__ void k() {}\n")
+    rec = {"k.cu@pages": {"bytes_per_launch": 123, "source_sha": bench.source_hash(str(src))}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("k.cu", "pages") == 123
+    assert bench.recorded_traffic("k.cu", "medium") is None
+    src.write_text("__global__ void k() { }\n")
+    assert bench.recorded_traffic("k.cu", "pages") is None
+
+
+def test_committed_traffic_matches_the_committed_sources():
+    # every record in profiles/traffic.json names a kernel source that exists
+    import json
+    import os
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    for key, r in rec.items():
+        f, wl = key.split("@")
+        path = os.path.join(bench.ROOT, "sparse_global_attention_view_b200", "csrc", f)
+        assert os.path.exists(path), key
+        assert r["bytes_per_launch"] == r["dram_bytes_read"] + r["dram_bytes_write"], key
+        assert f in bench.STAGE_SOURCE.values(), key

@@ -164,6 +164,22 @@ gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const
                                void* ws, void* stream);
 
 /*
+ * Debug output of steps 2-3: the fused kernel's own unscaled compressed
+ * logits, the values its streaming top-K ranks (S_guide = scale * logit;
+ * it page, section 2), for the compressed query rows [row0, row0 + n_rows):
+ *   logits [H][n_rows][Tc] fp32: tf32 tensor-core products qc32[a,h] . kc32[c,h]
+ *   for every compressed entry c (special entries included).
+ * qc32 / kc32 / vc as for gsa_compressed_attn (vc is only mapped, not read).
+ * Runs only the CTAs of the rows asked for; their ranking pass writes nothing
+ * else.  0 <= row0, n_rows >= 1, row0 + n_rows <= Tc, else GSA_ERR_INVALID_ARG.
+ * With the same inputs the values equal those gsa_forward ranks, so a test
+ * can check that its selection is the exact top-K of these logits.
+ */
+gsa_status gsa_guide_logits(const gsa_shape* shape, const float* qc32, const float* kc32,
+                            const gsa_bf16* vc, int64_t row0, int32_t n_rows, float* logits, void* ws,
+                            void* stream);
+
+/*
  * Step 4, Top-K block selection (technical summary 2.1, selection branch:
  * the K most relevant token regions per query by the compressed scores).
  * Merges the n_split candidate lists of gsa_compressed_attn into

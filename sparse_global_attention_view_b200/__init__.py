@@ -17,6 +17,7 @@ from .api import (  # noqa: F401
     forward,
     forward_noalloc,
     forward_timed,
+    guide_logits,
     frame_attn,
     sga_workspace_size,
     new_sga_workspace,

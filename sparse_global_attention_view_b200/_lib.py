@@ -82,6 +82,7 @@ SIGNATURES = {
     "gsa_pool_kv": [P_SHAPE] + [c_vp] * 12,
     "gsa_compressed_attn": [P_SHAPE] + [c_vp] * 8 + [c_i32, c_vp, c_vp],
     "gsa_topk_blocks": [P_SHAPE, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp],
+    "gsa_guide_logits": [P_SHAPE, c_vp, c_vp, c_vp, ctypes.c_int64, c_i32, c_vp, c_vp, c_vp],
     "gsa_selected_attn": [P_SHAPE] + [c_vp] * 10,
     "gsa_gate_combine": [P_SHAPE] + [c_vp] * 7,
     "dense_global_attn": [P_SHAPE] + [c_vp] * 6,

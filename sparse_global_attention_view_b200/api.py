@@ -134,6 +134,18 @@ def topk_blocks(shape, cand_score, cand_idx, n_split, sel, ws, stream=None):
         "gsa_topk_blocks")
 
 
+def guide_logits(shape, qc32, kc32, vc, row0, n_rows, logits, ws, stream=None):
+    """The fused kernel's own unscaled compressed logits for rows [row0, row0 + n_rows):
+    logits [H][n_rows][Tc] fp32 (gsa_guide_logits)."""
+    z = derive(shape)
+    n = shape.n_heads * z.Tc * shape.head_dim
+    check(load().gsa_guide_logits(
+        ctypes.byref(shape.c()), _ptr(qc32, F32, n, "qc32"), _ptr(kc32, F32, n, "kc32"),
+        _ptr(vc, BF16, n, "vc"), ctypes.c_int64(row0), ctypes.c_int32(n_rows),
+        _ptr(logits, F32, shape.n_heads * n_rows * z.Tc, "logits"), _ws(ws), _stream(stream)),
+        "gsa_guide_logits")
+
+
 def selected_attn(shape, q, k, v, ks, vs, sel, o_sel, lse=None, ws=None, stream=None):
     z = derive(shape)
     tok = z.T * shape.n_heads * shape.head_dim

@@ -48,7 +48,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int TQ = 128;
+constexpr int TQ = kCmpTileRows;
 constexpr int TK = 128;
 constexpr int ST = 2;
 constexpr int kThreads = 384;
@@ -205,6 +205,9 @@ __device__ __forceinline__ void tmem_wait_ld8(uint32_t (&r)[8]) {
                : "memory");
 }
 
+// kDump: the debug instantiation that also writes the requested rows'
+// logits (CmpPass::dump); the production one has no dump code at all.
+template <bool kDump>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_cmp_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                        const __grid_constant__ CUtensorMap tv, const Dims d, float* __restrict__ oc,
@@ -221,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
-  const long long m0 = (long long)blockIdx.x * TQ;
+  const long long m0 = (long long)(blockIdx.x + cp.tile0) * TQ;
   const long long n_k = d.Tc;
   const int nt = (int)((n_k + TK - 1) / TK);
 
@@ -375,6 +378,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t s_addr = tbase + lane_off + b * 128;
       const uint32_t p_addr = tbase + lane_off + 448;
       const long long rem = n_k - (long long)j * TK;
+      if constexpr (kDump) {
+        // debug: this row's unscaled logits of the tile, as ranked, re-read
+        // from TMEM 16 columns at a time (a short loop, off the hot path)
+        const long long row = m0 + r;
+        const bool mine = row >= cp.dump_row0 && row < cp.dump_row0 + cp.dump_rows && row < d.Tc;
+        float* o = cp.dump + ((long long)h * cp.dump_rows + (row - cp.dump_row0)) * n_k + (long long)j * TK;
+#pragma unroll 1
+        for (int c = 0; c < 8; ++c) {
+          uint32_t t[16];
+          tmem_ld16(s_addr + 16 * c, t);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            if (mine && 16 * c + i < rem) o[16 * c + i] = __uint_as_float(t[i]);
+        }
+      }
       // all 128 scores in one round of TMEM loads: the softmax is bound by
       // TMEM load latency, so a second round would cost as much as the first
       uint32_t sv[4][32];
@@ -388,8 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 32; ++i)
             if (32 * c + i >= rem) sv[c][i] = __float_as_uint(-CUDART_INF_F);
       }
-      // the maxima of the eight 16-column groups: eight independent chains keep
-      // the single softmax warp of each sub-partition from stalling on one
+      // the maxima of the sixteen 8-column groups: sixteen independent chains
+      // keep the single softmax warp of each sub-partition from stalling on one
       // 128-long dependency chain
       float mq[16];
       {
@@ -679,16 +698,17 @@ cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* 
             make_tmap_3d(&mk, true, kc32, 64, H, Tc, 256, H * 256, 32, 1, 128) &&
             make_tmap_3d(&mv, false, vc, 64, H, Tc, 128, H * 128, 64, 1, 128);
   if (!ok) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(attn_cmp_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kSmemBytes);
+  auto kernel = cp.dump != nullptr ? attn_cmp_tc_kernel<true> : attn_cmp_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, attn_cmp_tc_kernel);
+  e = cudaFuncGetAttributes(&fa, kernel);
   if (e != cudaSuccess) return e;
   if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-  dim3 grid((unsigned)((d.Tc + TQ - 1) / TQ), (unsigned)d.H);
-  attn_cmp_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, d, oc, cand_score, cand_idx, sel,
-                                                         err, cp);
+  const long long all_tiles = (d.Tc + TQ - 1) / TQ;
+  if (cp.tile0 < 0 || cp.tiles < 0 || cp.tile0 + cp.tiles > all_tiles) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)(cp.tiles > 0 ? cp.tiles : all_tiles - cp.tile0), (unsigned)d.H);
+  kernel<<<grid, kThreads, kSmemBytes, st>>>(mq, mk, mv, d, oc, cand_score, cand_idx, sel, err, cp);
   return cudaGetLastError();
 }
 

@@ -250,6 +250,29 @@ gsa_status gsa_compressed_attn(const gsa_shape* shape, const gsa_bf16* qc, const
   return cuda_status(gsa::launch_block_scores_topk(d, qc32, kc32, cand_score, cand_idx, n_split, s));
 }
 
+gsa_status gsa_guide_logits(const gsa_shape* shape, const float* qc32, const float* kc32,
+                            const gsa_bf16* vc, int64_t row0, int32_t n_rows, float* logits, void* ws,
+                            void* stream) {
+  Dims d;
+  gsa_status st = make_dims(shape, &d, nullptr);
+  if (st != GSA_OK) return st;
+  if (!dev_ptr(qc32) || !dev_ptr(kc32) || !dev_ptr(vc) || !dev_ptr(logits) || !dev_ptr(ws))
+    return GSA_ERR_INVALID_ARG;
+  if (row0 < 0 || n_rows < 1 || row0 + n_rows > d.Tc) return GSA_ERR_INVALID_ARG;
+  // the fused kernel ranks alongside (its lists are not written); its heaps
+  // hold at most kFusedTopK pairs
+  if (d.K > gsa::kFusedTopK) d.K = gsa::kFusedTopK;
+  gsa::CmpPass cp;
+  cp.scores_only = 1;
+  cp.dump = logits;
+  cp.dump_row0 = row0;
+  cp.dump_rows = n_rows;
+  cp.tile0 = (int)(row0 / gsa::kCmpTileRows);
+  cp.tiles = (int)((row0 + n_rows - 1) / gsa::kCmpTileRows) - cp.tile0 + 1;
+  return cuda_status(gsa::launch_compressed_tc(d, qc32, kc32, (const bf16*)vc, nullptr, nullptr, nullptr,
+                                               nullptr, (unsigned*)ws, as_stream(stream), cp));
+}
+
 gsa_status gsa_topk_blocks(const gsa_shape* shape, const float* cand_score,
                            const int32_t* cand_idx, int32_t n_split, int32_t* sel, void* ws,
                            void* stream) {

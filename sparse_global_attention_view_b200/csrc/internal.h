@@ -80,9 +80,17 @@ struct CmpPass {
   unsigned long long* root = nullptr;
   int scores_only = 0;
   int* best = nullptr;  // nullable [H][Tc]: each row's best-scoring block id (-1 if none)
+  // Debug dump of the kernel's own unscaled logits qc32 . kc32 (tf32 products)
+  // for rows [dump_row0, dump_row0 + dump_rows): dump[h][row - dump_row0][Tc].
+  float* dump = nullptr;
+  long long dump_row0 = 0;
+  int dump_rows = 0;
+  // Query tiles of the grid: tiles [tile0, tile0 + tiles) (tiles = 0: all).
+  int tile0 = 0, tiles = 0;
 };
 bool compressed_tc_supported(const Dims& d);
 constexpr int kFusedTopK = 64;  // heap capacity of one pass of the fused kernel
+constexpr int kCmpTileRows = 128;  // compressed-query rows per CTA of the fused kernel
 cudaError_t launch_compressed_tc(const Dims& d, const float* qc32, const float* kc32, const bf16* vc,
                                  float* oc, float* cand_score, int* cand_idx, int* sel, unsigned* err,
                                  cudaStream_t st, const CmpPass& cp = CmpPass());

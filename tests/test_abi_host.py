@@ -135,6 +135,9 @@ def test_null_and_misaligned_pointers_are_rejected(lib):
     assert lib.gsa_workspace_init(bad, st) == 1
     assert lib.gsa_derive(None, None) == 1
     assert lib.gsa_selftest_exp2(null, p, 4, st) == 1
+    assert lib.gsa_guide_logits(ctypes.byref(s), p, p, p, -1, 4, p, p, st) == 1
+    assert lib.gsa_guide_logits(ctypes.byref(s), p, p, p, 0, 0, p, p, st) == 1
+    assert lib.gsa_guide_logits(ctypes.byref(s), p, null, p, 0, 4, p, p, st) == 1
     assert lib.gsa_selftest_exp2(p, p, -1, st) == 1
     assert lib.frame_attn(ctypes.byref(s), p, p, bad, p, p, st) == 1
     assert lib.sga_attn(ctypes.byref(s), 2, 2, p, p, p, null, p, ctypes.c_size_t(1 << 40), st) == 1

@@ -475,3 +475,49 @@ def test_softmax_fma_exp2_error_bound():
     G.selftest_exp2(xd[:3].contiguous(), y3)
     torch.cuda.synchronize()
     assert torch.equal(y3, y[:3])
+
+
+@pytest.mark.parametrize("name", ["small", "p3_ragged", "p1_nospecial", "p2_onehead", "one_frame", "ref_small",
+                                  "ref_p3_ragged"])
+def test_selection_is_the_exact_top_k_of_the_kernels_own_logits(name):
+    # gsa_guide_logits dumps the logits the fused kernel ranks (tf32 products
+    # of the fp32 means).  They must lie within tf32 rounding of the exact
+    # products, and the kernel's selection must be exactly the top-K of them
+    # (score descending, lower id on ties): no tie window is needed here.
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case(name)
+    if shape.top_k > 64:
+        pytest.skip("two ranking passes")
+    z = G.derive(shape)
+    logits = torch.full((shape.n_heads, z.Tc, z.Tc), float("nan"), device="cuda")
+    G.guide_logits(shape, st.qc32, st.kc32, st.vc, 0, z.Tc, logits, st.ws)
+    torch.cuda.synchronize()
+    G.check_device_error(st.ws)
+    lg = logits.permute(1, 0, 2).double().cpu().numpy()  # [Tc, H, Tc]
+    assert np.isfinite(lg).all()
+    q64 = st.qc32.double().cpu()
+    k64 = st.kc32.double().cpu()
+    exact = torch.einsum("ahd,chd->ahc", q64, k64).numpy()
+    mag = torch.einsum("ahd,chd->ahc", q64.abs(), k64.abs()).numpy()
+    # tf32 keeps 10 explicit mantissa bits of each operand: below 2^-10
+    # relative per factor even if truncated, so below 2^-9 per product, plus
+    # the fp32 accumulation over 64 terms
+    assert (np.abs(lg - exact) <= 2.0 ** -8 * mag + 1e-6).all(), f"{name}: logits beyond tf32 rounding"
+    own = O.top_k_blocks(geo, O.guide_scores(geo, lg))
+    assert np.array_equal(st.sel_by_entry(), own), f"{name}: selection is not the top-K of the kernel's logits"
+    # a row range runs only its CTAs and gives the same values
+    if z.Tc > 140:
+        part = torch.full((shape.n_heads, 9, z.Tc), float("nan"), device="cuda")
+        G.guide_logits(shape, st.qc32, st.kc32, st.vc, 131, 9, part, st.ws)
+        torch.cuda.synchronize()
+        assert torch.equal(part, logits[:, 131:140]), f"{name}: row range differs"
+
+
+def test_guide_logits_rejects_bad_row_ranges():
+    import sparse_global_attention_view_b200 as G
+    x, geo, shape, st, res = case("small")
+    z = G.derive(shape)
+    for row0, n in ((-1, 4), (0, 0), (z.Tc - 3, 4)):
+        out = torch.empty((shape.n_heads, n, z.Tc), device="cuda")
+        with pytest.raises(G.GsaError):
+            G.guide_logits(shape, st.qc32, st.kc32, st.vc, row0, n, out, st.ws)

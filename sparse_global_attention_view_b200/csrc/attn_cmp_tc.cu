@@ -19,25 +19,28 @@
 // the tile before is complete), so the raw scores stay readable until the
 // top-K warpgroup is done with them; with three score buffers the top-K
 // warpgroup may trail the softmax by a tile without stalling the tensor core.
-// The softmax already forms the maxima of the tile's eight 16-column groups;
+// The softmax already forms the maxima of the tile's sixteen 8-column groups;
 // it compares them with each row's current K-th best score (published in
-// shared memory by the top-K thread) and hands the top-K warp an 8-bit mask
+// shared memory by the top-K thread) and hands the top-K warp a 16-bit mask
 // of the groups that may hold a candidate.  The top-K warp reads from TMEM
 // only the groups flagged for any of its 32 rows and releases the score
 // buffer after its last read.  Candidates (columns that beat the row's K-th
 // best) go to a per-row buffer in shared memory without branches (every
 // column is written to the next free slot, which is kept only for a
-// candidate); when any row's buffer is half full the warp inserts all
-// buffered candidates in lockstep (one round of insertions serves every row)
-// into the rows' heaps of K best (score, block id) pairs; special entries are
-// never ranked.  Once every heap of the warp is full, a round is one
+// candidate); when a row's buffer could not take the next group, the warp
+// inserts buffered candidates in lockstep (one round of insertions serves
+// every row, each row taking its newest) into the rows' heaps of K best
+// (score, block id) pairs until no row holds more than kKeep; special entries
+// are never ranked.  Once every heap of the warp is full, a round is one
 // predicated three-level replacement of the root per lane (lanes without a
 // candidate walk it without moving), with the next round's candidate loaded
-// during the current one: no lane diverges.  Columns arrive in ascending
-// block order and only a strictly larger score displaces the root, so equal
-// scores keep the lower id.  The softmax keeps eight
-// independent max and sum chains: one warp per sub-partition runs it, so
-// dependency latency, not throughput, is what it must avoid.
+// during the current one: no lane diverges.  Only a strictly larger key
+// displaces the root, and a key orders by score, then by the lower id, so
+// the heaps hold the K largest keys whatever the order of insertion.  The
+// softmax keeps independent max and sum chains (three-input maxima, paired
+// fp32 arithmetic): one warp per sub-partition runs it and shares the
+// sub-partition's issue slots with a top-K warp.  A second instantiation
+// (kDump) also writes the logits of requested rows for debugging.
 #include <math_constants.h>
 
 #include "internal.h"
@@ -107,7 +110,8 @@ __device__ __forceinline__ unsigned long long pair_key(float s, int id) {
 struct Heap {
   unsigned long long* hk;
   int r, K, cnt;
-  float tau;  // score a candidate must beat (-inf until the heap is full)
+  float tau;  // score of the worst pair kept (-inf until the heap is full)
+  unsigned long long rootkey;  // key of the worst pair kept (0 until the heap is full)
 
   __device__ __forceinline__ unsigned long long at(int i) const { return hk[i * TQ + r]; }
   __device__ __forceinline__ void put(int i, unsigned long long k) { hk[i * TQ + r] = k; }
@@ -159,6 +163,7 @@ struct Heap {
     }
     if (take) {
       put(p, key);
+      rootkey = root;
       tau = order_value((uint32_t)(root >> 32));
     }
   }
@@ -167,7 +172,8 @@ struct Heap {
       put(cnt, key);
       if (++cnt == K) {
         for (int p = (K - 2) / 4; p >= 0; --p) sift(p, at(p));
-        tau = order_value((uint32_t)(at(0) >> 32));
+        rootkey = at(0);
+        tau = order_value((uint32_t)(rootkey >> 32));
       }
       return;
     }
@@ -425,7 +431,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float tau = tau_s[r];
         uint32_t msk = 0;
 #pragma unroll
-        for (int q = 0; q < 16; ++q) msk |= (mq[q] > tau ? 1u : 0u) << q;
+        for (int q = 0; q < 16; ++q) msk |= (mq[q] >= tau ? 1u : 0u) << q;
+        if (m0 + r >= d.Tc) msk = 0u;  // rows past the sequence never rank
         mask_s[b * TQ + r] = (uint16_t)msk;
         mbar_arrive(bar(B_MR + b));
       }
@@ -524,10 +531,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     float* cb_s = reinterpret_cast<float*>(sp + OFF_CS);
     int* cb_e = reinterpret_cast<int*>(sp + OFF_CC);
-    Heap top{reinterpret_cast<unsigned long long*>(sp + OFF_HS), r, d.K, 0, -CUDART_INF_F};
+    Heap top{reinterpret_cast<unsigned long long*>(sp + OFF_HS), r, d.K, 0, -CUDART_INF_F, 0ull};
     const int E = d.E, S = d.S, Bf = d.Bf, B0 = (int)d.B0;
     const int ntok = (int)n_k;
     const long long my_row = m0 + r;
+    // rows past the sequence (zero-filled queries, all scores equal) never rank
+    const bool row_in = my_row < d.Tc;
     // a second ranking pass keeps only pairs strictly below the first pass's
     // K-th best (score, id) key of the row
     const unsigned long long ub =
@@ -546,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i >= E) i -= E, ++f;
     };
     auto flush = [&](int keep) {
-      if (__all_sync(0xffffffffu, top.cnt == d.K)) {
+      if (__all_sync(0xffffffffu, !row_in || top.cnt == d.K)) {
         // every heap of the warp is full: one predicated replacement per
         // round, each row taking its newest candidate, until no row holds
         // more than `keep` (the order of insertion does not change the K
@@ -567,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           decode(e, f, i);
           const int id = f * Bf + (i - S);
           const unsigned long long key = pair_key(v, id);
-          const bool take = have && v > top.tau && i >= S && id >= B0 && key < ub;
+          const bool take = have && key > top.rootkey && i >= S && id >= B0 && key < ub;
           top.replace_root(key, take);
         }
         tau_s[r] = top.tau;
@@ -575,14 +584,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int n = 0; n < nb; ++n) {
         const float v = cb_s[n * TQ + r];
-        if (!(v > top.tau)) continue;
+        if (v < top.tau) continue;
         int f, i;
         decode(cb_e[n * TQ + r], f, i);
         // special entries are never ranked, nor blocks below B0 (frame 0 when
-        // it is kept whole)
+        // it is kept whole); once the heap is full only a larger key enters
         if (i >= S && f * Bf + (i - S) >= B0) {
           const unsigned long long key = pair_key(v, f * Bf + (i - S));
-          if (key < ub) top.push(key);
+          if (key < ub && (top.cnt < top.K || key > top.rootkey)) top.push(key);
         }
       }
       nb = 0;
@@ -602,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const float v = __uint_as_float(g[i]);
-        const bool c = v > tau && i < n_in;
+        const bool c = row_in && v >= tau && i < n_in;
         ps[0] = v;
         ps[kCandGap] = __int_as_float(cbase + i);
         ps += c ? TQ : 0;

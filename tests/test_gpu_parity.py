@@ -521,3 +521,38 @@ def test_guide_logits_rejects_bad_row_ranges():
         out = torch.empty((shape.n_heads, n, z.Tc), device="cuda")
         with pytest.raises(G.GsaError):
             G.guide_logits(shape, st.qc32, st.kc32, st.vc, row0, n, out, st.ws)
+
+
+def test_exact_ties_go_to_the_lower_block_id():
+    # every frame a copy of frame 0: the blocks at one grid position in the
+    # six frames have identical pooled keys, so each query's scores tie exactly
+    # in groups of six and the K-th place falls inside a tie; the fused
+    # kernel must keep the lower block ids of a tie, as the oracle's ranking
+    # by (score descending, id ascending) does
+    import sparse_global_attention_view_b200 as G
+    wl = Workload("ties", 6, 2, 9, 10, 2, 64, 3, 7, 21, "gaussian")
+    x = generate(wl)
+    L = wl.n_special + wl.hp * wl.wp
+    for t in (x.q, x.k, x.v):
+        f = t.view(wl.n_frames, L, wl.n_heads, wl.head_dim)
+        f[1:] = f[0]
+    geo = O.geometry_of(wl)
+    shape = G.Shape.of(wl)
+    q, k, v, w = _dev(x)
+    st = PT.Stages(shape, q, k, v, w, 1).run()
+    z = G.derive(shape)
+    logits = torch.full((shape.n_heads, z.Tc, z.Tc), float("nan"), device="cuda")
+    G.guide_logits(shape, st.qc32, st.kc32, st.vc, 0, z.Tc, logits, st.ws)
+    torch.cuda.synchronize()
+    G.check_device_error(st.ws)
+    guide = O.guide_scores(geo, logits.permute(1, 0, 2).double().cpu().numpy())
+    srt = -np.sort(-guide, axis=-1)
+    assert (srt[..., geo.K_eff - 1] == srt[..., geo.K_eff]).mean() > 0.5, "the K-th place should fall in a tie"
+    own = O.top_k_blocks(geo, guide)
+    assert np.array_equal(st.sel_by_entry(), own), "ties must go to the lower block id"
+    # the whole layer's selection (gsa_forward) as well
+    layer = G.GsaLayer(shape)
+    layer(q, k, v, w)
+    torch.cuda.synchronize()
+    fwd = G.workspace_view(layer.ws, shape, "sel").permute(1, 0, 2).cpu().numpy()
+    assert np.array_equal(fwd, own)

@@ -16,8 +16,8 @@
 // or 1 of its 16 patches, and those are the blocks S_guide tends to rank
 // first: their means keep more of the tokens' noise, so their scores spread
 // wider), so a pair needs ceil(valid tokens / 128) tiles rather than K / 8.
-// The producer gathers each slot's 128 bytes with cp.async straight into the
-// 128-byte-swizzled operand layout; the entry's queries are one TMA box of
+// The gather warp copies each slot's 128 bytes with cp.async straight into
+// the 128-byte-swizzled operand layout; the entry's queries are one TMA box of
 // 4 x 4 patches over a per-frame view of the token grid.
 //
 // One CTA per SM works through (head, entry) pairs; 12 warps:
@@ -29,14 +29,16 @@
 //               ring; when the always-kept tokens are not supplied as a
 //               finished softmax state, their head-major copies are streamed
 //               first as plain 128-key TMA tiles;
-//   warp 1      MMA issuer (one thread): S^T(t+1) is issued before O^T(t), so
-//               the tensor core works while the softmax handles a tile;
+//   warp 1      MMA issuer (one thread): S^T(t+1) is issued before O^T(t)
+//               when tile t+1's keys have landed, so the tensor core works
+//               while the softmax handles a tile; otherwise O^T(t) goes first,
+//               so that an entry's epilogue never waits for the next gathers;
 //   warp 2      TMEM allocation (S^T at columns 0/16, O^T at 32 + 16 e for
 //               the four entry slots e);
 //   warps 4-7   softmax, one thread per key lane (16 queries per thread);
-//   warps 8-11  epilogue of the previous entry (normalise, merge with the
-//               always-kept segment, gate, store) while the softmax works on
-//               the next one.
+//   warps 8-11  epilogue of the previous entry (merge with the always-kept
+//               segment, one reciprocal denominator per query, gate, store)
+//               while the softmax works on the next one.
 // The softmax shifts every query by a fixed reference: the always-kept
 // segment's log-sum-exp when it is supplied (so that segment's normalised
 // output enters with weight 1), else the first tile's maximum.  A tile whose
